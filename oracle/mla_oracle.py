@@ -1,0 +1,226 @@
+"""Float64 CPU oracle for paged FP8-KV MLA decode.
+
+TEST INFRASTRUCTURE ONLY.  Nothing in the product path imports, calls or links
+this module: only tests/, __graft_entry__.smoke() and bench.py's cpu_baseline /
+reference leg use it.  It shares no code with the CUDA path.
+
+What it computes, step by step, in the order the pages lay out the data:
+
+1. Page-table gather ("generic_get_paged_cache_with_scales", Args: blocks,
+   cache_lengths, lookup_table, scales, scales_lookup_table).  Logical token t
+   of request b lives in physical block lookup_table[b, t // page_size], slot
+   t % page_size, of the 6-D blocks tensor at [blk, 0, layer_idx, slot, 0, :].
+   Its scale lives at the same slot of the 6-D scales tensor, in block
+   scales_lookup_table[b, t // page_size] when that table is given, else in
+   the value block id (the page says the shared id is right only while both
+   pools share one id space).  kv_dim index 0 is the latent ("k cache").
+2. Per-token dequantisation ("KVCacheScalesMHAOperand", description: MLA k_s
+   per-token scales, quantization_granularity = head_size):
+   K[t, d] = bf16_rn( f32_rn( e4m3(code[t, d]) * scale[t] ) ).
+   The e4m3 value is decoded from its bit fields (OCP FP8 E4M3: bias 7, no
+   infinities, S.1111.111 = NaN, subnormals m * 2^-9).
+3. Attention (the textbook definition; the pages give no formula):
+   x[t] = f32(softmax_scale) * sum_d q[d] K[t, d]   over keys t the query sees,
+   lse = log(sum_t exp(x[t]))  (natural log),  w[t] = exp(x[t] - lse),
+   out[v] = sum_t w[t] V[t, v]   with V[t, :] = K[t, :512].
+   Keys per request: n_b = cache_lengths[b] + max_prompt_length (the step's
+   new tokens are already in the cache); query i of request b sees keys
+   t <= cache_lengths[b] + i (causal among the new tokens).
+
+Everything after the e4m3 decode is float64 (the dequantised bf16 values are
+exact in float64).  Points the pages leave open and the reading taken here:
+cache_lengths count only tokens cached before this step (R1); query i sees
+keys t <= L_b + i (R2); the dequant rounds twice, product to fp32 then to
+bf16, both to nearest even, no flush to zero (R3); e4m3 is the OCP "fn"
+encoding (R4); lse is the natural log (R5); the scales tensor is the 6-D one
+and the page's 4-D shape is its (kv_dim 0, layer) slice (R7); kv_dim index 0
+is read (R8); slots past n_b and unused table entries are never read (R9).
+"""
+from __future__ import annotations
+
+import numpy as np
+
+HEAD_DIM = 576
+V_DIM = 512
+INVALID_PAGE = 0xFFFFFFFF
+
+
+# ----------------------------------------------------------------------------
+# number formats
+# ----------------------------------------------------------------------------
+def e4m3_decode(codes) -> np.ndarray:
+    """Value of each e4m3 byte (OCP E4M3, 'fn' flavour) as float64.
+
+    sign s = bit 7, exponent field e = bits 6..3 (bias 7), mantissa m = bits 2..0.
+    e == 0: subnormal (-1)^s * 2^-6 * m/8;  e == 15 and m == 7: NaN;
+    otherwise (-1)^s * 2^(e-7) * (1 + m/8).
+    """
+    c = np.asarray(codes, dtype=np.uint8).astype(np.int64)
+    s = (c >> 7) & 1
+    e = (c >> 3) & 0xF
+    m = c & 0x7
+    sign = np.where(s == 1, -1.0, 1.0)
+    normal = sign * np.ldexp(1.0 + m / 8.0, (e - 7).astype(np.int64))
+    sub = sign * np.ldexp(m / 8.0, -6)
+    v = np.where(e == 0, sub, normal)
+    v = np.where((e == 15) & (m == 7), np.nan, v)
+    return v.astype(np.float64)
+
+
+def f32_bits(x) -> np.ndarray:
+    return np.asarray(x, dtype=np.float32).view(np.uint32)
+
+
+def bf16_round_f32(x) -> np.ndarray:
+    """Round float32 values to bfloat16 with round-to-nearest-even; returns float64.
+
+    Works on the bit pattern: add 0x7FFF plus the lowest kept bit, then drop the
+    low 16 bits.  NaN stays NaN; overflow past the largest bf16 becomes inf, as
+    in IEEE rounding.
+    """
+    f = np.asarray(x, dtype=np.float32)
+    u = f.view(np.uint32).astype(np.uint64)
+    r = ((u + 0x7FFF + ((u >> 16) & 1)) >> 16) & 0xFFFF
+    with np.errstate(invalid="ignore"):
+        out = (r.astype(np.uint32) << 16).view(np.float32).astype(np.float64)
+    return np.where(np.isnan(f), np.nan, out)
+
+
+def bf16_bits_to_f64(bits) -> np.ndarray:
+    """float64 value of bf16 numbers given as uint16 bit patterns."""
+    b = np.asarray(bits, dtype=np.uint16).astype(np.uint32) << 16
+    return b.view(np.float32).astype(np.float64)
+
+
+def dequant_rows(codes, scale) -> np.ndarray:
+    """bf16_rn(f32_rn(e4m3(code) * scale)) for a [n, d] code block and [n] or [n, g] scales.
+
+    The product of an e4m3 value (4 significant bits) and an fp32 scale (24
+    bits) is exact in float64, so rounding it to float32 here is the single
+    fp32 rounding of the product; the second rounding is to bf16 (reading R3).
+    With g > 1 scales per row, dim d uses scale d // (d_total // g).
+    """
+    v = e4m3_decode(codes)
+    s = np.asarray(scale, dtype=np.float32).astype(np.float64)
+    if s.ndim == v.ndim - 1:
+        s = s[..., None]
+    if s.shape[-1] != 1 and s.shape[-1] != v.shape[-1]:
+        g = s.shape[-1]
+        s = np.repeat(s, v.shape[-1] // g, axis=-1)
+    prod = v * s
+    with np.errstate(over="ignore", invalid="ignore"):
+        p32 = prod.astype(np.float32)
+    return bf16_round_f32(p32)
+
+
+# ----------------------------------------------------------------------------
+# page-table gather
+# ----------------------------------------------------------------------------
+def num_keys(cache_lengths, max_prompt_length) -> np.ndarray:
+    """Keys stored for each request this step: n_b = L_b + T (reading R1)."""
+    return np.asarray(cache_lengths, dtype=np.int64) + int(max_prompt_length)
+
+
+def gather_request(blocks, scales, lookup_table, scales_lookup_table, b, n, layer_idx):
+    """Codes [n, D] and scales [n, g] of the first n logical tokens of request b."""
+    blocks = np.asarray(blocks)
+    scales = np.asarray(scales)
+    P = blocks.shape[3]
+    lut = np.asarray(lookup_table).astype(np.int64) & 0xFFFFFFFF
+    slut = None if scales_lookup_table is None else (np.asarray(scales_lookup_table).astype(np.int64) & 0xFFFFFFFF)
+    t = np.arange(n, dtype=np.int64)
+    page = t // P
+    slot = t % P
+    blk = lut[b, page]
+    sblk = blk if slut is None else slut[b, page]
+    if n and (blk.max() >= blocks.shape[0] or sblk.max() >= scales.shape[0]):
+        raise IndexError("page id outside the block pool")
+    codes = blocks[blk, 0, layer_idx, slot, 0, :]
+    sc = scales[sblk, 0, layer_idx, slot, 0, :]
+    return codes, sc
+
+
+def dequant_request(blocks, scales, lookup_table, scales_lookup_table, b, n, layer_idx):
+    codes, sc = gather_request(blocks, scales, lookup_table, scales_lookup_table, b, n, layer_idx)
+    return dequant_rows(codes, sc)
+
+
+# ----------------------------------------------------------------------------
+# attention
+# ----------------------------------------------------------------------------
+def attend(q, K, softmax_scale, return_weights=False):
+    """Softmax attention of queries q [H, D] over keys K [n, D], V = K[:, :512].
+
+    Returns out [H, 512] and natural-log lse [H] (and weights [H, n]).
+    """
+    q = np.asarray(q, dtype=np.float64)
+    s = float(np.float32(softmax_scale))
+    x = s * (q @ K.T)                                  # [H, n]
+    mx = x.max(axis=1, keepdims=True)
+    e = np.exp(x - mx)
+    tot = e.sum(axis=1, keepdims=True)
+    lse = (mx + np.log(tot))[:, 0]
+    w = np.exp(x - lse[:, None])
+    out = w @ K[:, :V_DIM]
+    if return_weights:
+        return out, lse, w
+    return out, lse
+
+
+def decode(q, blocks, scales, cache_lengths, lookup_table, scales_lookup_table,
+           max_prompt_length, layer_idx, softmax_scale, requests=None, heads=None,
+           return_weights=False):
+    """Full decode: out [B, T, H, 512] float64, lse [B, T, H] float64.
+
+    `requests` / `heads` restrict the work to a subset (rows not computed are NaN).
+    q: [B, T, H, 576] float values (bf16-exact), or uint16 bf16 bit patterns.
+    """
+    q = np.asarray(q)
+    if q.dtype == np.uint16:
+        q = bf16_bits_to_f64(q)
+    q = q.astype(np.float64)
+    B, T, H, D = q.shape
+    assert D == HEAD_DIM
+    T = int(max_prompt_length)
+    L = np.asarray(cache_lengths).astype(np.int64) & 0xFFFFFFFF
+    n_all = num_keys(L, T)
+    out = np.full((B, T, H, V_DIM), np.nan)
+    lse = np.full((B, T, H), np.nan)
+    weights = {}
+    reqs = range(B) if requests is None else requests
+    hs = np.arange(H) if heads is None else np.asarray(heads)
+    for b in reqs:
+        K = dequant_request(blocks, scales, lookup_table, scales_lookup_table, b, int(n_all[b]), layer_idx)
+        for i in range(T):
+            vis = int(L[b]) + i + 1                    # query i sees keys t <= L_b + i (R2)
+            r = attend(q[b, i, hs], K[:vis], softmax_scale, return_weights)
+            out[b, i, hs] = r[0]
+            lse[b, i, hs] = r[1]
+            if return_weights:
+                weights[(b, i)] = r[2]
+    if return_weights:
+        return out, lse, weights
+    return out, lse
+
+
+# ----------------------------------------------------------------------------
+# split-KV combine (used to pin that any split of the keys reaches the same result)
+# ----------------------------------------------------------------------------
+def attend_partial(q, K, softmax_scale, t0, t1):
+    """Normalised partial result over keys [t0, t1): (out_s [H, 512], lse_s [H]); empty -> lse -inf."""
+    if t1 <= t0:
+        H = np.asarray(q).shape[0]
+        return np.zeros((H, V_DIM)), np.full(H, -np.inf)
+    return attend(q, K[t0:t1], softmax_scale)
+
+
+def combine(parts):
+    """LSE-weighted merge of partial results: lse = log sum_s e^{lse_s}, out = sum_s e^{lse_s - lse} out_s."""
+    lses = np.stack([p[1] for p in parts])            # [S, H]
+    outs = np.stack([p[0] for p in parts])            # [S, H, 512]
+    mx = lses.max(axis=0)
+    w = np.exp(lses - mx)
+    tot = w.sum(axis=0)
+    lse = mx + np.log(tot)
+    out = (w[..., None] * outs).sum(axis=0) / tot[:, None]
+    return out, lse
