@@ -1,0 +1,356 @@
+#!/usr/bin/env python
+"""Benchmark of the paged FP8-KV MLA decode on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--config I] [--impl ours|reference]
+
+One step = one mla_decode_paged_fp8 call over the whole batch of the workload
+(plan + decode + split-KV combine kernels).  Inputs are seeded synthetic data
+resident in HBM; the L2 is flushed (a write larger than L2) before every timed
+step and the flush is outside the timed interval.  Prints one JSON line.
+
+Metric: KV+scale HBM GB/s (each visible key's 576 e4m3 bytes + 4-byte scale,
+read once) and decode tokens/s (batch * q_len / step time).  Under torchrun every
+rank runs its own batch (weak scaling, no collective on the data path); time is
+the max over ranks.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import subprocess
+import sys
+import tempfile
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import torch  # noqa: E402
+
+METRIC = "KV+scale HBM GB/s (% of B200 peak) and decode tokens/s for paged FP8 MLA"
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0}
+
+
+def parse():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--config", type=int, default=1)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--cpu-seconds", type=float, default=12.0, help="budget of the oracle CPU baseline")
+    return ap.parse_args()
+
+
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        return {"hbm_gbs": float(d["hbm_gbs"]), "bf16_tflops": float(d["bf16_tflops"]),
+                "bf16_tflops_sustained": float(d.get("bf16_tflops_sustained", d["bf16_tflops"])),
+                "source": "measured"}
+    return dict(FALLBACK_PEAKS, bf16_tflops_sustained=1400.0, source="fallback")
+
+
+def kernel_source_sha():
+    h = hashlib.sha256()
+    for f in ("ptx.cuh", "mla_kernels.cuh", "mla_api.cu"):
+        with open(os.path.join(ROOT, "paged_fp8_kv_mla_b200", "csrc", f), "rb") as fh:
+            h.update(fh.read())
+    return h.hexdigest()[:16]
+
+
+def recorded_traffic(config_name):
+    """DRAM bytes per decode-kernel launch from a committed ncu capture, if it matches this source."""
+    p = os.path.join(ROOT, "profiles", "decode_kernel_traffic.json")
+    if not os.path.exists(p):
+        return None
+    with open(p) as f:
+        d = json.load(f)
+    if d.get("source_sha") != kernel_source_sha():
+        return None
+    e = d.get("workloads", {}).get(config_name)
+    return None if e is None else e.get("dram_bytes_per_launch")
+
+
+class ClockSampler:
+    """nvidia-smi samples of SM clock and throttle reasons while the timed region runs."""
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index):
+        self.idx = gpu_index
+        self.proc = None
+        self.path = None
+
+    def start(self):
+        try:
+            fd, self.path = tempfile.mkstemp(suffix=".csv")
+            os.close(fd)
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits", "-lms", "50",
+                 "-i", str(self.idx), "-f", self.path], stdout=subprocess.DEVNULL, stderr=subprocess.DEVNULL)
+            time.sleep(0.3)
+        except Exception:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        time.sleep(0.1)
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except Exception:
+            self.proc.kill()
+        rows = []
+        try:
+            with open(self.path) as f:
+                for line in f:
+                    parts = [x.strip() for x in line.split(",")]
+                    if len(parts) >= 9 and parts[1].replace(".", "").isdigit():
+                        rows.append(parts)
+            os.unlink(self.path)
+        except Exception:
+            return None
+        if not rows:
+            return None
+        sm = sorted(float(r[1]) for r in rows)
+        mx = max(float(r[2]) for r in rows)
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for r in rows for i in range(4) if r[5 + i].lower() == "active"})
+        return {"sm_mhz": sm[len(sm) // 2], "sm_max_mhz": mx, "reasons": reasons, "samples": len(rows)}
+
+
+def cpu_oracle_baseline(inp, budget_s, rank_requests=None):
+    """The float64 oracle, as it stands, on whole requests of the same workload until ~budget_s."""
+    import numpy as np
+    from oracle import mla_oracle as O
+    from tests.oracle_io import to_numpy
+    try:
+        from threadpoolctl import threadpool_info
+        threads = max([t.get("num_threads", 1) for t in threadpool_info()] or [1])
+    except Exception:
+        threads = None
+    a = to_numpy(inp)
+    n = O.num_keys(a["cache_lengths"], a["max_prompt_length"])
+    order = rank_requests if rank_requests is not None else list(range(len(n)))
+    done, nbytes = [], 0
+    t0 = time.perf_counter()
+    for b in order:
+        O.decode(a["q"], a["blocks"], a["scales"], a["cache_lengths"], a["lookup_table"],
+                 a["scales_lookup_table"], a["max_prompt_length"], a["layer_idx"], a["softmax_scale"], requests=[b])
+        done.append(b)
+        nbytes += int(n[b]) * 580
+        if time.perf_counter() - t0 > budget_s:
+            break
+    dt = time.perf_counter() - t0
+    cores = len(os.sched_getaffinity(0))
+    return {"value": nbytes / dt / 1e9, "unit": "GB/s", "cores": cores, "blas_threads": threads, "kind": "oracle",
+            "sample": f"{len(done)} of {len(n)} requests (all {inp.cfg.num_q_heads} heads, "
+                      f"{int(sum(n[b] for b in done))} keys), float64 numpy, {dt:.1f} s"}
+
+
+def run_reference(args):
+    """Reference arm: the oracle timed on the host cores on the same workload's requests."""
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return 0
+    from paged_fp8_kv_mla_b200 import workloads as W
+    from oracle import mla_oracle as O
+    from tests.oracle_io import to_numpy
+    cfg = W.CONFIGS[args.config]
+    inp = W.make_inputs(cfg, device="cpu")
+    a = to_numpy(inp)
+    n = O.num_keys(a["cache_lengths"], a["max_prompt_length"])
+
+    def step(s):
+        b = s % len(n)
+        O.decode(a["q"], a["blocks"], a["scales"], a["cache_lengths"], a["lookup_table"],
+                 a["scales_lookup_table"], a["max_prompt_length"], a["layer_idx"], a["softmax_scale"], requests=[b])
+        return int(n[b]) * 580, a["max_prompt_length"]
+
+    for s in range(args.warmup):
+        step(s)
+    t0 = time.perf_counter()
+    nbytes = ntok = 0
+    for s in range(args.steps):
+        bb, tt = step(args.warmup + s)
+        nbytes += bb
+        ntok += tt
+    dt = time.perf_counter() - t0
+    v = nbytes / dt / 1e9
+    cores = len(os.sched_getaffinity(0))
+    line = {"impl": "reference", "metric": METRIC, "value": v, "unit": "GB/s", "n_gpus": args.gpus,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": dt / args.steps * 1e3,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "decode_tokens_per_s": ntok / dt,
+            "config": {"workload": cfg.name, "config_index": args.config, "step": "oracle decode of one request",
+                       "l2": "n/a (host)"},
+            "cpu_baseline": {"value": v, "unit": "GB/s", "cores": cores, "kind": "oracle",
+                             "sample": f"one request per step, rotating over {len(n)} requests"},
+            "e2e": {"value": v, "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+def main():
+    args = parse()
+    if args.impl == "reference":
+        return run_reference(args)
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local)
+    dist = None
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=torch.device("cuda", local))
+
+    import paged_fp8_kv_mla_b200 as M
+    from paged_fp8_kv_mla_b200 import workloads as W
+    M.load()
+    cfg = W.CONFIGS[args.config]
+    seed = cfg.seed + 7919 * rank
+    inp = W.make_inputs(cfg, device="cuda", seed=seed)
+    kv_bytes = inp.kv_scale_bytes()
+    flops = inp.flops()
+    B, T = cfg.batch, cfg.q_len
+    out = torch.empty((B, T, cfg.num_q_heads, 512), dtype=torch.bfloat16, device="cuda")
+    lse = torch.empty((B, T, cfg.num_q_heads), dtype=torch.float32, device="cuda")
+    l2 = torch.cuda.get_device_properties(local).L2_cache_size
+    flush = torch.empty(max(2 * l2, 256 << 20), dtype=torch.uint8, device="cuda")
+    stream = torch.cuda.current_stream()
+
+    def step():
+        M.decode_inputs(inp, out=out, lse=lse, stream=stream)
+
+    for _ in range(max(3, args.warmup)):
+        flush.zero_()
+        step()
+    torch.cuda.synchronize()
+    if M.device_status() != 0:
+        raise RuntimeError("device status error during warm-up")
+
+    K = args.steps
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(K)]
+    kev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(K)]
+    clocks = ClockSampler(local)
+    clocks.start()
+    if dist:
+        dist.barrier()
+    torch.cuda.synchronize()
+    for s in range(K):
+        flush.zero_()
+        M.set_timing_events(*kev[s])
+        ev[s][0].record(stream)
+        step()
+        ev[s][1].record(stream)
+    M.set_timing_events(None, None)
+    torch.cuda.synchronize()
+    if dist:
+        dist.barrier()
+    clk = clocks.stop()
+    step_ms = sum(a.elapsed_time(b) for a, b in ev) / K
+    kern_ms = sum(a.elapsed_time(b) for a, b in kev) / K
+    if M.device_status() != 0:
+        raise RuntimeError("device status error in the timed region")
+
+    # end to end through the public API with host buffers (pinned), copies inside the timed interval
+    e2e = None
+    if not args.no_e2e:
+        hq = inp.q.cpu().pin_memory()
+        hl = inp.cache_lengths.cpu().pin_memory()
+        hlut = inp.lookup_table.cpu().pin_memory()
+        hslut = None if inp.scales_lookup_table is None else inp.scales_lookup_table.cpu().pin_memory()
+        hout = torch.empty(out.shape, dtype=out.dtype, pin_memory=True)
+        hlse = torch.empty(lse.shape, dtype=lse.dtype, pin_memory=True)
+        dq, dl, dlut = torch.empty_like(inp.q), torch.empty_like(inp.cache_lengths), torch.empty_like(inp.lookup_table)
+        dslut = None if hslut is None else torch.empty_like(inp.scales_lookup_table)
+        h2d = hq.numel() * hq.element_size() + hl.numel() * 4 + hlut.numel() * 4 + (0 if hslut is None else hslut.numel() * 4)
+        d2h = hout.numel() * 2 + hlse.numel() * 4
+        Ke = min(K, 100)
+
+        def e2e_step():
+            dq.copy_(hq, non_blocking=True)
+            dl.copy_(hl, non_blocking=True)
+            dlut.copy_(hlut, non_blocking=True)
+            if dslut is not None:
+                dslut.copy_(hslut, non_blocking=True)
+            M.decode(dq, inp.blocks, inp.scales, dl, dlut, dslut, T, inp.max_cache_length, inp.layer_idx,
+                     inp.softmax_scale, out=out, lse=lse, stream=stream)
+            hout.copy_(out, non_blocking=True)
+            hlse.copy_(lse, non_blocking=True)
+
+        for _ in range(3):
+            e2e_step()
+        torch.cuda.synchronize()
+        eev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(Ke)]
+        if dist:
+            dist.barrier()
+        torch.cuda.synchronize()
+        for s in range(Ke):
+            flush.zero_()
+            eev[s][0].record(stream)
+            e2e_step()
+            eev[s][1].record(stream)
+        torch.cuda.synchronize()
+        e2e_ms = sum(a.elapsed_time(b) for a, b in eev) / Ke
+        if dist:
+            t = torch.tensor([e2e_ms], device="cuda")
+            dist.all_reduce(t, op=dist.ReduceOp.MAX)
+            e2e_ms = float(t.item())
+        e2e = {"value": kv_bytes * world / (e2e_ms * 1e-3) / 1e9, "unit": "GB/s", "h2d_bytes_per_step": h2d,
+               "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms}
+
+    if dist:
+        t = torch.tensor([step_ms, kern_ms], device="cuda")
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        step_ms, kern_ms = float(t[0].item()), float(t[1].item())
+
+    peaks = load_peaks()
+    gbs = kv_bytes * world / (step_ms * 1e-3) / 1e9
+    tflops_k = flops / (kern_ms * 1e-3) / 1e12
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        cpu = cpu_oracle_baseline(inp, args.cpu_seconds)
+    if rank == 0:
+        line = {
+            "metric": METRIC, "value": gbs, "unit": "GB/s", "n_gpus": world, "steps": K, "warmup": args.warmup,
+            "ms_per_step": step_ms, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+            "dtype": "e4m3 KV, bf16 MMA, fp32 accumulate", "data": "synthetic",
+            "decode_tokens_per_s": B * T * world / (step_ms * 1e-3),
+            "hbm_frac": gbs / world / peaks["hbm_gbs"],
+            "config": {"workload": cfg.name, "config_index": args.config, "batch": B, "q_len": T,
+                       "num_q_heads": cfg.num_q_heads, "page_size": cfg.page_size,
+                       "kv_scale_bytes_per_step": kv_bytes, "flops_per_step": flops,
+                       "l2": "flushed before every timed step (write of %d MB)" % (flush.numel() >> 20),
+                       "parallelism": f"replicas x{world}"},
+            "roofline": {"kernel": "mla_decode_kernel", "bound": "tensor", "achieved": tflops_k,
+                         "peak": peaks["bf16_tflops"], "unit": "TFLOP/s", "frac": tflops_k / peaks["bf16_tflops"],
+                         "peak_source": peaks["source"] + " bf16 burst",
+                         "traffic": recorded_traffic(cfg.name), "kernel_ms": kern_ms,
+                         "kv_gbs_in_kernel": kv_bytes / (kern_ms * 1e-3) / 1e9,
+                         "hbm_frac_in_kernel": kv_bytes / (kern_ms * 1e-3) / 1e9 / peaks["hbm_gbs"]},
+            "gpu_launches": 3 * K,
+            "clocks": clk,
+            "e2e": e2e,
+            "cpu_baseline": cpu,
+        }
+        print(json.dumps(line), flush=True)
+    if dist:
+        dist.barrier()
+        dist.destroy_process_group()
+    return 0
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -1,0 +1,169 @@
+/*
+ * mla_paged_fp8.h -- C ABI of the B200 (sm_100a) paged FP8-KV MLA decode library.
+ *
+ * The operation (one decode step of one layer):
+ *   A paged KV cache holds, for every token, one MLA latent row of 576 values
+ *   (512 latent + 64 rope) stored as FP8 e4m3 bytes, plus one fp32 scale per
+ *   token (quantization_granularity = head_size, so one scale per token per
+ *   head; Modular page "KVCacheScalesMHAOperand", description).  The cache
+ *   tensors and page tables are the arguments of the Modular function
+ *   "generic_get_paged_cache_with_scales" (Args):
+ *     blocks  [num_blocks, kv_dim, num_layers, page_size, num_heads, head_dim]
+ *     scales  [num_blocks, kv_dim, num_layers, page_size, num_heads, head_dim_granularity]
+ *     cache_lengths [batch], lookup_table [batch, max_pages],
+ *     max_prompt_length, max_cache_length, optional scales_lookup_table
+ *     [batch, max_pages] whose ids index the scales pool when the scales are
+ *     paged independently of the values.
+ *   For request b, query token i < T (= max_prompt_length) and query head h:
+ *     n_b   = cache_lengths[b] + T keys are stored (the step's T new tokens are
+ *             already written at positions cache_lengths[b] .. n_b - 1),
+ *     K[t]  = bf16_rn(f32_rn(e4m3(blocks[blk, 0, layer_idx, t % P, 0, :]) * s_t)),
+ *             blk = lookup_table[b][t / P], s_t read through scales_lookup_table
+ *             (or lookup_table when it is NULL) at the same slot,
+ *     V[t]  = K[t][0:512],
+ *     x[t]  = softmax_scale * <q[b,i,h,:], K[t]>  for t <= cache_lengths[b] + i,
+ *     lse   = ln sum_t exp(x[t]),   out[b,i,h,:] = sum_t exp(x[t] - lse) V[t].
+ *
+ * Conventions shared by every entry point:
+ *   - All tensor pointers are device pointers owned by the caller, contiguous
+ *     row-major in the shapes given.  The library keeps no pointer after the
+ *     call returns; the work is enqueued on `stream` and runs asynchronously,
+ *     so inputs must stay alive and outputs untouched until the stream passes it.
+ *   - uint32 tables are read as raw 32-bit values.
+ *   - Errors are returned as mla_status_t; nothing is thrown across the ABI.
+ *     mla_last_error_string() describes the last failure of the calling thread.
+ *   - Device-side preconditions (page ids < pool size, cache_lengths[b] <=
+ *     max_cache_length, lookup_table covering ceil(n_b / page_size) pages) are
+ *     checked by the kernels: a violation skips the bad page (its rows read as
+ *     stale data), sets a sticky device status word and never faults.
+ *     mla_get_device_status() returns and clears that word.
+ */
+#ifndef MLA_PAGED_FP8_H_
+#define MLA_PAGED_FP8_H_
+
+#include <stdint.h>
+#include <cuda_runtime_api.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  MLA_OK = 0,
+  MLA_ERR_INVALID_ARG = 1,   /* null pointer, bad shape, index out of range, misaligned pointer */
+  MLA_ERR_UNSUPPORTED = 2,   /* valid request outside the implemented subset (see below) */
+  MLA_ERR_CUDA = 3,          /* a CUDA runtime / driver call failed */
+  MLA_ERR_WORKSPACE = 4,     /* workspace allocation failed */
+  MLA_ERR_TIMEOUT = 5,       /* a kernel wait gave up (device status word) */
+  MLA_ERR_DEVICE_BOUNDS = 6  /* a page id or length was out of range on the device (status word) */
+} mla_status_t;
+
+/* Shapes of the paged cache (the 6-D tensors of "generic_get_paged_cache_with_scales")
+ * and of q.  Implemented subset: head_dim == 576, v_dim == 512, num_kv_heads == 1,
+ * head_dim_granularity == 1 (one fp32 scale per token), page_size a multiple of 16,
+ * kv_dim >= 1 (index 0, the latent cache, is read), any num_q_heads >= 1 (processed
+ * in groups of 128). */
+typedef struct {
+  int32_t batch;                /* B */
+  int32_t num_q_heads;          /* H */
+  int32_t head_dim;             /* 576 */
+  int32_t v_dim;                /* 512 */
+  int32_t num_blocks;           /* leading dim of blocks */
+  int32_t kv_dim;               /* second dim of blocks and scales */
+  int32_t num_layers;           /* third dim of blocks and scales */
+  int32_t page_size;            /* P */
+  int32_t num_kv_heads;         /* num_heads of blocks / scales: 1 */
+  int32_t num_scale_blocks;     /* leading dim of scales (may differ from num_blocks
+                                   when scales_lookup_table != NULL) */
+  int32_t head_dim_granularity; /* last dim of scales: 1 */
+  int32_t max_pages;            /* second dim of lookup_table (and scales_lookup_table) */
+} mla_paged_shape_t;
+
+/*
+ * mla_decode_paged_fp8 -- decode attention over the paged FP8 cache.
+ *
+ *   q                    bf16 [batch, max_prompt_length, num_q_heads, 576], 16-byte aligned
+ *   blocks               e4m3 [num_blocks, kv_dim, num_layers, page_size, 1, 576], 16-byte aligned
+ *   scales               fp32 [num_scale_blocks, kv_dim, num_layers, page_size, 1, 1], 16-byte aligned
+ *   cache_lengths        uint32 [batch]: tokens cached before this step
+ *   lookup_table         uint32 [batch, max_pages]: logical page -> block id
+ *   scales_lookup_table  NULL, or uint32 [batch, max_pages]: logical page -> scale block id
+ *   max_prompt_length    T >= 1, query tokens per request (uniform); host scalar
+ *   max_cache_length     max_b cache_lengths[b]; host scalar, used to size the launch
+ *   layer_idx            layer read from the num_layers dim, < num_layers
+ *   softmax_scale        multiplies q.k before the softmax
+ *   out                  bf16 [batch, max_prompt_length, num_q_heads, 512], fully overwritten
+ *   lse                  fp32 [batch, max_prompt_length, num_q_heads], natural log; may be NULL
+ *
+ * The pages pass max_prompt_length / max_cache_length as one-element device
+ * tensors; here they are host scalars so that sizing the launch needs no
+ * device-to-host read.  Long requests are split across SMs and merged with an
+ * LSE-weighted combine; the partial results live in a per-device workspace the
+ * library allocates on the first call (and grows when a larger problem needs
+ * it), so the first call on a device should not be inside stream capture.
+ * Calls on different streams of one device must not overlap (they share the
+ * workspace).
+ */
+mla_status_t mla_decode_paged_fp8(
+    const void* q, const void* blocks, const float* scales,
+    const uint32_t* cache_lengths, const uint32_t* lookup_table, const uint32_t* scales_lookup_table,
+    uint32_t max_prompt_length, uint32_t max_cache_length, uint32_t layer_idx, float softmax_scale,
+    const mla_paged_shape_t* shape, void* out, float* lse, cudaStream_t stream);
+
+/*
+ * mla_gather_dequant_bf16 -- steps A and C of the decode on their own: gather every
+ * stored key of every request through the page tables and dequantise it to bf16
+ * with the per-token scale, K[t] = bf16_rn(f32_rn(e4m3 * s_t)).  Runs the same
+ * page loader and converter code the decode kernel runs.
+ *
+ *   out_k  bf16 [batch, max_keys, 576]; row t of request b is written for
+ *          t < cache_lengths[b] + max_prompt_length, other rows are left untouched.
+ *   max_keys >= max_cache_length + max_prompt_length.
+ * Other arguments as for mla_decode_paged_fp8.
+ */
+mla_status_t mla_gather_dequant_bf16(
+    const void* blocks, const float* scales, const uint32_t* cache_lengths,
+    const uint32_t* lookup_table, const uint32_t* scales_lookup_table,
+    uint32_t max_prompt_length, uint32_t max_cache_length, uint32_t layer_idx,
+    const mla_paged_shape_t* shape, void* out_k, uint32_t max_keys, cudaStream_t stream);
+
+/*
+ * mla_set_num_clusters -- test and tuning hook: fix the number of 2-CTA clusters
+ * the decode splits the keys over (0 restores the default, one per resident
+ * cluster slot of the device).  Process-wide.  Smaller values make fewer, longer
+ * pieces; values above the resident count run in several waves.
+ */
+mla_status_t mla_set_num_clusters(int32_t num_clusters);
+
+/*
+ * mla_set_timing_events -- measurement hook: when both events are non-NULL, every later
+ * mla_decode_paged_fp8 call on this thread records `before` on its stream right before
+ * launching the decode kernel and `after` right after it, so that the caller can time that
+ * kernel alone (cudaEventElapsedTime).  Pass NULL, NULL to stop.  The events stay owned by
+ * the caller.
+ */
+mla_status_t mla_set_timing_events(cudaEvent_t before, cudaEvent_t after);
+
+/* Number of clusters the next decode on the current device will use. */
+int32_t mla_get_num_clusters(void);
+
+/* Text of the last error on the calling thread ("" if none). */
+const char* mla_last_error_string(void);
+
+/*
+ * mla_get_device_status -- synchronises `stream`, then returns and clears the
+ * sticky device status word of the current device: MLA_OK, MLA_ERR_DEVICE_BOUNDS
+ * or MLA_ERR_TIMEOUT.
+ */
+mla_status_t mla_get_device_status(cudaStream_t stream);
+
+/* Frees the workspace of every device this thread's process used (synchronises them). */
+mla_status_t mla_release_workspace(void);
+
+/* Library version, e.g. "0.1.0". */
+const char* mla_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* MLA_PAGED_FP8_H_ */

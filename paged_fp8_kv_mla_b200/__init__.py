@@ -1,0 +1,10 @@
+"""Paged FP8-KV MLA decode for B200 (sm_100a).
+
+The decode runs in the CUDA kernels of libmla_paged_fp8.so behind the C ABI in
+include/mla_paged_fp8.h; this package holds its Python binding (`_lib`), the
+build step (`build`) and the seeded workload generators (`workloads`).
+"""
+from ._lib import (  # noqa: F401
+    MlaError, decode, decode_inputs, gather_dequant, set_num_clusters, get_num_clusters, device_status,
+    release_workspace, version, set_timing_events, load, LIB_PATH, EXPORTED,
+)

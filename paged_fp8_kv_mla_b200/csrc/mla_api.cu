@@ -1,0 +1,399 @@
+// Host side of the C ABI declared in include/mla_paged_fp8.h: argument validation, the
+// per-device workspace, TMA descriptors for the FP8 block pool, and the three launches
+// (plan -> decode -> combine) on the caller's stream.
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include <cstdarg>
+#include <cstdio>
+#include <cstring>
+#include <mutex>
+#include <string>
+#include <vector>
+
+#include "mla_kernels.cuh"
+#include "mla_paged_fp8.h"
+
+namespace {
+
+thread_local std::string g_last_error;
+thread_local cudaEvent_t g_ev_before = nullptr;
+thread_local cudaEvent_t g_ev_after = nullptr;
+
+mla_status_t fail(mla_status_t st, const char* fmt, ...) {
+  char buf[512];
+  va_list ap;
+  va_start(ap, fmt);
+  vsnprintf(buf, sizeof(buf), fmt, ap);
+  va_end(ap);
+  g_last_error = buf;
+  return st;
+}
+
+#define MLA_CUDA(call)                                                                     \
+  do {                                                                                     \
+    cudaError_t e_ = (call);                                                               \
+    if (e_ != cudaSuccess) return fail(MLA_ERR_CUDA, "%s: %s", #call, cudaGetErrorString(e_)); \
+  } while (0)
+
+// ---------------------------------------------------------------- workspace (per device)
+struct Workspace {
+  void* ptr = nullptr;
+  size_t bytes = 0;
+};
+
+constexpr int kMaxDevices = 64;
+std::mutex g_mu;
+Workspace g_ws[kMaxDevices];
+int g_default_nc[kMaxDevices];         // resident 2-CTA cluster slots, 0 = not queried yet
+bool g_attr_set[kMaxDevices];
+int g_forced_nc = 0;
+
+size_t align_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
+
+struct WsLayout {
+  size_t hdr, item_start, item_nvis, cluster_first, part_lse, part_o, total;
+};
+
+WsLayout ws_layout(int items, int NC) {
+  WsLayout L{};
+  size_t o = 0;
+  L.hdr = o;           o = align_up(o + 64, 256);
+  L.item_start = o;    o = align_up(o + sizeof(int32_t) * (items + 1), 256);
+  L.item_nvis = o;     o = align_up(o + sizeof(int32_t) * items, 256);
+  L.cluster_first = o; o = align_up(o + sizeof(int32_t) * NC, 256);
+  L.part_lse = o;      o = align_up(o + sizeof(float) * 2 * NC * mla::MROWS, 256);
+  L.part_o = o;        o = align_up(o + sizeof(float) * 2 * NC * mla::MROWS * mla::V_DIM, 256);
+  L.total = o;
+  return L;
+}
+
+mla_status_t ensure_workspace(int dev, size_t bytes, void** out) {
+  std::lock_guard<std::mutex> lk(g_mu);
+  Workspace& w = g_ws[dev];
+  if (w.bytes < bytes) {
+    if (w.ptr) {
+      MLA_CUDA(cudaDeviceSynchronize());
+      MLA_CUDA(cudaFree(w.ptr));
+      w.ptr = nullptr;
+      w.bytes = 0;
+    }
+    const size_t want = align_up(bytes + bytes / 4, 1 << 20);
+    cudaError_t e = cudaMalloc(&w.ptr, want);
+    if (e != cudaSuccess) {
+      w.ptr = nullptr;
+      return fail(MLA_ERR_WORKSPACE, "workspace cudaMalloc(%zu) failed: %s", want, cudaGetErrorString(e));
+    }
+    w.bytes = want;
+  }
+  *out = w.ptr;
+  return MLA_OK;
+}
+
+mla_status_t device_setup(int dev, int* nc_out) {
+  std::lock_guard<std::mutex> lk(g_mu);
+  if (!g_attr_set[dev]) {
+    MLA_CUDA(cudaFuncSetAttribute(mla::mla_decode_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                  static_cast<int>(mla::SMEM_ALLOC)));
+    MLA_CUDA(cudaFuncSetAttribute(mla::mla_dequant_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                  static_cast<int>(mla::DQ_SMEM_ALLOC)));
+    g_attr_set[dev] = true;
+  }
+  if (g_default_nc[dev] == 0) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(2 * 1024);
+    cfg.blockDim = dim3(mla::NUM_THREADS);
+    cfg.dynamicSmemBytes = mla::SMEM_ALLOC;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = 2;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    int n = 0;
+    MLA_CUDA(cudaOccupancyMaxActiveClusters(&n, mla::mla_decode_kernel, &cfg));
+    if (n <= 0) return fail(MLA_ERR_UNSUPPORTED, "no 2-CTA cluster of the decode kernel fits on this device");
+    g_default_nc[dev] = n;
+  }
+  *nc_out = g_forced_nc > 0 ? g_forced_nc : g_default_nc[dev];
+  return MLA_OK;
+}
+
+// ---------------------------------------------------------------- TMA descriptors
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                  const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+mla_status_t get_encode_fn(EncodeTiledFn* fn) {
+  static EncodeTiledFn cached = nullptr;
+  static std::once_flag once;
+  static cudaError_t err = cudaSuccess;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    err = cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q);
+    if (err == cudaSuccess && q == cudaDriverEntryPointSuccess) cached = reinterpret_cast<EncodeTiledFn>(p);
+  });
+  if (!cached) return fail(MLA_ERR_CUDA, "cuTensorMapEncodeTiled unavailable (%s)", cudaGetErrorString(err));
+  *fn = cached;
+  return MLA_OK;
+}
+
+// 2-D view of the block pool: rows of 576 e4m3 bytes; box = (box_cols bytes, box_rows rows).
+mla_status_t make_block_map(CUtensorMap* map, const void* blocks, uint64_t rows, uint32_t box_cols,
+                            uint32_t box_rows) {
+  EncodeTiledFn enc;
+  mla_status_t st = get_encode_fn(&enc);
+  if (st != MLA_OK) return st;
+  cuuint64_t gdim[2] = {static_cast<cuuint64_t>(mla::HEAD_DIM), rows};
+  cuuint64_t gstride[1] = {static_cast<cuuint64_t>(mla::HEAD_DIM)};
+  cuuint32_t box[2] = {box_cols, box_rows};
+  cuuint32_t estride[2] = {1, 1};
+  CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void*>(blocks), gdim, gstride, box, estride,
+                   CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                   CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) return fail(MLA_ERR_CUDA, "cuTensorMapEncodeTiled failed (%d)", static_cast<int>(r));
+  return MLA_OK;
+}
+
+int gcd_int(int a, int b) {
+  while (b) {
+    const int t = a % b;
+    a = b;
+    b = t;
+  }
+  return a;
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+// Shared validation of the cache description; fills the parts of DecodeParams that describe it.
+mla_status_t check_cache(const void* blocks, const float* scales, const uint32_t* cache_lengths,
+                         const uint32_t* lookup_table, uint32_t max_prompt_length, uint32_t max_cache_length,
+                         uint32_t layer_idx, const mla_paged_shape_t* s, mla::DecodeParams* p, uint64_t* rows) {
+  if (!s) return fail(MLA_ERR_INVALID_ARG, "shape is NULL");
+  if (!blocks || !scales || !cache_lengths || !lookup_table)
+    return fail(MLA_ERR_INVALID_ARG, "blocks, scales, cache_lengths and lookup_table must be non-NULL");
+  if (s->batch < 0 || s->num_q_heads < 1 || s->num_blocks < 1 || s->kv_dim < 1 || s->num_layers < 1 ||
+      s->page_size < 1 || s->num_kv_heads < 1 || s->num_scale_blocks < 1 || s->head_dim_granularity < 1 ||
+      s->max_pages < 1)
+    return fail(MLA_ERR_INVALID_ARG, "non-positive dimension in shape");
+  if (s->head_dim != mla::HEAD_DIM || s->v_dim != mla::V_DIM)
+    return fail(MLA_ERR_UNSUPPORTED, "head_dim must be 576 and v_dim 512 (got %d, %d)", s->head_dim, s->v_dim);
+  if (s->num_kv_heads != 1) return fail(MLA_ERR_UNSUPPORTED, "num_kv_heads must be 1 (MLA latent cache)");
+  if (s->head_dim_granularity != 1)
+    return fail(MLA_ERR_UNSUPPORTED, "only one scale per token (head_dim_granularity 1) is implemented");
+  if (s->page_size % 16 != 0) return fail(MLA_ERR_UNSUPPORTED, "page_size must be a multiple of 16");
+  if (layer_idx >= static_cast<uint32_t>(s->num_layers))
+    return fail(MLA_ERR_INVALID_ARG, "layer_idx %u >= num_layers %d", layer_idx, s->num_layers);
+  if (max_prompt_length < 1) return fail(MLA_ERR_INVALID_ARG, "max_prompt_length must be >= 1");
+  if (!aligned16(blocks) || !aligned16(scales)) return fail(MLA_ERR_INVALID_ARG, "blocks and scales must be 16-byte aligned");
+  const uint64_t r = static_cast<uint64_t>(s->num_blocks) * s->kv_dim * s->num_layers * s->page_size;
+  const uint64_t sr = static_cast<uint64_t>(s->num_scale_blocks) * s->kv_dim * s->num_layers * s->page_size;
+  if (r >= (1ull << 31) || sr >= (1ull << 32))
+    return fail(MLA_ERR_UNSUPPORTED, "block pool too large (%llu rows)", static_cast<unsigned long long>(r));
+  const uint64_t need_pages = (static_cast<uint64_t>(max_cache_length) + max_prompt_length + s->page_size - 1) / s->page_size;
+  if (need_pages > static_cast<uint64_t>(s->max_pages))
+    return fail(MLA_ERR_INVALID_ARG, "lookup_table has %d pages per request, %llu needed for max_cache_length %u",
+                s->max_pages, static_cast<unsigned long long>(need_pages), max_cache_length);
+  if (static_cast<uint64_t>(max_cache_length) + max_prompt_length + 64 >= (1ull << 30))
+    return fail(MLA_ERR_UNSUPPORTED, "max_cache_length too large");
+  p->scales = scales;
+  p->lut = lookup_table;
+  p->B = s->batch;
+  p->T = static_cast<int>(max_prompt_length);
+  p->H = s->num_q_heads;
+  p->G = (s->num_q_heads + mla::MROWS - 1) / mla::MROWS;
+  p->P = s->page_size;
+  p->KVD = s->kv_dim;
+  p->NL = s->num_layers;
+  p->layer = static_cast<int>(layer_idx);
+  p->NB = s->num_blocks;
+  p->NSB = s->num_scale_blocks;
+  p->max_pages = s->max_pages;
+  p->boxr = gcd_int(s->page_size, mla::BN);
+  *rows = r;
+  return MLA_OK;
+}
+
+unsigned int* status_ptr() {
+  unsigned int* p = nullptr;
+  if (cudaGetSymbolAddress(reinterpret_cast<void**>(&p), mla::g_status_word) != cudaSuccess) return nullptr;
+  return p;
+}
+
+}  // namespace
+
+extern "C" {
+
+const char* mla_version(void) { return "0.1.0"; }
+
+const char* mla_last_error_string(void) { return g_last_error.c_str(); }
+
+mla_status_t mla_set_num_clusters(int32_t num_clusters) {
+  if (num_clusters < 0 || num_clusters > 65535) return fail(MLA_ERR_INVALID_ARG, "num_clusters out of range");
+  std::lock_guard<std::mutex> lk(g_mu);
+  g_forced_nc = num_clusters;
+  return MLA_OK;
+}
+
+mla_status_t mla_set_timing_events(cudaEvent_t before, cudaEvent_t after) {
+  if ((before == nullptr) != (after == nullptr)) return fail(MLA_ERR_INVALID_ARG, "pass both events or neither");
+  g_ev_before = before;
+  g_ev_after = after;
+  return MLA_OK;
+}
+
+int32_t mla_get_num_clusters(void) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev >= kMaxDevices) return -1;
+  int nc = 0;
+  if (device_setup(dev, &nc) != MLA_OK) return -1;
+  return nc;
+}
+
+mla_status_t mla_decode_paged_fp8(const void* q, const void* blocks, const float* scales,
+                                  const uint32_t* cache_lengths, const uint32_t* lookup_table,
+                                  const uint32_t* scales_lookup_table, uint32_t max_prompt_length,
+                                  uint32_t max_cache_length, uint32_t layer_idx, float softmax_scale,
+                                  const mla_paged_shape_t* shape, void* out, float* lse, cudaStream_t stream) {
+  mla::DecodeParams p{};
+  uint64_t rows = 0;
+  mla_status_t st = check_cache(blocks, scales, cache_lengths, lookup_table, max_prompt_length, max_cache_length,
+                                layer_idx, shape, &p, &rows);
+  if (st != MLA_OK) return st;
+  if (!q || !out) return fail(MLA_ERR_INVALID_ARG, "q and out must be non-NULL");
+  if (!aligned16(q) || !aligned16(out)) return fail(MLA_ERR_INVALID_ARG, "q and out must be 16-byte aligned");
+  if (!(softmax_scale == softmax_scale)) return fail(MLA_ERR_INVALID_ARG, "softmax_scale is NaN");
+  if (p.B == 0) return MLA_OK;
+  const int64_t items64 = static_cast<int64_t>(p.B) * p.T * p.G;
+  if (items64 > (1 << 24)) return fail(MLA_ERR_UNSUPPORTED, "too many (request, token, head-group) items");
+  p.items = static_cast<int>(items64);
+
+  int dev = 0;
+  MLA_CUDA(cudaGetDevice(&dev));
+  if (dev >= kMaxDevices) return fail(MLA_ERR_UNSUPPORTED, "device index too large");
+  int NC = 0;
+  st = device_setup(dev, &NC);
+  if (st != MLA_OK) return st;
+  p.NC = NC;
+
+  const WsLayout L = ws_layout(p.items, NC);
+  void* ws = nullptr;
+  st = ensure_workspace(dev, L.total, &ws);
+  if (st != MLA_OK) return st;
+  char* w = static_cast<char*>(ws);
+  p.hdr = reinterpret_cast<int32_t*>(w + L.hdr);
+  p.item_start = reinterpret_cast<int32_t*>(w + L.item_start);
+  p.item_nvis = reinterpret_cast<int32_t*>(w + L.item_nvis);
+  p.cluster_first = reinterpret_cast<int32_t*>(w + L.cluster_first);
+  p.part_lse = reinterpret_cast<float*>(w + L.part_lse);
+  p.part_o = reinterpret_cast<float*>(w + L.part_o);
+  p.q = static_cast<const uint16_t*>(q);
+  p.slut = scales_lookup_table;
+  p.out = static_cast<uint16_t*>(out);
+  p.lse = lse;
+  p.status = status_ptr();
+  if (!p.status) return fail(MLA_ERR_CUDA, "status word address unavailable");
+  p.scale_log2 = softmax_scale * 1.4426950408889634f;
+
+  CUtensorMap tm_lat, tm_rope;
+  st = make_block_map(&tm_lat, blocks, rows, 256, static_cast<uint32_t>(p.boxr));
+  if (st != MLA_OK) return st;
+  st = make_block_map(&tm_rope, blocks, rows, 32, static_cast<uint32_t>(p.boxr));
+  if (st != MLA_OK) return st;
+
+  mla::mla_plan_kernel<<<1, mla::PLAN_THREADS, 0, stream>>>(
+      cache_lengths, p.B, p.T, p.G, max_cache_length, NC, const_cast<int32_t*>(p.item_start),
+      const_cast<int32_t*>(p.item_nvis), const_cast<int32_t*>(p.cluster_first), const_cast<int32_t*>(p.hdr), p.status);
+  MLA_CUDA(cudaGetLastError());
+
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(2 * NC);
+  cfg.blockDim = dim3(mla::NUM_THREADS);
+  cfg.dynamicSmemBytes = mla::SMEM_ALLOC;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = 2;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  if (g_ev_before && g_ev_after) MLA_CUDA(cudaEventRecord(g_ev_before, stream));
+  MLA_CUDA(cudaLaunchKernelEx(&cfg, mla::mla_decode_kernel, p, tm_lat, tm_rope));
+  if (g_ev_before && g_ev_after) MLA_CUDA(cudaEventRecord(g_ev_after, stream));
+
+  const int per_item = mla::MROWS / mla::COMBINE_HEADS;
+  const int64_t cgrid = static_cast<int64_t>(p.items) * per_item;
+  if (cgrid > 0x7FFFFFFF) return fail(MLA_ERR_UNSUPPORTED, "combine grid too large");
+  mla::mla_combine_kernel<<<static_cast<unsigned>(cgrid), 32 * mla::COMBINE_HEADS, 0, stream>>>(p);
+  MLA_CUDA(cudaGetLastError());
+  return MLA_OK;
+}
+
+mla_status_t mla_gather_dequant_bf16(const void* blocks, const float* scales, const uint32_t* cache_lengths,
+                                     const uint32_t* lookup_table, const uint32_t* scales_lookup_table,
+                                     uint32_t max_prompt_length, uint32_t max_cache_length, uint32_t layer_idx,
+                                     const mla_paged_shape_t* shape, void* out_k, uint32_t max_keys,
+                                     cudaStream_t stream) {
+  mla::DecodeParams p{};
+  uint64_t rows = 0;
+  mla_status_t st = check_cache(blocks, scales, cache_lengths, lookup_table, max_prompt_length, max_cache_length,
+                                layer_idx, shape, &p, &rows);
+  if (st != MLA_OK) return st;
+  if (!out_k || !aligned16(out_k)) return fail(MLA_ERR_INVALID_ARG, "out_k must be non-NULL and 16-byte aligned");
+  if (static_cast<uint64_t>(max_keys) < static_cast<uint64_t>(max_cache_length) + max_prompt_length)
+    return fail(MLA_ERR_INVALID_ARG, "max_keys %u < max_cache_length + max_prompt_length", max_keys);
+  if (p.B == 0) return MLA_OK;
+  int dev = 0;
+  MLA_CUDA(cudaGetDevice(&dev));
+  if (dev >= kMaxDevices) return fail(MLA_ERR_UNSUPPORTED, "device index too large");
+  int NC = 0;
+  st = device_setup(dev, &NC);
+  if (st != MLA_OK) return st;
+  p.slut = scales_lookup_table;
+  p.status = status_ptr();
+  if (!p.status) return fail(MLA_ERR_CUDA, "status word address unavailable");
+  CUtensorMap tm_lat, tm_rope;
+  st = make_block_map(&tm_lat, blocks, rows, 256, static_cast<uint32_t>(p.boxr));
+  if (st != MLA_OK) return st;
+  st = make_block_map(&tm_rope, blocks, rows, 32, static_cast<uint32_t>(p.boxr));
+  if (st != MLA_OK) return st;
+  const int tiles = static_cast<int>((static_cast<uint64_t>(max_keys) + mla::BN - 1) / mla::BN);
+  const int64_t gx = static_cast<int64_t>(p.B) * tiles;
+  if (gx > 0x7FFFFFFF) return fail(MLA_ERR_UNSUPPORTED, "grid too large");
+  mla::mla_dequant_kernel<<<dim3(static_cast<unsigned>(gx), 2), mla::DQ_THREADS, mla::DQ_SMEM_ALLOC, stream>>>(
+      p, tm_lat, tm_rope, cache_lengths, static_cast<int>(max_keys), tiles, static_cast<uint16_t*>(out_k));
+  MLA_CUDA(cudaGetLastError());
+  return MLA_OK;
+}
+
+mla_status_t mla_get_device_status(cudaStream_t stream) {
+  MLA_CUDA(cudaStreamSynchronize(stream));
+  unsigned int v = 0, zero = 0;
+  MLA_CUDA(cudaMemcpyFromSymbol(&v, mla::g_status_word, sizeof(v)));
+  MLA_CUDA(cudaMemcpyToSymbol(mla::g_status_word, &zero, sizeof(zero)));
+  if (v & mla::STATUS_TIMEOUT) return fail(MLA_ERR_TIMEOUT, "a kernel wait timed out (status 0x%x)", v);
+  if (v & mla::STATUS_BOUNDS) return fail(MLA_ERR_DEVICE_BOUNDS, "page id or cache length out of range (status 0x%x)", v);
+  return MLA_OK;
+}
+
+mla_status_t mla_release_workspace(void) {
+  std::lock_guard<std::mutex> lk(g_mu);
+  int cur = 0;
+  cudaGetDevice(&cur);
+  for (int d = 0; d < kMaxDevices; ++d) {
+    if (!g_ws[d].ptr) continue;
+    MLA_CUDA(cudaSetDevice(d));
+    MLA_CUDA(cudaDeviceSynchronize());
+    MLA_CUDA(cudaFree(g_ws[d].ptr));
+    g_ws[d].ptr = nullptr;
+    g_ws[d].bytes = 0;
+  }
+  cudaSetDevice(cur);
+  return MLA_OK;
+}
+
+}  // extern "C"

@@ -1,0 +1,80 @@
+"""CPU-side checks of the C-ABI library: it loads, exports every declared symbol, and rejects bad
+arguments on the host before any CUDA work is enqueued."""
+import ctypes
+import os
+import re
+
+import pytest
+import torch
+
+import paged_fp8_kv_mla_b200 as M
+from paged_fp8_kv_mla_b200 import _lib, build
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="module")
+def lib():
+    build.build()
+    return _lib.load()
+
+
+def test_header_declarations_match_exports(lib):
+    hdr = open(os.path.join(ROOT, "include", "mla_paged_fp8.h")).read()
+    declared = set(re.findall(r"^\s*(?:mla_status_t|const char\*|int32_t)\s+(mla_\w+)\s*\(", hdr, re.M))
+    assert declared == set(_lib.EXPORTED)
+    for name in declared:
+        assert hasattr(lib, name), name
+
+
+def test_version(lib):
+    assert re.match(r"\d+\.\d+\.\d+", M.version())
+
+
+def _shape(**kw):
+    base = dict(batch=2, num_q_heads=16, head_dim=576, v_dim=512, num_blocks=16, kv_dim=1, num_layers=1,
+                page_size=16, num_kv_heads=1, num_scale_blocks=16, head_dim_granularity=1, max_pages=8)
+    base.update(kw)
+    return _lib.PagedShape(**base)
+
+
+FAKE = ctypes.c_void_p(0x10000)     # 16-byte aligned, never dereferenced: validation fails first
+
+
+def _call(lib, shape, q=FAKE, blocks=FAKE, scales=FAKE, lens=FAKE, lut=FAKE, slut=None, T=1, maxc=64, layer=0,
+          out=FAKE):
+    return lib.mla_decode_paged_fp8(q, blocks, scales, lens, lut, slut, T, maxc, layer, 0.07,
+                                    ctypes.byref(shape) if shape is not None else None, out, None, None)
+
+
+@pytest.mark.parametrize("kw,want", [
+    (dict(head_dim=512), 2), (dict(v_dim=256), 2), (dict(num_kv_heads=2), 2),
+    (dict(head_dim_granularity=9), 2), (dict(page_size=24), 2), (dict(num_layers=0), 1),
+    (dict(max_pages=2), 1),
+])
+def test_host_validation_rejects_bad_shapes(lib, kw, want):
+    assert _call(lib, _shape(**kw)) == want
+    assert lib.mla_last_error_string().decode()
+
+
+def test_host_validation_rejects_null_and_misaligned(lib):
+    assert _call(lib, None) == 1
+    assert _call(lib, _shape(), blocks=None) == 1
+    assert _call(lib, _shape(), q=ctypes.c_void_p(0x10004)) == 1
+    assert _call(lib, _shape(), layer=1) == 1
+    assert _call(lib, _shape(), T=0) == 1
+
+
+def test_set_num_clusters_range(lib):
+    assert lib.mla_set_num_clusters(-1) == 1
+    assert lib.mla_set_num_clusters(0) == 0
+
+
+def test_product_path_fails_loudly_without_library(tmp_path):
+    saved = _lib._lib
+    try:
+        _lib._lib = None
+        with pytest.raises(FileNotFoundError):
+            _lib.load(str(tmp_path / "missing.so"))
+    finally:
+        _lib._lib = saved
