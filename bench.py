@@ -243,6 +243,10 @@ def main():
     K = args.steps
     ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(K)]
     kev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(K)]
+    for a, b in kev:            # torch creates the CUDA event on first record; the library records them later
+        a.record(stream)
+        b.record(stream)
+    torch.cuda.synchronize()
     clocks = ClockSampler(local)
     clocks.start()
     if dist:

@@ -170,6 +170,8 @@ def release_workspace():
 
 def set_timing_events(before=None, after=None):
     """Record torch.cuda.Event `before`/`after` around every later decode-kernel launch (None, None stops)."""
+    if before is not None and (before.cuda_event == 0 or after.cuda_event == 0):
+        raise ValueError("record each event once before handing it to the library (torch creates it lazily)")
     b = None if before is None else ctypes.c_void_p(before.cuda_event)
     a = None if after is None else ctypes.c_void_p(after.cuda_event)
     _check(load().mla_set_timing_events(b, a))

@@ -19,6 +19,9 @@ namespace {
 thread_local std::string g_last_error;
 thread_local cudaEvent_t g_ev_before = nullptr;
 thread_local cudaEvent_t g_ev_after = nullptr;
+#ifdef MLA_TRACE
+unsigned long long* g_trace = nullptr;
+#endif
 
 mla_status_t fail(mla_status_t st, const char* fmt, ...) {
   char buf[512];
@@ -297,6 +300,9 @@ mla_status_t mla_decode_paged_fp8(const void* q, const void* blocks, const float
   p.status = status_ptr();
   if (!p.status) return fail(MLA_ERR_CUDA, "status word address unavailable");
   p.scale_log2 = softmax_scale * 1.4426950408889634f;
+#ifdef MLA_TRACE
+  p.trace = g_trace;
+#endif
 
   CUtensorMap tm_lat, tm_rope;
   st = make_block_map(&tm_lat, blocks, rows, 256, static_cast<uint32_t>(p.boxr));
@@ -369,6 +375,15 @@ mla_status_t mla_gather_dequant_bf16(const void* blocks, const float* scales, co
   MLA_CUDA(cudaGetLastError());
   return MLA_OK;
 }
+
+#ifdef MLA_TRACE
+// Trace builds only: cluster 0 of later decodes writes per-stage %clock64 stamps to `buf`
+// (2 * TRACE_TILES * TRACE_EVENTS uint64 values).
+mla_status_t mla_debug_set_trace(unsigned long long* buf) {
+  g_trace = buf;
+  return MLA_OK;
+}
+#endif
 
 mla_status_t mla_get_device_status(cudaStream_t stream) {
   MLA_CUDA(cudaStreamSynchronize(stream));

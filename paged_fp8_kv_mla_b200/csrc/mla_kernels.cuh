@@ -47,9 +47,11 @@ constexpr uint32_t SF0 = SK0 + 2 * SK_STRIDE;   // FP8 stages
 constexpr uint32_t SF_STRIDE = 19456;
 constexpr uint32_t SF_ROPE = 16384;       // 64 rows x 32 B
 constexpr uint32_t SF_SC = 18432;         // 64 fp32 scales
-constexpr uint32_t SX = SF0 + NFP8 * SF_STRIDE; // partial-score exchange, 128 rows x 272 B
-constexpr uint32_t SX_ROW = 272;
-constexpr uint32_t SBAR = SX + MROWS * SX_ROW;
+// partial-score exchange: [16 chunks][128 rows][16 B], so that one warp-wide store of chunk v by
+// 32 consecutive rows is 512 contiguous bytes
+constexpr uint32_t SX = SF0 + NFP8 * SF_STRIDE;
+constexpr uint32_t SX_CHUNK = MROWS * 16;
+constexpr uint32_t SBAR = SX + 16 * SX_CHUNK;
 constexpr uint32_t SMEM_USED = SBAR + 512;
 constexpr uint32_t SMEM_ALLOC = SMEM_USED + 1024;   // slack for aligning the base
 
@@ -74,7 +76,13 @@ constexpr unsigned STATUS_BOUNDS = 1u;
 constexpr unsigned STATUS_TIMEOUT = 2u;
 constexpr uint64_t WAIT_LIMIT_NS = 2000000000ull;   // 2 s per wait
 
+// Optional per-stage timestamps (build with -DMLA_TRACE): cluster 0 writes %clock64 values
+// to trace[(cta * TRACE_TILES + tile) * TRACE_EVENTS + event] for its first TRACE_TILES tiles.
+constexpr int TRACE_TILES = 64;
+constexpr int TRACE_EVENTS = 32;
+
 struct DecodeParams {
+  unsigned long long* trace;       // null unless tracing
   const uint16_t* q;               // bf16 bits [B, T, H, 576]
   const float* scales;
   const int32_t* item_start;       // [items + 1] tile prefix
@@ -127,6 +135,16 @@ struct UnitWalker {
   }
 };
 
+#ifdef MLA_TRACE
+#define MLA_TRACE_EV(tile, ev)                                                                        \
+  do {                                                                                                \
+    if (p.trace && k == 0 && (tile) < static_cast<uint32_t>(TRACE_TILES))                            \
+      p.trace[(c * TRACE_TILES + (tile)) * TRACE_EVENTS + (ev)] = clock64();                         \
+  } while (0)
+#else
+#define MLA_TRACE_EV(tile, ev) do {} while (0)
+#endif
+
 struct Smem {
   uint32_t base;
   __device__ uint32_t bar(uint32_t i) const { return base + SBAR + 8 * i; }
@@ -142,15 +160,17 @@ __device__ __forceinline__ void raise_status(unsigned int* status, unsigned bits
   atomicOr(status ? status : &g_status_word, bits);
 }
 
-// Bounded wait on an mbarrier phase.  Returns false (and marks the CTA, its peer and the
+// Bounded wait on an mbarrier phase (slow path below).  Returns false (and marks the CTA, its peer and the
 // status word) when the wait gives up or another role already gave up.
-__device__ __noinline__ bool wait_bar(uint32_t addr, uint32_t parity, bool cluster_scope,
-                                      volatile uint32_t* abort, unsigned int* status, uint32_t peer_abort) {
-  if (cluster_scope ? ptx::mbar_try_wait_cluster(addr, parity) : ptx::mbar_try_wait(addr, parity)) return true;
+__device__ __noinline__ bool wait_bar_slow(uint32_t addr, uint32_t parity, bool cluster_scope,
+                                           volatile uint32_t* abort, unsigned int* status, uint32_t peer_abort) {
   const uint64_t t0 = ptx::globaltimer();
   while (true) {
     for (int i = 0; i < 256; ++i) {
-      if (cluster_scope ? ptx::mbar_try_wait_cluster(addr, parity) : ptx::mbar_try_wait(addr, parity)) return true;
+      if (cluster_scope ? ptx::mbar_try_wait_relaxed_cluster(addr, parity) : ptx::mbar_try_wait(addr, parity)) {
+        if (cluster_scope) ptx::fence_acq_rel_cluster();
+        return true;
+      }
     }
     if (*abort) return false;
     if (ptx::globaltimer() - t0 > WAIT_LIMIT_NS) {
@@ -160,6 +180,19 @@ __device__ __noinline__ bool wait_bar(uint32_t addr, uint32_t parity, bool clust
       return false;
     }
   }
+}
+
+__device__ __forceinline__ bool wait_bar(uint32_t addr, uint32_t parity, bool cluster_scope, volatile uint32_t* abort,
+                                         unsigned int* status, uint32_t peer_abort) {
+  if (cluster_scope) {
+    if (ptx::mbar_try_wait_relaxed_cluster(addr, parity)) {
+      ptx::fence_acq_rel_cluster();
+      return true;
+    }
+  } else if (ptx::mbar_try_wait(addr, parity)) {
+    return true;
+  }
+  return wait_bar_slow(addr, parity, cluster_scope, abort, status, peer_abort);
 }
 
 // ---------------------------------------------------------------------------------------------
@@ -233,14 +266,23 @@ __device__ __forceinline__ uint32_t sw64_off(int r, int u) {
 // Convert one FP8 stage (this CTA's 288 dims of 64 rows) into a bf16 K tile; rows >= nv become 0.
 // Called by 128 threads (t = 0..127).
 __device__ __forceinline__ void convert_tile(int t, uint32_t stage, uint32_t ktile, int nv) {
-#pragma unroll 2
+  uint4 raw[9];
+  float sc[9];
+#pragma unroll
   for (int it = 0; it < 8; ++it) {
     const int id = it * 128 + t;
     const int row = id >> 4, cc = id & 15;
-    const uint4 raw = ptx::ld_shared_v4(stage + row * 256 + cc * 16);
-    const float s = ptx::ld_shared_f32(stage + SF_SC + row * 4);
+    raw[it] = ptx::ld_shared_v4(stage + row * 256 + cc * 16);
+    sc[it] = ptx::ld_shared_f32(stage + SF_SC + row * 4);
+  }
+  raw[8] = ptx::ld_shared_v4(stage + SF_ROPE + (t >> 1) * 32 + (t & 1) * 16);
+  sc[8] = ptx::ld_shared_f32(stage + SF_SC + (t >> 1) * 4);
+#pragma unroll
+  for (int it = 0; it < 8; ++it) {
+    const int id = it * 128 + t;
+    const int row = id >> 4, cc = id & 15;
     uint32_t w[8];
-    dequant16(raw, s, w);
+    dequant16(raw[it], sc[it], w);
     if (row >= nv) {
 #pragma unroll
       for (int k = 0; k < 8; ++k) w[k] = 0u;
@@ -252,10 +294,8 @@ __device__ __forceinline__ void convert_tile(int t, uint32_t stage, uint32_t kti
   }
   {
     const int row = t >> 1, cc = t & 1;
-    const uint4 raw = ptx::ld_shared_v4(stage + SF_ROPE + row * 32 + cc * 16);
-    const float s = ptx::ld_shared_f32(stage + SF_SC + row * 4);
     uint32_t w[8];
-    dequant16(raw, s, w);
+    dequant16(raw[8], sc[8], w);
     if (row >= nv) {
 #pragma unroll
       for (int k = 0; k < 8; ++k) w[k] = 0u;
@@ -362,18 +402,23 @@ mla_decode_kernel(const __grid_constant__ DecodeParams p, const __grid_constant_
     uint32_t g = 0, uu = 0;
     while (wk.next(u)) {
       MLA_WAIT_WARP(S.bar(B_Q_FREE), (uu & 1) ^ 1, false);
+      if (t == 0) MLA_TRACE_EV(g, 3);
       load_q(p, u, c, t, S.base);
       ptx::fence_proxy_async_smem();
       ptx::mbar_arrive(S.bar(B_Q_FULL));
+      if (t == 0) MLA_TRACE_EV(g, 4);
       for (int j = u.tb; j < u.te; ++j, ++g) {
         const uint32_t s = g & 1, ph = (g >> 1) & 1;
         MLA_WAIT_WARP(S.bar(B_FP8_FULL + s), ph, false);
+        if (t == 0) MLA_TRACE_EV(g, 0);
         MLA_WAIT_WARP(S.bar(B_K_EMPTY + s), ph ^ 1, false);
+        if (t == 0) MLA_TRACE_EV(g, 1);
         const int nv = min(BN, u.nvis - j * BN);
         convert_tile(t, S.base + SF0 + s * SF_STRIDE, S.base + SK0 + s * SK_STRIDE, nv);
         ptx::fence_proxy_async_smem();
         ptx::mbar_arrive(S.bar(B_FP8_EMPTY + s));
         ptx::mbar_arrive(S.bar(B_K_FULL + s));
+        if (t == 0) MLA_TRACE_EV(g, 2);
       }
       ++uu;
     }
@@ -382,7 +427,7 @@ mla_decode_kernel(const __grid_constant__ DecodeParams p, const __grid_constant_
     const int h = threadIdx.x - 128;
     const int quad = warp - 4;
     const uint32_t lane_base = tbase + (static_cast<uint32_t>(quad * 32) << 16);
-    const uint32_t xrow_local = S.base + SX + h * SX_ROW;
+    const uint32_t xrow_local = S.base + SX + h * 16;
     const uint32_t xrow_peer = ptx::mapa(xrow_local, peer);
     const uint32_t xs_full_peer = ptx::mapa(S.bar(B_XS_FULL), peer);
     const uint32_t xs_free_peer = ptx::mapa(S.bar(B_XS_FREE), peer);
@@ -394,6 +439,7 @@ mla_decode_kernel(const __grid_constant__ DecodeParams p, const __grid_constant_
       for (int j = u.tb; j < u.te; ++j, ++g, ++e) {
         const uint32_t sb = g & 1;
         MLA_WAIT_WARP(S.bar(B_S_FULL + sb), (g >> 1) & 1, false);
+        if (h == 0) MLA_TRACE_EV(g, 8);
         ptx::tc_fence_after();
         float x[BN];
         {
@@ -407,21 +453,27 @@ mla_decode_kernel(const __grid_constant__ DecodeParams p, const __grid_constant_
 #pragma unroll
           for (int q = 0; q < 32; ++q) x[32 + q] = __uint_as_float(r[q]);
         }
+        if (h == 0) MLA_TRACE_EV(g, 9);
         // exchange partial scores with the peer CTA (it holds the other 288 dims)
         MLA_WAIT_WARP(S.bar(B_XS_FREE), (e & 1) ^ 1, true);
+        if (h == 0) MLA_TRACE_EV(g, 10);
 #pragma unroll
-        for (int v = 0; v < 16; ++v) ptx::st_cluster_v4(xrow_peer + 16 * v, x[4 * v], x[4 * v + 1], x[4 * v + 2], x[4 * v + 3]);
+        for (int v = 0; v < 16; ++v)
+          ptx::st_cluster_v4(xrow_peer + v * SX_CHUNK, x[4 * v], x[4 * v + 1], x[4 * v + 2], x[4 * v + 3]);
         ptx::mbar_arrive_remote(xs_full_peer);
+        if (h == 0) MLA_TRACE_EV(g, 11);
         MLA_WAIT_WARP(S.bar(B_XS_FULL), e & 1, true);
+        if (h == 0) MLA_TRACE_EV(g, 12);
 #pragma unroll
         for (int v = 0; v < 16; ++v) {
-          const uint4 o = ptx::ld_shared_v4(xrow_local + 16 * v);
+          const uint4 o = ptx::ld_shared_v4(xrow_local + v * SX_CHUNK);
           x[4 * v] += __uint_as_float(o.x);
           x[4 * v + 1] += __uint_as_float(o.y);
           x[4 * v + 2] += __uint_as_float(o.z);
           x[4 * v + 3] += __uint_as_float(o.w);
         }
         ptx::mbar_arrive_remote(xs_free_peer);
+        if (h == 0) MLA_TRACE_EV(g, 13);
         // online softmax in the log2 domain
         const int nv = min(BN, u.nvis - j * BN);
         float mt = -INFINITY;
@@ -470,6 +522,7 @@ mla_decode_kernel(const __grid_constant__ DecodeParams p, const __grid_constant_
         ptx::tmem_wait_st();
         ptx::tc_fence_before();
         ptx::mbar_arrive(S.bar(B_P_FULL + sb));
+        if (h == 0) MLA_TRACE_EV(g, 14);
       }
       // epilogue: O / l
       {
@@ -516,6 +569,7 @@ mla_decode_kernel(const __grid_constant__ DecodeParams p, const __grid_constant_
         }
         ptx::tc_fence_before();
         ptx::mbar_arrive(S.bar(B_O_FREE));
+        if (h == 0) MLA_TRACE_EV(g - 1, 15);
       }
     }
   } else if (warp == 8) {
@@ -532,9 +586,11 @@ mla_decode_kernel(const __grid_constant__ DecodeParams p, const __grid_constant_
             ok = false;
             break;
           }
+          MLA_TRACE_EV(g, 16);
           const int nv = min(BN, u.nvis - j * BN);
           produce_tile(p, &tm_lat, &tm_rope, static_cast<int>(c), u.b, j * BN, nv, S.base + SF0 + s * SF_STRIDE,
                        S.bar(B_FP8_FULL + s));
+          MLA_TRACE_EV(g, 17);
           ++g;
         }
       }
@@ -559,6 +615,7 @@ mla_decode_kernel(const __grid_constant__ DecodeParams p, const __grid_constant_
         const uint32_t hb = hg & 1;
         if (first && !wait_bar(S.bar(B_O_FREE), (hu & 1) ^ 1, false, abort, p.status, peer_abort)) return false;
         if (!wait_bar(S.bar(B_P_FULL + hb), (hg >> 1) & 1, false, abort, p.status, peer_abort)) return false;
+        MLA_TRACE_EV(hg, 22);
         ptx::tc_fence_after();
         const uint32_t kt = S.base + SK0 + hb * SK_STRIDE;
 #pragma unroll
@@ -568,6 +625,7 @@ mla_decode_kernel(const __grid_constant__ DecodeParams p, const __grid_constant_
         }
         ptx::mma_commit(S.bar(B_O_DONE + hb));
         ptx::mma_commit(S.bar(B_K_EMPTY + hb));
+        MLA_TRACE_EV(hg, 23);
         return true;
       };
       while (wk.next(u)) {
@@ -576,6 +634,7 @@ mla_decode_kernel(const __grid_constant__ DecodeParams p, const __grid_constant_
         for (int j = u.tb; j < u.te; ++j, ++g) {
           const uint32_t kb = g & 1;
           MLA_WAIT(S.bar(B_K_FULL + kb), (g >> 1) & 1, false);
+          MLA_TRACE_EV(g, 20);
           ptx::tc_fence_after();
           const uint32_t kt = S.base + SK0 + kb * SK_STRIDE;
           const uint32_t dS = tbase + T_S + 64 * kb;
@@ -592,6 +651,7 @@ mla_decode_kernel(const __grid_constant__ DecodeParams p, const __grid_constant_
             ptx::mma_ss(dS, ad, bd, IDESC_QK, 1u);
           }
           ptx::mma_commit(S.bar(B_S_FULL + kb));
+          MLA_TRACE_EV(g, 21);
           if (j == u.te - 1) ptx::mma_commit(S.bar(B_Q_FREE));
           if (have_prev && !issue_pv(prev_g, prev_first, prev_u)) goto role_done;
           have_prev = true;
