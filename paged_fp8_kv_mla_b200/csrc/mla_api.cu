@@ -1,7 +1,5 @@
 // Host side of the C ABI declared in include/mla_paged_fp8.h: argument validation, the
-// per-device workspace, TMA descriptors for the FP8 block pool, and the three launches
-// (plan -> decode -> combine) on the caller's stream.
-#include <cuda.h>
+// per-device workspace, and the three launches (plan -> decode -> combine) on the caller's stream.
 #include <cuda_runtime.h>
 
 #include <cstdarg>
@@ -123,52 +121,6 @@ mla_status_t device_setup(int dev, int* nc_out) {
   return MLA_OK;
 }
 
-// ---------------------------------------------------------------- TMA descriptors
-typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
-                                  const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
-                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
-
-mla_status_t get_encode_fn(EncodeTiledFn* fn) {
-  static EncodeTiledFn cached = nullptr;
-  static std::once_flag once;
-  static cudaError_t err = cudaSuccess;
-  std::call_once(once, [] {
-    void* p = nullptr;
-    cudaDriverEntryPointQueryResult q;
-    err = cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q);
-    if (err == cudaSuccess && q == cudaDriverEntryPointSuccess) cached = reinterpret_cast<EncodeTiledFn>(p);
-  });
-  if (!cached) return fail(MLA_ERR_CUDA, "cuTensorMapEncodeTiled unavailable (%s)", cudaGetErrorString(err));
-  *fn = cached;
-  return MLA_OK;
-}
-
-// 2-D view of the block pool: rows of 576 e4m3 bytes; box = (box_cols bytes, box_rows rows).
-mla_status_t make_block_map(CUtensorMap* map, const void* blocks, uint64_t rows, uint32_t box_cols,
-                            uint32_t box_rows) {
-  EncodeTiledFn enc;
-  mla_status_t st = get_encode_fn(&enc);
-  if (st != MLA_OK) return st;
-  cuuint64_t gdim[2] = {static_cast<cuuint64_t>(mla::HEAD_DIM), rows};
-  cuuint64_t gstride[1] = {static_cast<cuuint64_t>(mla::HEAD_DIM)};
-  cuuint32_t box[2] = {box_cols, box_rows};
-  cuuint32_t estride[2] = {1, 1};
-  CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void*>(blocks), gdim, gstride, box, estride,
-                   CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-                   CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
-  if (r != CUDA_SUCCESS) return fail(MLA_ERR_CUDA, "cuTensorMapEncodeTiled failed (%d)", static_cast<int>(r));
-  return MLA_OK;
-}
-
-int gcd_int(int a, int b) {
-  while (b) {
-    const int t = a % b;
-    a = b;
-    b = t;
-  }
-  return a;
-}
-
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
 // Shared validation of the cache description; fills the parts of DecodeParams that describe it.
@@ -215,7 +167,7 @@ mla_status_t check_cache(const void* blocks, const float* scales, const uint32_t
   p->NB = s->num_blocks;
   p->NSB = s->num_scale_blocks;
   p->max_pages = s->max_pages;
-  p->boxr = gcd_int(s->page_size, mla::BN);
+  p->blocks = static_cast<const uint8_t*>(blocks);
   *rows = r;
   return MLA_OK;
 }
@@ -304,12 +256,6 @@ mla_status_t mla_decode_paged_fp8(const void* q, const void* blocks, const float
   p.trace = g_trace;
 #endif
 
-  CUtensorMap tm_lat, tm_rope;
-  st = make_block_map(&tm_lat, blocks, rows, 256, static_cast<uint32_t>(p.boxr));
-  if (st != MLA_OK) return st;
-  st = make_block_map(&tm_rope, blocks, rows, 32, static_cast<uint32_t>(p.boxr));
-  if (st != MLA_OK) return st;
-
   mla::mla_plan_kernel<<<1, mla::PLAN_THREADS, 0, stream>>>(
       cache_lengths, p.B, p.T, p.G, max_cache_length, NC, const_cast<int32_t*>(p.item_start),
       const_cast<int32_t*>(p.item_nvis), const_cast<int32_t*>(p.cluster_first), const_cast<int32_t*>(p.hdr), p.status);
@@ -328,7 +274,7 @@ mla_status_t mla_decode_paged_fp8(const void* q, const void* blocks, const float
   cfg.attrs = attr;
   cfg.numAttrs = 1;
   if (g_ev_before && g_ev_after) MLA_CUDA(cudaEventRecord(g_ev_before, stream));
-  MLA_CUDA(cudaLaunchKernelEx(&cfg, mla::mla_decode_kernel, p, tm_lat, tm_rope));
+  MLA_CUDA(cudaLaunchKernelEx(&cfg, mla::mla_decode_kernel, p));
   if (g_ev_before && g_ev_after) MLA_CUDA(cudaEventRecord(g_ev_after, stream));
 
   const int per_item = mla::MROWS / mla::COMBINE_HEADS;
@@ -362,16 +308,11 @@ mla_status_t mla_gather_dequant_bf16(const void* blocks, const float* scales, co
   p.slut = scales_lookup_table;
   p.status = status_ptr();
   if (!p.status) return fail(MLA_ERR_CUDA, "status word address unavailable");
-  CUtensorMap tm_lat, tm_rope;
-  st = make_block_map(&tm_lat, blocks, rows, 256, static_cast<uint32_t>(p.boxr));
-  if (st != MLA_OK) return st;
-  st = make_block_map(&tm_rope, blocks, rows, 32, static_cast<uint32_t>(p.boxr));
-  if (st != MLA_OK) return st;
   const int tiles = static_cast<int>((static_cast<uint64_t>(max_keys) + mla::BN - 1) / mla::BN);
   const int64_t gx = static_cast<int64_t>(p.B) * tiles;
   if (gx > 0x7FFFFFFF) return fail(MLA_ERR_UNSUPPORTED, "grid too large");
   mla::mla_dequant_kernel<<<dim3(static_cast<unsigned>(gx), 2), mla::DQ_THREADS, mla::DQ_SMEM_ALLOC, stream>>>(
-      p, tm_lat, tm_rope, cache_lengths, static_cast<int>(max_keys), tiles, static_cast<uint16_t*>(out_k));
+      p, cache_lengths, static_cast<int>(max_keys), tiles, static_cast<uint16_t*>(out_k));
   MLA_CUDA(cudaGetLastError());
   return MLA_OK;
 }

@@ -1,28 +1,33 @@
 // Device code of the paged FP8-KV MLA decode for sm_100a.
 //
-// Work decomposition.  An "item" is one (request b, query token i, group of 128
-// query heads g).  Item keys are tiled in BN = 64-token tiles; all items' tiles
-// are laid end to end and cut into equal contiguous ranges, one per 2-CTA
-// cluster.  A cluster walks the pieces ("units") of items that fall in its
-// range.  An item cut by a range boundary is "split": each piece writes a
-// normalised fp32 partial and its LSE, and the combine kernel merges them.
+// Work decomposition.  An "item" is one (request b, query token i, group of 128 query heads g).
+// Item keys are tiled in BN = 64-key tiles; all items' tiles are laid end to end and cut into
+// equal contiguous ranges, one per 2-CTA cluster.  A cluster walks the pieces ("units") of the
+// items in its range.  An item cut by a range boundary is "split": each piece writes a normalised
+// fp32 partial and its LSE, and the combine kernel merges them.
 //
-// Inside a cluster the two CTAs split the 576 latent dims: CTA c owns latent
-// dims [256c, 256c+256) and rope dims [512+32c, 512+32c+32), i.e. half of every
-// token's bytes.  Each CTA computes a partial Q.K^T over its 288 dims with
-// tcgen05 MMAs (M = 128 heads), the two partial score tiles are exchanged
-// through distributed shared memory and added, both CTAs run the same online
-// softmax, and each computes P.V for its own 256 V dims (V = the first 512
-// latent dims).  TMEM per CTA: O 128 x 256 fp32 (cols 0..255) and two score
-// buffers of 64 cols (P overwrites its score buffer as packed bf16).
+// The two CTAs of a cluster form one tcgen05 CTA pair (cta_group::2).  Pair MMAs have M = 128:
+// CTA c supplies rows 64c..64c+63 of A and half of B along N, and receives rows 64c..64c+63 of D
+// in its tensor memory (row r's first N/2 columns in TMEM lane r, the other N/2 in lane r + 64).
+//   Q.K^T : A = Q (CTA c holds heads 64c..64c+63, all 576 dims), B = the 64 keys of a tile
+//           (CTA c holds keys 32c..32c+31, all 576 dims).  Each CTA gets complete score rows for
+//           its 64 heads, so the softmax needs no cross-CTA exchange.
+//   P.V   : two MMAs of N = 256 (V dims 0..255 and 256..511).  A = P (CTA c's 64 heads, 64 keys);
+//           B = V split along N: CTA c holds, for all 64 keys of the tile, the V dims
+//           D_c = [128c, 128c+128) u [256+128c, 256+128c+128).  Its own 32 keys' D_c dims come from
+//           the same conversion as its K half; it dequantises the other CTA's 32 keys' D_c dims
+//           itself (256 of their 576 bytes), so no converted data crosses between SMs.
+// Every KV byte is read from HBM once (the second CTA's partial reads hit L2).
 //
-// Warp roles per CTA (320 threads):
-//   warps 0-3  converter: Q tile load at each unit start; FP8 -> bf16 dequant of
-//              every KV tile into the UMMA K-major SWIZZLE_128B/64B layout
-//   warps 4-7  softmax: score exchange, online softmax, P -> TMEM, O rescale,
-//              epilogue (one thread per head row / TMEM lane)
-//   warp 8     producer: TMA loads of the FP8 rows + bulk copies of the scales
-//   warp 9     MMA issuer (lane 0) and TMEM owner
+// Warp roles per CTA (448 threads):
+//   warps 0-7   converter: Q tile at each unit start; FP8 -> bf16 dequant of the tile's keys into
+//               the UMMA K-major SWIZZLE_128B layout (K half and V operand buffers); the FP8 bytes
+//               of tile g+1 are loaded into registers while tile g is converted
+//   warps 8-11  softmax: online softmax of the CTA's 64 heads (two lanes per head row), P -> SMEM,
+//               lazy O rescale, epilogue
+//   warp 12     producer: L2 prefetch of upcoming page runs
+//   warp 13     MMA issuer (CTA 0 of the pair; one elected lane issues) and TMEM owner (pair
+//               allocation in both CTAs)
 #pragma once
 #include <cuda_bf16.h>
 #include <cstdint>
@@ -30,43 +35,57 @@
 
 namespace mla {
 
-constexpr int BN = 64;          // tokens per tile
+constexpr int BN = 64;          // keys per tile (both CTAs)
+constexpr int HALF_BN = 32;     // keys per CTA in the Q.K^T B operand
 constexpr int HEAD_DIM = 576;
 constexpr int V_DIM = 512;
-constexpr int MROWS = 128;      // query heads per item (MMA M)
-constexpr int NUM_THREADS = 320;
-constexpr int NFP8 = 2;         // FP8 staging stages
+constexpr int MROWS = 128;      // query heads per item (pair MMA M)
+constexpr int HPC = 64;         // query heads per CTA
+constexpr int NUM_THREADS = 448;
+constexpr int CONV_THREADS = 256;
+constexpr int CONV_WARPS = CONV_THREADS / 32;
+constexpr int SM_WARP0 = 8;     // first softmax warp (warps 8..11 reach TMEM lane quadrants 0..3)
+constexpr int PROD_WARP = 12;
+constexpr int MMA_WARP = 13;
+constexpr int PF_DIST = 4;      // tiles of L2 prefetch lead
 
-// ---- shared memory map (offsets from a 1024-byte aligned base)
-constexpr uint32_t SQ_LAT = 0;            // Q latent half: 4 atom columns x (128 rows x 128 B), SW128
-constexpr uint32_t SQ_ROPE = 65536;       // Q rope half: 128 rows x 64 B, SW64
-constexpr uint32_t SK0 = 73728;           // bf16 K tiles (2): latent 4 x (64 x 128 B) SW128, rope 64 x 64 B SW64
-constexpr uint32_t SK_STRIDE = 36864;
-constexpr uint32_t SK_ROPE = 32768;
-constexpr uint32_t SF0 = SK0 + 2 * SK_STRIDE;   // FP8 stages
-constexpr uint32_t SF_STRIDE = 19456;
-constexpr uint32_t SF_ROPE = 16384;       // 64 rows x 32 B
-constexpr uint32_t SF_SC = 18432;         // 64 fp32 scales
-// partial-score exchange: [16 chunks][128 rows][16 B], so that one warp-wide store of chunk v by
-// 32 consecutive rows is 512 contiguous bytes
-constexpr uint32_t SX = SF0 + NFP8 * SF_STRIDE;
-constexpr uint32_t SX_CHUNK = MROWS * 16;
-constexpr uint32_t SBAR = SX + 16 * SX_CHUNK;
-constexpr uint32_t SMEM_USED = SBAR + 512;
+// ---- shared memory map (offsets from a 1024-byte aligned base); all operands K-major SWIZZLE_128B,
+//      one "atom column" = 64 bf16 dims x rows at 128 B, 8-row groups 1024 B apart
+constexpr uint32_t SQ = 0;                       // Q: 9 atom columns x (64 rows x 128 B)
+constexpr uint32_t SQ_ATOM = 8192;
+constexpr uint32_t SK0 = 9 * SQ_ATOM;            // K half (2 buffers): 9 atom columns x (32 rows x 128 B)
+constexpr uint32_t SK_ATOM = 4096;
+constexpr uint32_t SK_STRIDE = 9 * SK_ATOM;
+constexpr uint32_t SV0 = SK0 + 2 * SK_STRIDE;    // V operand (2 buffers): 4 atom columns x (64 rows x 128 B)
+constexpr uint32_t SV_ATOM = 8192;
+constexpr uint32_t SV_STRIDE = 4 * SV_ATOM;
+constexpr uint32_t SP0 = SV0 + 2 * SV_STRIDE;    // P (2 buffers): 64 rows x 128 B
+constexpr uint32_t SP_STRIDE = 8192;
+constexpr uint32_t SRED = SP0 + 2 * SP_STRIDE;   // row-max exchange [2][128] f32, row-sum exchange [128] f32
+constexpr uint32_t SBAR = SRED + 1536;
+constexpr uint32_t SMEM_USED = SBAR + 256;
 constexpr uint32_t SMEM_ALLOC = SMEM_USED + 1024;   // slack for aligning the base
 
-// barrier indices (8 bytes each from SBAR)
 enum Bar : uint32_t {
-  B_FP8_FULL = 0, B_FP8_EMPTY = 2, B_K_FULL = 4, B_K_EMPTY = 6, B_S_FULL = 8, B_P_FULL = 10,
-  B_O_DONE = 12, B_O_FREE = 14, B_Q_FULL = 15, B_Q_FREE = 16, B_XS_FULL = 17, B_XS_FREE = 18,
-  B_DRAIN = 19, NUM_BARS = 20
+  B_KV_FULL = 0,   // [2] CTA 0: 16 warp arrivals (8 converter warps of each CTA)
+  B_PV_DONE = 2,   // [2] both CTAs: pair commit after P.V of a tile (its K/V/P buffers are free)
+  B_S_FULL = 4,    // [2] both CTAs: pair commit after Q.K^T of a tile
+  B_P_FULL = 6,    // [2] CTA 0: 8 warp arrivals (4 softmax warps of each CTA)
+  B_Q_FULL = 8,    // CTA 0: 16 warp arrivals (converter warps)
+  B_Q_FREE = 9,    // both CTAs: pair commit after the last Q.K^T of a unit
+  B_O_FREE = 10,   // CTA 0: 8 warp arrivals after each CTA's epilogue
+  B_DRAIN = 11,
+  B_RED = 12,      // [2] softmax warps of this CTA: row-max exchange of a tile (4 warp arrivals)
+  B_REDL = 14,     // softmax warps of this CTA: row-sum exchange at a unit's end (4 warp arrivals)
+  NUM_BARS = 15
 };
-constexpr uint32_t S_TMEM_BASE = SBAR + 256;
-constexpr uint32_t S_ABORT = SBAR + 260;
+constexpr uint32_t S_TMEM_BASE = SBAR + 128;
+constexpr uint32_t S_ABORT = SBAR + 132;
+constexpr uint32_t S_CONV_TILE = SBAR + 136;
 
-// TMEM columns
-constexpr uint32_t T_O = 0;
-constexpr uint32_t T_S = 256;             // + 64 * buffer
+// TMEM columns (pair layout)
+constexpr uint32_t T_O = 0;                      // P.V halves: cols 0..127 (dims 0..255), 128..255 (256..511)
+constexpr uint32_t T_S = 256;                    // + 32 * buffer
 constexpr uint32_t TMEM_COLS = 512;
 
 constexpr uint32_t IDESC_QK = ptx::idesc_bf16_f32(128, BN, false, false);
@@ -76,15 +95,16 @@ constexpr unsigned STATUS_BOUNDS = 1u;
 constexpr unsigned STATUS_TIMEOUT = 2u;
 constexpr uint64_t WAIT_LIMIT_NS = 2000000000ull;   // 2 s per wait
 
-// Optional per-stage timestamps (build with -DMLA_TRACE): cluster 0 writes %clock64 values
-// to trace[(cta * TRACE_TILES + tile) * TRACE_EVENTS + event] for its first TRACE_TILES tiles.
+// Optional per-stage timestamps (build with -DMLA_TRACE): cluster 0 writes %clock64 values to
+// trace[(cta * TRACE_TILES + tile) * TRACE_EVENTS + event] for its first TRACE_TILES tiles.
 constexpr int TRACE_TILES = 64;
 constexpr int TRACE_EVENTS = 32;
 
 struct DecodeParams {
   unsigned long long* trace;       // null unless tracing
   const uint16_t* q;               // bf16 bits [B, T, H, 576]
-  const float* scales;
+  const uint8_t* blocks;           // e4m3 [NB, KVD, NL, P, 1, 576]
+  const float* scales;             // fp32 [NSB, KVD, NL, P, 1, 1]
   const int32_t* item_start;       // [items + 1] tile prefix
   const int32_t* item_nvis;        // [items] visible keys (clamped)
   const int32_t* cluster_first;    // [NC] first item of each cluster range
@@ -96,7 +116,7 @@ struct DecodeParams {
   float* part_o;                   // [2 NC][128][512]
   float* part_lse;                 // [2 NC][128]
   unsigned int* status;
-  int B, T, H, G, P, KVD, NL, layer, NB, NSB, max_pages, boxr, items, NC;
+  int B, T, H, G, P, KVD, NL, layer, NB, NSB, max_pages, items, NC;
   float scale_log2;                // softmax_scale * log2(e)
 };
 
@@ -108,24 +128,24 @@ struct Unit {
 
 // Walks the units of cluster `k`: the pieces of items inside tile range [R0, R1).
 struct UnitWalker {
-  const DecodeParams& p;
+  const DecodeParams* p;
   int k, R0, R1, it;
-  __device__ UnitWalker(const DecodeParams& p_, int k_) : p(p_), k(k_) {
-    const int tpc = p.hdr[0], total = p.hdr[1];
+  __device__ UnitWalker(const DecodeParams& p_, int k_) : p(&p_), k(k_) {
+    const int tpc = p->hdr[0], total = p->hdr[1];
     R0 = k * tpc;
     R1 = min(total, R0 + tpc);
-    it = p.cluster_first[k];
+    it = p->cluster_first[k];
   }
   __device__ bool next(Unit& u) {
-    if (R0 >= R1 || it >= p.items) return false;
-    const int s = p.item_start[it], e = p.item_start[it + 1];
+    if (R0 >= R1 || it >= p->items) return false;
+    const int s = p->item_start[it], e = p->item_start[it + 1];
     const int a = max(s, R0), z = min(e, R1);
     if (a >= z) return false;
     u.item = it;
-    u.g = it % p.G;
-    u.i = (it / p.G) % p.T;
-    u.b = it / (p.G * p.T);
-    u.nvis = p.item_nvis[it];
+    u.g = it % p->G;
+    u.i = (it / p->G) % p->T;
+    u.b = it / (p->G * p->T);
+    u.nvis = p->item_nvis[it];
     u.tb = a - s;
     u.te = z - s;
     const bool split = (s < R0) || (e > R1);
@@ -134,6 +154,12 @@ struct UnitWalker {
     return true;
   }
 };
+
+__device__ unsigned int g_status_word;   // sticky device status (bit 0 bounds, bit 1 timeout)
+
+__device__ __forceinline__ void raise_status(unsigned int* status, unsigned bits) {
+  atomicOr(status ? status : &g_status_word, bits);
+}
 
 #ifdef MLA_TRACE
 #define MLA_TRACE_EV(tile, ev)                                                                        \
@@ -145,32 +171,19 @@ struct UnitWalker {
 #define MLA_TRACE_EV(tile, ev) do {} while (0)
 #endif
 
-struct Smem {
-  uint32_t base;
-  __device__ uint32_t bar(uint32_t i) const { return base + SBAR + 8 * i; }
-};
-
-__device__ __forceinline__ volatile uint32_t* abort_flag(uint8_t* smem_base) {
-  return reinterpret_cast<volatile uint32_t*>(smem_base + S_ABORT);
-}
-
-__device__ unsigned int g_status_word;   // sticky device status (bit 0 bounds, bit 1 timeout)
-
-__device__ __forceinline__ void raise_status(unsigned int* status, unsigned bits) {
-  atomicOr(status ? status : &g_status_word, bits);
-}
-
-// Bounded wait on an mbarrier phase (slow path below).  Returns false (and marks the CTA, its peer and the
-// status word) when the wait gives up or another role already gave up.
-__device__ __noinline__ bool wait_bar_slow(uint32_t addr, uint32_t parity, bool cluster_scope,
-                                           volatile uint32_t* abort, unsigned int* status, uint32_t peer_abort) {
+// Bounded waits on an mbarrier phase.  wait_bar: CTA-scope acquire, for barriers arrived on by
+// this CTA's threads or by tcgen05 commits.  wait_bar_cl: cluster-scope acquire, for barriers the
+// other CTA's threads arrive on (their shared-memory writes must be visible afterwards).  Both
+// return false (and mark the CTA, its peer and the status word) when the wait gives up or another
+// role already gave up.
+template <bool CLUSTER>
+__device__ __noinline__ bool wait_bar_slow(uint32_t addr, uint32_t parity, volatile uint32_t* abort,
+                                           unsigned int* status, uint32_t peer_abort) {
   const uint64_t t0 = ptx::globaltimer();
   while (true) {
-    for (int i = 0; i < 256; ++i) {
-      if (cluster_scope ? ptx::mbar_try_wait_relaxed_cluster(addr, parity) : ptx::mbar_try_wait(addr, parity)) {
-        if (cluster_scope) ptx::fence_acq_rel_cluster();
+    for (int i = 0; i < 16; ++i) {
+      if (CLUSTER ? ptx::mbar_try_wait_acq_cluster(addr, parity) : ptx::mbar_try_wait_sleep(addr, parity, 100000u))
         return true;
-      }
     }
     if (*abort) return false;
     if (ptx::globaltimer() - t0 > WAIT_LIMIT_NS) {
@@ -182,61 +195,41 @@ __device__ __noinline__ bool wait_bar_slow(uint32_t addr, uint32_t parity, bool 
   }
 }
 
-__device__ __forceinline__ bool wait_bar(uint32_t addr, uint32_t parity, bool cluster_scope, volatile uint32_t* abort,
+__device__ __forceinline__ bool wait_bar(uint32_t addr, uint32_t parity, volatile uint32_t* abort,
                                          unsigned int* status, uint32_t peer_abort) {
-  if (cluster_scope) {
-    if (ptx::mbar_try_wait_relaxed_cluster(addr, parity)) {
-      ptx::fence_acq_rel_cluster();
-      return true;
-    }
-  } else if (ptx::mbar_try_wait(addr, parity)) {
-    return true;
-  }
-  return wait_bar_slow(addr, parity, cluster_scope, abort, status, peer_abort);
+  if (ptx::mbar_try_wait(addr, parity)) return true;
+  return wait_bar_slow<false>(addr, parity, abort, status, peer_abort);
+}
+
+__device__ __forceinline__ bool wait_bar_cl(uint32_t addr, uint32_t parity, volatile uint32_t* abort,
+                                            unsigned int* status, uint32_t peer_abort) {
+  if (ptx::mbar_try_wait_acq_cluster(addr, parity)) return true;
+  return wait_bar_slow<true>(addr, parity, abort, status, peer_abort);
 }
 
 // ---------------------------------------------------------------------------------------------
-// Producer: issue the loads of one 64-token tile of request b starting at token tok0 (nv valid
-// rows) into one FP8 stage, completing on `full`.  Rows are loaded in boxes of `boxr` rows, each
-// inside one page; boxes whose page id is out of range are skipped and flagged.
+// Page-table gather: where token `tok` of request b lives (value row and scale).  Out-of-range
+// page ids are reported (false) instead of being dereferenced.
 // ---------------------------------------------------------------------------------------------
-__device__ __forceinline__ bool box_source(const DecodeParams& p, int b, int tok, uint32_t& row, uint32_t& srow) {
+__device__ __forceinline__ bool row_source(const DecodeParams& p, int b, int tok, const uint8_t*& vptr,
+                                           const float*& sptr) {
   const int page = tok / p.P;
   const int slot = tok - page * p.P;
   if (page >= p.max_pages) return false;
-  const uint32_t blk = p.lut[static_cast<size_t>(b) * p.max_pages + page];
-  const uint32_t sblk = p.slut ? p.slut[static_cast<size_t>(b) * p.max_pages + page] : blk;
+  const uint32_t blk = __ldg(p.lut + static_cast<size_t>(b) * p.max_pages + page);
+  const uint32_t sblk = p.slut ? __ldg(p.slut + static_cast<size_t>(b) * p.max_pages + page) : blk;
   if (blk >= static_cast<uint32_t>(p.NB) || sblk >= static_cast<uint32_t>(p.NSB)) return false;
-  row = ((blk * static_cast<uint32_t>(p.KVD)) * p.NL + p.layer) * p.P + slot;
-  srow = ((sblk * static_cast<uint32_t>(p.KVD)) * p.NL + p.layer) * p.P + slot;
+  const size_t row = ((static_cast<size_t>(blk) * p.KVD) * p.NL + p.layer) * p.P + slot;
+  const size_t srow = ((static_cast<size_t>(sblk) * p.KVD) * p.NL + p.layer) * p.P + slot;
+  vptr = p.blocks + row * HEAD_DIM;
+  sptr = p.scales + srow;
   return true;
 }
 
-__device__ __forceinline__ void produce_tile(const DecodeParams& p, const CUtensorMap* tm_lat,
-                                             const CUtensorMap* tm_rope, int c, int b, int tok0, int nv,
-                                             uint32_t stage, uint32_t full) {
-  uint32_t bytes = 0;
-  bool bad = false;
-  for (int r = 0; r < nv; r += p.boxr) {
-    uint32_t row, srow;
-    if (box_source(p, b, tok0 + r, row, srow)) bytes += p.boxr * (256 + 32 + 4);
-    else bad = true;
-  }
-  if (bad) raise_status(p.status, STATUS_BOUNDS);
-  ptx::mbar_arrive_expect_tx(full, bytes);
-  for (int r = 0; r < nv; r += p.boxr) {
-    uint32_t row, srow;
-    if (!box_source(p, b, tok0 + r, row, srow)) continue;
-    ptx::tma_load_2d(stage + r * 256, tm_lat, 256 * c, static_cast<int32_t>(row), full);
-    ptx::tma_load_2d(stage + SF_ROPE + r * 32, tm_rope, 512 + 32 * c, static_cast<int32_t>(row), full);
-    ptx::bulk_load(stage + SF_SC + r * 4, p.scales + srow, p.boxr * 4, full);
-  }
-}
-
 // ---------------------------------------------------------------------------------------------
-// Converter: 16 e4m3 bytes of one row times the row's scale -> 16 bf16 (8 packed words).
-// bf16_rn(f32_rn(e4m3 * s)): the e4m3 -> f16 -> f32 steps are exact, the multiply rounds to
-// nearest in fp32, the pack rounds to nearest-even bf16.
+// Dequantisation of 16 e4m3 bytes of one row with the row's scale -> 16 bf16 (8 packed words):
+// bf16_rn(f32_rn(e4m3 * s)).  e4m3 -> f16 -> f32 is exact; the multiply rounds to nearest in fp32;
+// the pack rounds to nearest-even bf16.
 // ---------------------------------------------------------------------------------------------
 __device__ __forceinline__ void dequant16(uint4 raw, float s, uint32_t (&w)[8]) {
   const uint32_t in[4] = {raw.x, raw.y, raw.z, raw.w};
@@ -253,432 +246,617 @@ __device__ __forceinline__ void dequant16(uint4 raw, float s, uint32_t (&w)[8]) 
   }
 }
 
-// Byte offset of 16-byte unit `u` (0..7) of row `r` in a K-major SWIZZLE_128B region whose
+// Byte offset of 16-byte unit `u` (0..7) of row `r` in a K-major SWIZZLE_128B atom column whose
 // 8-row groups are 1024 B apart.
 __device__ __forceinline__ uint32_t sw128_off(int r, int u) {
   return (r >> 3) * 1024 + (r & 7) * 128 + ((u ^ (r & 7)) << 4);
 }
-// Same for SWIZZLE_64B (64-byte rows, 8-row groups 512 B apart, units 0..3).
-__device__ __forceinline__ uint32_t sw64_off(int r, int u) {
-  return (r >> 3) * 512 + (r & 7) * 64 + ((u ^ ((r & 7) >> 1)) << 4);
+
+__device__ __forceinline__ void st_chunk(uint32_t atom_base, int row, int u0, const uint32_t (&w)[8]) {
+  ptx::st_shared_v4(atom_base + sw128_off(row, u0), w[0], w[1], w[2], w[3]);
+  ptx::st_shared_v4(atom_base + sw128_off(row, u0 + 1), w[4], w[5], w[6], w[7]);
 }
 
-// Convert one FP8 stage (this CTA's 288 dims of 64 rows) into a bf16 K tile; rows >= nv become 0.
-// Called by 128 threads (t = 0..127).
-__device__ __forceinline__ void convert_tile(int t, uint32_t stage, uint32_t ktile, int nv) {
-  uint4 raw[9];
-  float sc[9];
+// The FP8 bytes of one tile that one converter thread converts.  Thread t (of 256) owns row t >> 3
+// of both key halves and the 16-byte chunks (t & 7) + 8k:
+//   own key   32c + row    : the 36 chunks of its 576-byte row (576 dims) -> K half buffer; its D_c
+//                            chunks also -> V buffer
+//   other key 32(1-c) + row: the 16 chunks of D_c -> V buffer
+struct RawTile {
+  uint4 own[5];
+  uint4 oth[2];
+  float so, sp;
+  bool own_ok, oth_ok;
+};
+
+// Three phases so that the page-table reads and the data reads of later tiles overlap the
+// conversion of the current one:
+//   lut_issue : read the page-table entries of thread t's two keys of tile j (request b)
+//   lut_finish: turn them into row pointers (ids past the pool are flagged; that key reads as zero)
+//   fetch     : issue the 16-byte loads of those rows and their scales
+struct LutVals {
+  uint32_t ob, osb, pb, psb;       // value / scale block ids of the own and other key
+  int otok, ptok;
+  bool own_in, oth_in;             // key inside the visible length and its page inside the table
+  bool bad;
+};
+
+struct TilePtrs {
+  const uint8_t* ov;
+  const float* os;
+  const uint8_t* pv;
+  const float* ps;
+  bool own_ok, oth_ok;
+};
+
+__device__ __forceinline__ LutVals lut_issue(const DecodeParams& p, int c, int t, int b, int nvis, int j) {
+  const int row = t >> 3;
+  LutVals V;
+  V.otok = j * BN + HALF_BN * c + row;
+  V.ptok = j * BN + HALF_BN * (1 - c) + row;
+  V.bad = false;
+  const uint32_t* lrow = p.lut + static_cast<size_t>(b) * p.max_pages;
+  const uint32_t* srow = p.slut ? p.slut + static_cast<size_t>(b) * p.max_pages : lrow;
+  const int opage = V.otok / p.P, ppage = V.ptok / p.P;
+  V.own_in = V.otok < nvis;
+  V.oth_in = V.ptok < nvis;
+  if (V.own_in && opage >= p.max_pages) { V.own_in = false; V.bad = true; }
+  if (V.oth_in && ppage >= p.max_pages) { V.oth_in = false; V.bad = true; }
+  V.ob = V.osb = V.pb = V.psb = 0;
+  if (V.own_in) { V.ob = __ldg(lrow + opage); V.osb = __ldg(srow + opage); }
+  if (V.oth_in) { V.pb = __ldg(lrow + ppage); V.psb = __ldg(srow + ppage); }
+  return V;
+}
+
+__device__ __forceinline__ TilePtrs lut_finish(const DecodeParams& p, const LutVals& V, bool& bad) {
+  TilePtrs T;
+  bad = V.bad;
+  T.own_ok = V.own_in && V.ob < static_cast<uint32_t>(p.NB) && V.osb < static_cast<uint32_t>(p.NSB);
+  T.oth_ok = V.oth_in && V.pb < static_cast<uint32_t>(p.NB) && V.psb < static_cast<uint32_t>(p.NSB);
+  if (V.own_in && !T.own_ok) bad = true;
+  if (V.oth_in && !T.oth_ok) bad = true;
+  const int oslot = V.otok % p.P, pslot = V.ptok % p.P;
+  const size_t lay = static_cast<size_t>(p.layer);
+  T.ov = p.blocks + (((static_cast<size_t>(V.ob) * p.KVD) * p.NL + lay) * p.P + oslot) * HEAD_DIM;
+  T.os = p.scales + ((static_cast<size_t>(V.osb) * p.KVD) * p.NL + lay) * p.P + oslot;
+  T.pv = p.blocks + (((static_cast<size_t>(V.pb) * p.KVD) * p.NL + lay) * p.P + pslot) * HEAD_DIM;
+  T.ps = p.scales + ((static_cast<size_t>(V.psb) * p.KVD) * p.NL + lay) * p.P + pslot;
+  return T;
+}
+
+__device__ __forceinline__ void fetch(const TilePtrs& T, int c, int t, RawTile& R) {
+  const int q = t & 7;
+  R.own_ok = T.own_ok;
+  R.oth_ok = T.oth_ok;
+  if (T.own_ok) {
+    R.so = __ldg(T.os);
 #pragma unroll
-  for (int it = 0; it < 8; ++it) {
-    const int id = it * 128 + t;
-    const int row = id >> 4, cc = id & 15;
-    raw[it] = ptx::ld_shared_v4(stage + row * 256 + cc * 16);
-    sc[it] = ptx::ld_shared_f32(stage + SF_SC + row * 4);
-  }
-  raw[8] = ptx::ld_shared_v4(stage + SF_ROPE + (t >> 1) * 32 + (t & 1) * 16);
-  sc[8] = ptx::ld_shared_f32(stage + SF_SC + (t >> 1) * 4);
-#pragma unroll
-  for (int it = 0; it < 8; ++it) {
-    const int id = it * 128 + t;
-    const int row = id >> 4, cc = id & 15;
-    uint32_t w[8];
-    dequant16(raw[it], sc[it], w);
-    if (row >= nv) {
-#pragma unroll
-      for (int k = 0; k < 8; ++k) w[k] = 0u;
+    for (int k = 0; k < 5; ++k) {
+      const int qq = q + 8 * k;
+      if (qq < 36) R.own[k] = ptx::ldg_stream_v4(T.ov + 16 * qq);
     }
-    const uint32_t base = ktile + (cc >> 2) * 8192;
-    const int u0 = (cc & 3) * 2;
-    ptx::st_shared_v4(base + sw128_off(row, u0), w[0], w[1], w[2], w[3]);
-    ptx::st_shared_v4(base + sw128_off(row, u0 + 1), w[4], w[5], w[6], w[7]);
   }
-  {
-    const int row = t >> 1, cc = t & 1;
-    uint32_t w[8];
-    dequant16(raw[8], sc[8], w);
-    if (row >= nv) {
+  if (T.oth_ok) {
+    R.sp = __ldg(T.ps);
 #pragma unroll
-      for (int k = 0; k < 8; ++k) w[k] = 0u;
+    for (int k = 0; k < 2; ++k) {
+      const int jc = q + 8 * k;                              // chunk index within D_c (0..15)
+      const int qq = jc < 8 ? 8 * c + jc : 16 + 8 * c + (jc - 8);
+      R.oth[k] = ptx::ldg_stream_v4(T.pv + 16 * qq);
     }
-    const uint32_t base = ktile + SK_ROPE;
-    ptx::st_shared_v4(base + sw64_off(row, cc * 2), w[0], w[1], w[2], w[3]);
-    ptx::st_shared_v4(base + sw64_off(row, cc * 2 + 1), w[4], w[5], w[6], w[7]);
   }
 }
 
-// Q rows of one item, this CTA's 288 dims, into the SW128 / SW64 K-major layout. Rows >= H are 0.
+// All three phases at once (for callers with nothing to overlap).  Returns false on a bad page id.
+__device__ __forceinline__ bool load_tile(const DecodeParams& p, int c, int t, int b, int nvis, int j, RawTile& R) {
+  bool bad;
+  const TilePtrs T = lut_finish(p, lut_issue(p, c, t, b, nvis, j), bad);
+  fetch(T, c, t, R);
+  return !bad;
+}
+
+// Dequantises thread t's part of a loaded tile into the K half buffer `sk` and the V buffer `sv`.
+__device__ __forceinline__ void store_tile(int c, int t, const RawTile& R, uint32_t sk, uint32_t sv) {
+  const int row = t >> 3, q = t & 7;
+  const int vrow_own = HALF_BN * c + row;
+  const int vrow_oth = HALF_BN * (1 - c) + row;
+#pragma unroll
+  for (int k = 0; k < 5; ++k) {
+    const int qq = q + 8 * k;                                // chunk of the 576-byte row
+    if (qq >= 36) continue;
+    uint32_t w[8];
+    if (R.own_ok) {
+      dequant16(R.own[k], R.so, w);
+    } else {
+#pragma unroll
+      for (int x = 0; x < 8; ++x) w[x] = 0u;
+    }
+    st_chunk(sk + (qq >> 2) * SK_ATOM, row, (qq & 3) * 2, w);
+    const int blk128 = qq >> 3;                              // 128-dim block of the latent
+    if (blk128 == c || blk128 == 2 + c) {
+      const int jc = (qq & 7) + (blk128 >= 2 ? 8 : 0);
+      st_chunk(sv + (jc >> 2) * SV_ATOM, vrow_own, (jc & 3) * 2, w);
+    }
+  }
+#pragma unroll
+  for (int k = 0; k < 2; ++k) {
+    const int jc = q + 8 * k;
+    uint32_t w[8];
+    if (R.oth_ok) {
+      dequant16(R.oth[k], R.sp, w);
+    } else {
+#pragma unroll
+      for (int x = 0; x < 8; ++x) w[x] = 0u;
+    }
+    st_chunk(sv + (jc >> 2) * SV_ATOM, vrow_oth, (jc & 3) * 2, w);
+  }
+}
+
+// Sequential cursor over the tiles a cluster processes (unit by unit).
+struct TileCursor {
+  UnitWalker wk;
+  Unit u;
+  int j;
+  bool valid, first;
+  __device__ TileCursor(const DecodeParams& p, int k) : wk(p, k) {
+    valid = wk.next(u);
+    j = valid ? u.tb : 0;
+    first = true;
+  }
+  __device__ void advance() {
+    ++j;
+    first = false;
+    if (j >= u.te) {
+      valid = wk.next(u);
+      j = valid ? u.tb : 0;
+      first = true;
+    }
+  }
+};
+
+// Q rows 64c..64c+63 of an item's head group (all 576 dims) into the SW128 K-major layout, by the
+// 256 converter threads.  Rows whose head index is >= H are zero.
 __device__ __forceinline__ void load_q(const DecodeParams& p, const Unit& u, int c, int t, uint32_t sq) {
   const uint16_t* qrow0 = p.q + (static_cast<size_t>(u.b) * p.T + u.i) * p.H * HEAD_DIM;
-  const int h0 = u.g * MROWS;
+  const int h0 = u.g * MROWS + HPC * c;
 #pragma unroll 1
-  for (int batch = 0; batch < 3; ++batch) {
-    uint4 v[12];
+  for (int batch = 0; batch < 2; ++batch) {
+    uint4 v[9];
 #pragma unroll
-    for (int k = 0; k < 12; ++k) {
-      const int id = (batch * 12 + k) * 128 + t;
-      const int row = id / 36, cc = id - row * 36;
-      const int col = cc < 32 ? 256 * c + cc * 8 : 512 + 32 * c + (cc - 32) * 8;
+    for (int k = 0; k < 9; ++k) {
+      const int id = (batch * 9 + k) * CONV_THREADS + t;   // 64 rows x 72 chunks of 8 bf16
+      const int row = id / 72, cc = id - row * 72;
       v[k] = make_uint4(0, 0, 0, 0);
       if (h0 + row < p.H)
-        v[k] = __ldg(reinterpret_cast<const uint4*>(qrow0 + static_cast<size_t>(h0 + row) * HEAD_DIM + col));
+        v[k] = __ldg(reinterpret_cast<const uint4*>(qrow0 + static_cast<size_t>(h0 + row) * HEAD_DIM + cc * 8));
     }
 #pragma unroll
-    for (int k = 0; k < 12; ++k) {
-      const int id = (batch * 12 + k) * 128 + t;
-      const int row = id / 36, cc = id - row * 36;
-      const uint32_t dst = cc < 32 ? sq + SQ_LAT + (cc >> 3) * 16384 + sw128_off(row, cc & 7)
-                                   : sq + SQ_ROPE + sw64_off(row, cc - 32);
-      ptx::st_shared_v4(dst, v[k].x, v[k].y, v[k].z, v[k].w);
+    for (int k = 0; k < 9; ++k) {
+      const int id = (batch * 9 + k) * CONV_THREADS + t;
+      const int row = id / 72, cc = id - row * 72;
+      ptx::st_shared_v4(sq + SQ + (cc >> 3) * SQ_ATOM + sw128_off(row, cc & 7), v[k].x, v[k].y, v[k].z, v[k].w);
     }
+  }
+}
+
+// L2 prefetch of the value rows and scales of CTA c's own keys of tile j (whole page runs).
+__device__ __forceinline__ void prefetch_tile(const DecodeParams& p, int c, int b, int nvis, int j) {
+  const int first = j * BN + HALF_BN * c;
+  int tok = first;
+  const int end = min(first + HALF_BN, nvis);
+  while (tok < end) {
+    const int page = tok / p.P;
+    const int slot = tok - page * p.P;
+    const int run = min(end - tok, p.P - slot);
+    const uint8_t* vptr;
+    const float* sptr;
+    if (row_source(p, b, tok, vptr, sptr)) {
+      ptx::prefetch_l2(vptr, static_cast<uint32_t>(run) * HEAD_DIM);
+      // the whole page's scale run (P * 4 bytes, 64-byte aligned because P % 16 == 0)
+      if (slot == 0 || tok == first) ptx::prefetch_l2(sptr - slot, static_cast<uint32_t>(p.P) * 4);
+    }
+    tok += run;
   }
 }
 
 // =============================================================================================
 // decode kernel
 // =============================================================================================
-__global__ void __launch_bounds__(NUM_THREADS, 1)
-mla_decode_kernel(const __grid_constant__ DecodeParams p, const __grid_constant__ CUtensorMap tm_lat,
-                  const __grid_constant__ CUtensorMap tm_rope) {
+__global__ void __launch_bounds__(NUM_THREADS, 1) mla_decode_kernel(const __grid_constant__ DecodeParams p) {
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  const Smem S{ptx::smem_u32(smem)};
+  const uint32_t base = ptx::smem_u32(smem);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const uint32_t c = ptx::cluster_ctarank();
   const uint32_t peer = c ^ 1u;
   const int k = static_cast<int>(ptx::cluster_id_x());
-  volatile uint32_t* abort = abort_flag(smem);
-  const uint32_t peer_abort = ptx::mapa(S.base + S_ABORT, peer);
+  volatile uint32_t* abort = reinterpret_cast<volatile uint32_t*>(smem + S_ABORT);
+  volatile uint32_t* conv_tile = reinterpret_cast<volatile uint32_t*>(smem + S_CONV_TILE);
+  const uint32_t peer_abort = ptx::mapa(base + S_ABORT, peer);
+#define BAR(i) (base + SBAR + 8u * (i))
 
   if (threadIdx.x == 0) {
-    ptx::mbar_init(S.bar(B_FP8_FULL + 0), 1);
-    ptx::mbar_init(S.bar(B_FP8_FULL + 1), 1);
-    ptx::mbar_init(S.bar(B_FP8_EMPTY + 0), 128);
-    ptx::mbar_init(S.bar(B_FP8_EMPTY + 1), 128);
-    ptx::mbar_init(S.bar(B_K_FULL + 0), 128);
-    ptx::mbar_init(S.bar(B_K_FULL + 1), 128);
-    ptx::mbar_init(S.bar(B_K_EMPTY + 0), 1);
-    ptx::mbar_init(S.bar(B_K_EMPTY + 1), 1);
-    ptx::mbar_init(S.bar(B_S_FULL + 0), 1);
-    ptx::mbar_init(S.bar(B_S_FULL + 1), 1);
-    ptx::mbar_init(S.bar(B_P_FULL + 0), 128);
-    ptx::mbar_init(S.bar(B_P_FULL + 1), 128);
-    ptx::mbar_init(S.bar(B_O_DONE + 0), 1);
-    ptx::mbar_init(S.bar(B_O_DONE + 1), 1);
-    ptx::mbar_init(S.bar(B_O_FREE), 128);
-    ptx::mbar_init(S.bar(B_Q_FULL), 128);
-    ptx::mbar_init(S.bar(B_Q_FREE), 1);
-    ptx::mbar_init(S.bar(B_XS_FULL), 128);
-    ptx::mbar_init(S.bar(B_XS_FREE), 128);
-    ptx::mbar_init(S.bar(B_DRAIN), 1);
+    for (uint32_t i = 0; i < 2; ++i) {
+      ptx::mbar_init(BAR(B_KV_FULL + i), 2 * CONV_WARPS);
+      ptx::mbar_init(BAR(B_PV_DONE + i), 1);
+      ptx::mbar_init(BAR(B_S_FULL + i), 1);
+      ptx::mbar_init(BAR(B_P_FULL + i), 8);
+    }
+    ptx::mbar_init(BAR(B_Q_FULL), 2 * CONV_WARPS);
+    ptx::mbar_init(BAR(B_Q_FREE), 1);
+    ptx::mbar_init(BAR(B_O_FREE), 8);
+    ptx::mbar_init(BAR(B_DRAIN), 1);
+    ptx::mbar_init(BAR(B_RED + 0), 4);
+    ptx::mbar_init(BAR(B_RED + 1), 4);
+    ptx::mbar_init(BAR(B_REDL), 4);
     *abort = 0u;
+    *conv_tile = 0u;
     ptx::fence_mbar_init();
   }
-  if (warp == 8 && lane == 0) {
-    ptx::prefetch_tmap(&tm_lat);
-    ptx::prefetch_tmap(&tm_rope);
-  }
-  if (warp == 9) {
-    ptx::tmem_alloc(S.base + S_TMEM_BASE, TMEM_COLS);
-    ptx::tmem_relinquish();
+  if (warp == MMA_WARP) {
+    ptx::tmem_alloc_pair(base + S_TMEM_BASE, TMEM_COLS);
+    ptx::tmem_relinquish_pair();
   }
   ptx::tc_fence_before();
   __syncthreads();
-  ptx::tc_fence_after();
   ptx::cluster_sync();   // the peer's barriers exist before any remote arrive
+  ptx::tc_fence_after();
   const uint32_t tbase = *reinterpret_cast<volatile uint32_t*>(smem + S_TMEM_BASE);
 
-// Single-thread roles bail out alone; whole-warp roles bail out together so that the
-// warp-collective tcgen05 instructions after a wait never run on a partial warp.
-#define MLA_WAIT(bar, parity, cl)                                                    \
-  if (!wait_bar((bar), (parity), (cl), abort, p.status, peer_abort)) goto role_done;
-#define MLA_WAIT_WARP(bar, parity, cl)                                               \
-  if (!__all_sync(0xffffffffu, wait_bar((bar), (parity), (cl), abort, p.status, peer_abort))) goto role_done;
+// Whole-warp roles bail out together so that the warp-collective instructions after a wait never
+// run on a partial warp.
+#define MLA_WAIT_WARP(b_, parity)                                                              \
+  if (!__all_sync(0xffffffffu, wait_bar((b_), (parity), abort, p.status, peer_abort))) goto role_done;
+#define MLA_WAIT_WARP_CL(b_, parity)                                                           \
+  if (!__all_sync(0xffffffffu, wait_bar_cl((b_), (parity), abort, p.status, peer_abort))) goto role_done;
 
-  if (warp < 4) {
+  if (warp < CONV_WARPS) {
     // ------------------------------------------------------------------ converter
+    // Software pipeline over the tile sequence: while tile g is converted, the FP8 bytes of tile g+1
+    // are in flight and the page-table entries of tile g+2 are being read.
     const int t = threadIdx.x;
+    const int cc = static_cast<int>(c);
+    const uint32_t kv_full0 = ptx::mapa(BAR(B_KV_FULL), 0), q_full = ptx::mapa(BAR(B_Q_FULL), 0);
+    TileCursor cur(p, k);
+    if (cur.valid) {
+      TileCursor n1 = cur;
+      n1.advance();
+      TileCursor n2 = n1;
+      if (n2.valid) n2.advance();
+      RawTile ra, rb;
+      bool bad = false;
+      {
+        const TilePtrs t0 = lut_finish(p, lut_issue(p, cc, t, cur.u.b, cur.u.nvis, cur.j), bad);
+        if (bad) raise_status(p.status, STATUS_BOUNDS);
+        fetch(t0, cc, t, ra);
+      }
+      TilePtrs t1{};
+      if (n1.valid) {
+        t1 = lut_finish(p, lut_issue(p, cc, t, n1.u.b, n1.u.nvis, n1.j), bad);
+        if (bad) raise_status(p.status, STATUS_BOUNDS);
+      }
+      uint32_t g = 0, uu = 0;
+      // One tile.  Unrolled twice below so that the two register sets alternate statically.
+#define MLA_CONV_STEP(RCUR, RNXT)                                                                        \
+      {                                                                                                  \
+        if (cur.first) {                                                                                 \
+          MLA_WAIT_WARP(BAR(B_Q_FREE), (uu & 1) ^ 1);                                                    \
+          if (t == 0) MLA_TRACE_EV(g, 3);                                                                \
+          load_q(p, cur.u, cc, t, base);                                                                 \
+          ptx::fence_proxy_async_smem();                                                                 \
+          __syncwarp();                                                                                  \
+          if (lane == 0) ptx::mbar_arrive_remote(q_full);                                                \
+          ++uu;                                                                                          \
+        }                                                                                                \
+        const uint32_t kb = g & 1;                                                                       \
+        MLA_WAIT_WARP(BAR(B_PV_DONE + kb), ((g >> 1) & 1) ^ 1);                                          \
+        if (t == 0) MLA_TRACE_EV(g, 1);                                                                  \
+        if (n1.valid) fetch(t1, cc, t, RNXT);                                                            \
+        LutVals v2{};                                                                                    \
+        if (n2.valid) v2 = lut_issue(p, cc, t, n2.u.b, n2.u.nvis, n2.j);                                 \
+        if (t == 0) MLA_TRACE_EV(g, 4);                                                                  \
+        store_tile(cc, t, RCUR, base + SK0 + kb * SK_STRIDE, base + SV0 + kb * SV_STRIDE);               \
+        ptx::fence_proxy_async_smem();                                                                   \
+        __syncwarp();                                                                                    \
+        if (lane == 0) ptx::mbar_arrive_remote(kv_full0 + 8u * kb);                                      \
+        if (t == 0) {                                                                                    \
+          *conv_tile = g + 1;                                                                            \
+          MLA_TRACE_EV(g, 2);                                                                            \
+        }                                                                                                \
+        if (n2.valid) {                                                                                  \
+          t1 = lut_finish(p, v2, bad);                                                                   \
+          if (bad) raise_status(p.status, STATUS_BOUNDS);                                                \
+        }                                                                                                \
+        ++g;                                                                                             \
+      }
+      while (true) {
+        MLA_CONV_STEP(ra, rb)
+        if (!n1.valid) break;
+        cur = n1;
+        n1 = n2;
+        if (n2.valid) n2.advance();
+        MLA_CONV_STEP(rb, ra)
+        if (!n1.valid) break;
+        cur = n1;
+        n1 = n2;
+        if (n2.valid) n2.advance();
+      }
+#undef MLA_CONV_STEP
+    }
+  } else if (warp < SM_WARP0 + 4) {
+    // ------------------------------------------------------------------ softmax / epilogue
+    const int t = threadIdx.x - 32 * SM_WARP0;
+    const int quad = warp - SM_WARP0;
+    const int r = t & 63, hh = t >> 6;             // head row within the CTA, key half of the tile
+    const uint32_t lane_base = tbase + (static_cast<uint32_t>(quad * 32) << 16);
+    const uint32_t p_full0 = ptx::mapa(BAR(B_P_FULL), 0), o_free = ptx::mapa(BAR(B_O_FREE), 0);
+    volatile float* red_max = reinterpret_cast<volatile float*>(smem + SRED);
+    volatile float* red_l = reinterpret_cast<volatile float*>(smem + SRED + 1024);
     UnitWalker wk(p, k);
     Unit u;
     uint32_t g = 0, uu = 0;
     while (wk.next(u)) {
-      MLA_WAIT_WARP(S.bar(B_Q_FREE), (uu & 1) ^ 1, false);
-      if (t == 0) MLA_TRACE_EV(g, 3);
-      load_q(p, u, c, t, S.base);
-      ptx::fence_proxy_async_smem();
-      ptx::mbar_arrive(S.bar(B_Q_FULL));
-      if (t == 0) MLA_TRACE_EV(g, 4);
-      for (int j = u.tb; j < u.te; ++j, ++g) {
-        const uint32_t s = g & 1, ph = (g >> 1) & 1;
-        MLA_WAIT_WARP(S.bar(B_FP8_FULL + s), ph, false);
-        if (t == 0) MLA_TRACE_EV(g, 0);
-        MLA_WAIT_WARP(S.bar(B_K_EMPTY + s), ph ^ 1, false);
-        if (t == 0) MLA_TRACE_EV(g, 1);
-        const int nv = min(BN, u.nvis - j * BN);
-        convert_tile(t, S.base + SF0 + s * SF_STRIDE, S.base + SK0 + s * SK_STRIDE, nv);
-        ptx::fence_proxy_async_smem();
-        ptx::mbar_arrive(S.bar(B_FP8_EMPTY + s));
-        ptx::mbar_arrive(S.bar(B_K_FULL + s));
-        if (t == 0) MLA_TRACE_EV(g, 2);
-      }
-      ++uu;
-    }
-  } else if (warp < 8) {
-    // ------------------------------------------------------------------ softmax / epilogue
-    const int h = threadIdx.x - 128;
-    const int quad = warp - 4;
-    const uint32_t lane_base = tbase + (static_cast<uint32_t>(quad * 32) << 16);
-    const uint32_t xrow_local = S.base + SX + h * 16;
-    const uint32_t xrow_peer = ptx::mapa(xrow_local, peer);
-    const uint32_t xs_full_peer = ptx::mapa(S.bar(B_XS_FULL), peer);
-    const uint32_t xs_free_peer = ptx::mapa(S.bar(B_XS_FREE), peer);
-    UnitWalker wk(p, k);
-    Unit u;
-    uint32_t g = 0, e = 0;
-    while (wk.next(u)) {
       float m_ref = -INFINITY, l = 0.f;
-      for (int j = u.tb; j < u.te; ++j, ++g, ++e) {
+      for (int j = u.tb; j < u.te; ++j, ++g) {
         const uint32_t sb = g & 1;
-        MLA_WAIT_WARP(S.bar(B_S_FULL + sb), (g >> 1) & 1, false);
-        if (h == 0) MLA_TRACE_EV(g, 8);
+        MLA_WAIT_WARP(BAR(B_S_FULL + sb), (g >> 1) & 1);
+        if (t == 0) MLA_TRACE_EV(g, 8);
         ptx::tc_fence_after();
-        float x[BN];
+        float x[32];
         {
-          uint32_t r[32];
-          ptx::tmem_ld32(lane_base + T_S + 64 * sb, r);
+          uint32_t rr[32];
+          ptx::tmem_ld32(lane_base + T_S + 32 * sb, rr);
           ptx::tmem_wait_ld();
 #pragma unroll
-          for (int q = 0; q < 32; ++q) x[q] = __uint_as_float(r[q]);
-          ptx::tmem_ld32(lane_base + T_S + 64 * sb + 32, r);
-          ptx::tmem_wait_ld();
-#pragma unroll
-          for (int q = 0; q < 32; ++q) x[32 + q] = __uint_as_float(r[q]);
+          for (int q = 0; q < 32; ++q) x[q] = __uint_as_float(rr[q]);
         }
-        if (h == 0) MLA_TRACE_EV(g, 9);
-        // exchange partial scores with the peer CTA (it holds the other 288 dims)
-        MLA_WAIT_WARP(S.bar(B_XS_FREE), (e & 1) ^ 1, true);
-        if (h == 0) MLA_TRACE_EV(g, 10);
-#pragma unroll
-        for (int v = 0; v < 16; ++v)
-          ptx::st_cluster_v4(xrow_peer + v * SX_CHUNK, x[4 * v], x[4 * v + 1], x[4 * v + 2], x[4 * v + 3]);
-        ptx::mbar_arrive_remote(xs_full_peer);
-        if (h == 0) MLA_TRACE_EV(g, 11);
-        MLA_WAIT_WARP(S.bar(B_XS_FULL), e & 1, true);
-        if (h == 0) MLA_TRACE_EV(g, 12);
-#pragma unroll
-        for (int v = 0; v < 16; ++v) {
-          const uint4 o = ptx::ld_shared_v4(xrow_local + v * SX_CHUNK);
-          x[4 * v] += __uint_as_float(o.x);
-          x[4 * v + 1] += __uint_as_float(o.y);
-          x[4 * v + 2] += __uint_as_float(o.z);
-          x[4 * v + 3] += __uint_as_float(o.w);
-        }
-        ptx::mbar_arrive_remote(xs_free_peer);
-        if (h == 0) MLA_TRACE_EV(g, 13);
-        // online softmax in the log2 domain
-        const int nv = min(BN, u.nvis - j * BN);
+        if (t == 0) MLA_TRACE_EV(g, 9);
+        const int nv = min(BN, u.nvis - j * BN) - HALF_BN * hh;   // valid keys in this lane's half
         float mt = -INFINITY;
 #pragma unroll
-        for (int q = 0; q < BN; ++q) {
+        for (int q = 0; q < 32; ++q) {
           x[q] = (q < nv) ? x[q] * p.scale_log2 : -INFINITY;
           mt = fmaxf(mt, x[q]);
         }
+        // the other half of this head row lives in lane t ^ 64 (another warp of this warpgroup)
+        red_max[sb * 128 + t] = mt;
+        __syncwarp();
+        if (lane == 0) ptx::mbar_arrive(BAR(B_RED + sb));
+        MLA_WAIT_WARP(BAR(B_RED + sb), (g >> 1) & 1);
+        mt = fmaxf(mt, red_max[sb * 128 + (t ^ 64)]);
+        if (t == 0) MLA_TRACE_EV(g, 10);
         float alpha = 1.f;
         bool rescale = false;
         if (mt > m_ref + 8.f) {           // lazy max: keep the reference unless it grows by > 2^8
-          const float m_new = mt;
-          alpha = (m_ref == -INFINITY) ? 0.f : ptx::ex2_approx(m_ref - m_new);
+          alpha = (m_ref == -INFINITY) ? 0.f : ptx::ex2_approx(m_ref - mt);
           l *= alpha;
           rescale = (j != u.tb);
-          m_ref = m_new;
+          m_ref = mt;
         }
         float lsum = 0.f;
-        uint32_t pw[32];
+        uint32_t pw[16];
 #pragma unroll
-        for (int q = 0; q < 32; ++q) {
+        for (int q = 0; q < 16; ++q) {
           const float p0 = ptx::ex2_approx(x[2 * q] - m_ref);
           const float p1 = ptx::ex2_approx(x[2 * q + 1] - m_ref);
           lsum += p0 + p1;
           pw[q] = ptx::pack_bf16x2(p0, p1);
         }
         l += lsum;
-        ptx::tmem_st32(lane_base + T_S + 64 * sb, pw);
-        // the O rescale uses warp-collective TMEM access: a warp rescales when any of its rows
-        // moved its reference max (rows that did not move have alpha == 1)
+        if (t == 0) MLA_TRACE_EV(g, 11);
+        {
+          const uint32_t sp = base + SP0 + sb * SP_STRIDE;
+#pragma unroll
+          for (int v = 0; v < 4; ++v)
+            ptx::st_shared_v4(sp + sw128_off(r, 4 * hh + v), pw[4 * v], pw[4 * v + 1], pw[4 * v + 2], pw[4 * v + 3]);
+        }
+        // O rescale (warp-collective TMEM access): a warp rescales when any of its rows moved its
+        // reference max; rows that did not move use alpha = 1
         if (!rescale) alpha = 1.f;
         if (__any_sync(0xffffffffu, rescale)) {
           const uint32_t gp = g - 1;
-          MLA_WAIT_WARP(S.bar(B_O_DONE + (gp & 1)), (gp >> 1) & 1, false);
+          MLA_WAIT_WARP(BAR(B_PV_DONE + (gp & 1)), (gp >> 1) & 1);
           ptx::tc_fence_after();
 #pragma unroll 1
           for (int ch = 0; ch < 8; ++ch) {
-            uint32_t r[32];
-            ptx::tmem_ld32(lane_base + T_O + 32 * ch, r);
+            uint32_t rr[32];
+            ptx::tmem_ld32(lane_base + T_O + 32 * ch, rr);
             ptx::tmem_wait_ld();
 #pragma unroll
-            for (int q = 0; q < 32; ++q) r[q] = __float_as_uint(__uint_as_float(r[q]) * alpha);
-            ptx::tmem_st32(lane_base + T_O + 32 * ch, r);
+            for (int q = 0; q < 32; ++q) rr[q] = __float_as_uint(__uint_as_float(rr[q]) * alpha);
+            ptx::tmem_st32(lane_base + T_O + 32 * ch, rr);
           }
+          ptx::tmem_wait_st();
         }
-        ptx::tmem_wait_st();
+        ptx::fence_proxy_async_smem();
         ptx::tc_fence_before();
-        ptx::mbar_arrive(S.bar(B_P_FULL + sb));
-        if (h == 0) MLA_TRACE_EV(g, 14);
+        __syncwarp();
+        if (lane == 0) ptx::mbar_arrive_remote(p_full0 + 8u * sb);
+        if (t == 0) MLA_TRACE_EV(g, 14);
       }
-      // epilogue: O / l
+      // epilogue: O / l for this lane's 256 V dims of head row r
       {
         const uint32_t gl = g - 1;
-        MLA_WAIT_WARP(S.bar(B_O_DONE + (gl & 1)), (gl >> 1) & 1, false);
+        MLA_WAIT_WARP(BAR(B_PV_DONE + (gl & 1)), (gl >> 1) & 1);
         ptx::tc_fence_after();
-        const float inv_l = 1.f / l;
-        const int head = u.g * MROWS + h;
+        red_l[t] = l;
+        __syncwarp();
+        if (lane == 0) ptx::mbar_arrive(BAR(B_REDL));
+        MLA_WAIT_WARP(BAR(B_REDL), uu & 1);
+        const float l_row = l + red_l[t ^ 64];
+        const float inv_l = 1.f / l_row;
+        const int head = u.g * MROWS + HPC * static_cast<int>(c) + r;
         const bool row_ok = head < p.H;
-        const float lse_v = (m_ref + ptx::lg2_approx(l)) * 0.69314718055994530942f;
+        const float lse_v = (m_ref + ptx::lg2_approx(l_row)) * 0.69314718055994530942f;
 #pragma unroll 1
         for (int ch = 0; ch < 8; ++ch) {
-          uint32_t r[32];
-          ptx::tmem_ld32(lane_base + T_O + 32 * ch, r);
+          uint32_t rr[32];
+          ptx::tmem_ld32(lane_base + T_O + 32 * ch, rr);
           ptx::tmem_wait_ld();
           if (!row_ok) continue;
+          const int dv = (ch < 4 ? 0 : 256) + 128 * hh + 32 * (ch & 3);
           if (u.slot < 0) {
-            uint16_t* dst = p.out + ((static_cast<size_t>(u.b) * p.T + u.i) * p.H + head) * V_DIM + 256 * c + 32 * ch;
+            uint16_t* dst = p.out + ((static_cast<size_t>(u.b) * p.T + u.i) * p.H + head) * V_DIM + dv;
 #pragma unroll
             for (int v = 0; v < 4; ++v) {
               uint4 w;
-              w.x = ptx::pack_bf16x2(__uint_as_float(r[8 * v + 0]) * inv_l, __uint_as_float(r[8 * v + 1]) * inv_l);
-              w.y = ptx::pack_bf16x2(__uint_as_float(r[8 * v + 2]) * inv_l, __uint_as_float(r[8 * v + 3]) * inv_l);
-              w.z = ptx::pack_bf16x2(__uint_as_float(r[8 * v + 4]) * inv_l, __uint_as_float(r[8 * v + 5]) * inv_l);
-              w.w = ptx::pack_bf16x2(__uint_as_float(r[8 * v + 6]) * inv_l, __uint_as_float(r[8 * v + 7]) * inv_l);
+              w.x = ptx::pack_bf16x2(__uint_as_float(rr[8 * v + 0]) * inv_l, __uint_as_float(rr[8 * v + 1]) * inv_l);
+              w.y = ptx::pack_bf16x2(__uint_as_float(rr[8 * v + 2]) * inv_l, __uint_as_float(rr[8 * v + 3]) * inv_l);
+              w.z = ptx::pack_bf16x2(__uint_as_float(rr[8 * v + 4]) * inv_l, __uint_as_float(rr[8 * v + 5]) * inv_l);
+              w.w = ptx::pack_bf16x2(__uint_as_float(rr[8 * v + 6]) * inv_l, __uint_as_float(rr[8 * v + 7]) * inv_l);
               reinterpret_cast<uint4*>(dst)[v] = w;
             }
           } else {
-            float* dst = p.part_o + (static_cast<size_t>(u.slot) * MROWS + h) * V_DIM + 256 * c + 32 * ch;
+            float* dst = p.part_o + (static_cast<size_t>(u.slot) * MROWS + HPC * c + r) * V_DIM + dv;
 #pragma unroll
             for (int v = 0; v < 8; ++v) {
-              float4 w = make_float4(__uint_as_float(r[4 * v]) * inv_l, __uint_as_float(r[4 * v + 1]) * inv_l,
-                                     __uint_as_float(r[4 * v + 2]) * inv_l, __uint_as_float(r[4 * v + 3]) * inv_l);
+              const float4 w = make_float4(__uint_as_float(rr[4 * v]) * inv_l, __uint_as_float(rr[4 * v + 1]) * inv_l,
+                                           __uint_as_float(rr[4 * v + 2]) * inv_l,
+                                           __uint_as_float(rr[4 * v + 3]) * inv_l);
               reinterpret_cast<float4*>(dst)[v] = w;
             }
           }
         }
-        if (c == 0 && row_ok) {
+        if (hh == 0 && row_ok) {
           if (u.slot < 0) {
             if (p.lse) p.lse[(static_cast<size_t>(u.b) * p.T + u.i) * p.H + head] = lse_v;
           } else {
-            p.part_lse[static_cast<size_t>(u.slot) * MROWS + h] = lse_v;
+            p.part_lse[static_cast<size_t>(u.slot) * MROWS + HPC * c + r] = lse_v;
           }
         }
         ptx::tc_fence_before();
-        ptx::mbar_arrive(S.bar(B_O_FREE));
-        if (h == 0) MLA_TRACE_EV(g - 1, 15);
+        __syncwarp();
+        if (lane == 0) ptx::mbar_arrive_remote(o_free);
+        if (t == 0) MLA_TRACE_EV(g - 1, 15);
       }
+      ++uu;
     }
-  } else if (warp == 8) {
-    // ------------------------------------------------------------------ producer
+  } else if (warp == PROD_WARP) {
+    // ------------------------------------------------------------------ producer: L2 prefetch
     if (lane == 0) {
       UnitWalker wk(p, k);
       Unit u;
       uint32_t g = 0;
       bool ok = true;
+      const uint64_t t0 = ptx::globaltimer();
       while (ok && wk.next(u)) {
-        for (int j = u.tb; j < u.te; ++j) {
-          const uint32_t s = g & 1, ph = (g >> 1) & 1;
-          if (!wait_bar(S.bar(B_FP8_EMPTY + s), ph ^ 1, false, abort, p.status, peer_abort)) {
-            ok = false;
-            break;
+        for (int j = u.tb; j < u.te && ok; ++j, ++g) {
+          while (g >= *conv_tile + PF_DIST) {
+            if (*abort || ptx::globaltimer() - t0 > 8 * WAIT_LIMIT_NS) {
+              ok = false;
+              break;
+            }
+            __nanosleep(256);
           }
-          MLA_TRACE_EV(g, 16);
-          const int nv = min(BN, u.nvis - j * BN);
-          produce_tile(p, &tm_lat, &tm_rope, static_cast<int>(c), u.b, j * BN, nv, S.base + SF0 + s * SF_STRIDE,
-                       S.bar(B_FP8_FULL + s));
-          MLA_TRACE_EV(g, 17);
-          ++g;
-        }
-      }
-      // drain: every issued stage has landed before the CTA may exit
-      for (uint32_t d = (g >= 2 ? g - 2 : 0); d < g; ++d) {
-        const uint32_t s = d & 1, ph = (d >> 1) & 1;
-        if (!ptx::mbar_try_wait(S.bar(B_FP8_FULL + s), ph)) {
-          const uint64_t t0 = ptx::globaltimer();
-          while (!ptx::mbar_try_wait(S.bar(B_FP8_FULL + s), ph) && ptx::globaltimer() - t0 < WAIT_LIMIT_NS) {}
+          if (ok) prefetch_tile(p, static_cast<int>(c), u.b, u.nvis, j);
         }
       }
     }
-  } else {
-    // ------------------------------------------------------------------ MMA issuer
-    if (lane == 0) {
-      UnitWalker wk(p, k);
-      Unit u;
-      uint32_t g = 0, uu = 0;
-      bool have_prev = false, prev_first = false;
-      uint32_t prev_g = 0, prev_u = 0;
-      auto issue_pv = [&](uint32_t hg, bool first, uint32_t hu) -> bool {
-        const uint32_t hb = hg & 1;
-        if (first && !wait_bar(S.bar(B_O_FREE), (hu & 1) ^ 1, false, abort, p.status, peer_abort)) return false;
-        if (!wait_bar(S.bar(B_P_FULL + hb), (hg >> 1) & 1, false, abort, p.status, peer_abort)) return false;
-        MLA_TRACE_EV(hg, 22);
-        ptx::tc_fence_after();
-        const uint32_t kt = S.base + SK0 + hb * SK_STRIDE;
-#pragma unroll
-        for (int kk = 0; kk < 4; ++kk) {
-          const uint64_t bd = ptx::smem_desc(kt + kk * 2048, 8192, 1024, ptx::SW_128B);
-          ptx::mma_ts(tbase + T_O, tbase + T_S + 64 * hb + 8 * kk, bd, IDESC_PV, (first && kk == 0) ? 0u : 1u);
-        }
-        ptx::mma_commit(S.bar(B_O_DONE + hb));
-        ptx::mma_commit(S.bar(B_K_EMPTY + hb));
-        MLA_TRACE_EV(hg, 23);
-        return true;
-      };
-      while (wk.next(u)) {
-        MLA_WAIT(S.bar(B_Q_FULL), uu & 1, false);
-        ptx::tc_fence_after();
-        for (int j = u.tb; j < u.te; ++j, ++g) {
-          const uint32_t kb = g & 1;
-          MLA_WAIT(S.bar(B_K_FULL + kb), (g >> 1) & 1, false);
-          MLA_TRACE_EV(g, 20);
+  } else if (c == 0) {
+    // ------------------------------------------------------------------ MMA issuer (CTA 0 of the pair)
+    // The whole warp runs the loop (descriptors stay warp-uniform); one elected lane issues.
+    // Greedy order: P.V(h) as soon as both CTAs' P(h) is in shared memory; Q.K^T(g) as soon as both
+    // CTAs' K/V tile g is converted and P.V(g - 2) (which frees score buffer g & 1) was issued.
+    TileCursor qc(p, k), pc(p, k);
+    uint32_t gq = 0, gp = 0, uq = 0, up = 0;
+    // descriptor bases; per K step only the start-address field (bits 0..13, bytes >> 4) moves
+    const uint64_t dq0 = ptx::smem_desc(base + SQ, 16, 1024, ptx::SW_128B);
+    const uint64_t dk0 = ptx::smem_desc(base + SK0, 16, 1024, ptx::SW_128B);
+    const uint64_t dp0 = ptx::smem_desc(base + SP0, 16, 1024, ptx::SW_128B);
+    const uint64_t dv0 = ptx::smem_desc(base + SV0, SV_ATOM, 1024, ptx::SW_128B);
+    uint64_t t_idle = 0;
+    while (pc.valid) {
+      bool progress = false;
+      // ---- P.V of tile gp
+      if (gp < gq) {
+        const uint32_t hb = gp & 1;
+        const bool first = pc.first;
+        bool ready = ptx::mbar_test_wait_acq_cluster(BAR(B_P_FULL + hb), (gp >> 1) & 1);
+        if (ready && first) ready = ptx::mbar_test_wait_acq_cluster(BAR(B_O_FREE), (up & 1) ^ 1);
+        if (__all_sync(0xffffffffu, ready)) {
           ptx::tc_fence_after();
-          const uint32_t kt = S.base + SK0 + kb * SK_STRIDE;
-          const uint32_t dS = tbase + T_S + 64 * kb;
+          if (ptx::elect_one()) {
+            MLA_TRACE_EV(gp, 22);
 #pragma unroll
-          for (int ks = 0; ks < 16; ++ks) {
-            const uint64_t ad = ptx::smem_desc(S.base + SQ_LAT + (ks >> 2) * 16384 + (ks & 3) * 32, 16, 1024, ptx::SW_128B);
-            const uint64_t bd = ptx::smem_desc(kt + (ks >> 2) * 8192 + (ks & 3) * 32, 16, 1024, ptx::SW_128B);
-            ptx::mma_ss(dS, ad, bd, IDESC_QK, ks > 0 ? 1u : 0u);
-          }
+            for (int jv = 0; jv < 2; ++jv) {
 #pragma unroll
-          for (int ks = 0; ks < 2; ++ks) {
-            const uint64_t ad = ptx::smem_desc(S.base + SQ_ROPE + ks * 32, 16, 512, ptx::SW_64B);
-            const uint64_t bd = ptx::smem_desc(kt + SK_ROPE + ks * 32, 16, 512, ptx::SW_64B);
-            ptx::mma_ss(dS, ad, bd, IDESC_QK, 1u);
+              for (int kk = 0; kk < 4; ++kk) {
+                const uint64_t ad = dp0 + ((hb * SP_STRIDE + kk * 32) >> 4);
+                const uint64_t bd = dv0 + ((hb * SV_STRIDE + 2 * jv * SV_ATOM + kk * 2048) >> 4);
+                ptx::mma_pair_ss(tbase + T_O + 128 * jv, ad, bd, IDESC_PV, (first && kk == 0) ? 0u : 1u);
+              }
+            }
+            ptx::mma_commit_pair(BAR(B_PV_DONE + hb), 0x3);
+            MLA_TRACE_EV(gp, 23);
           }
-          ptx::mma_commit(S.bar(B_S_FULL + kb));
-          MLA_TRACE_EV(g, 21);
-          if (j == u.te - 1) ptx::mma_commit(S.bar(B_Q_FREE));
-          if (have_prev && !issue_pv(prev_g, prev_first, prev_u)) goto role_done;
-          have_prev = true;
-          prev_g = g;
-          prev_first = (j == u.tb);
-          prev_u = uu;
+          __syncwarp();
+          if (first) ++up;
+          ++gp;
+          pc.advance();
+          progress = true;
         }
-        ++uu;
       }
-      if (have_prev && !issue_pv(prev_g, prev_first, prev_u)) goto role_done;
+      // ---- Q.K^T of tile gq
+      if (qc.valid && gq < gp + 2) {
+        const uint32_t kb = gq & 1;
+        bool ready = ptx::mbar_test_wait_acq_cluster(BAR(B_KV_FULL + kb), (gq >> 1) & 1);
+        if (ready && qc.first) ready = ptx::mbar_test_wait_acq_cluster(BAR(B_Q_FULL), uq & 1);
+        if (__all_sync(0xffffffffu, ready)) {
+          ptx::tc_fence_after();
+          if (ptx::elect_one()) {
+            MLA_TRACE_EV(gq, 20);
+            const uint32_t dS = tbase + T_S + 32 * kb;
+#pragma unroll
+            for (int ks = 0; ks < 36; ++ks) {
+              const uint32_t off = (ks & 3) * 32;
+              const uint64_t ad = dq0 + (((ks >> 2) * SQ_ATOM + off) >> 4);
+              const uint64_t bd = dk0 + ((kb * SK_STRIDE + (ks >> 2) * SK_ATOM + off) >> 4);
+              ptx::mma_pair_ss(dS, ad, bd, IDESC_QK, ks > 0 ? 1u : 0u);
+            }
+            ptx::mma_commit_pair(BAR(B_S_FULL + kb), 0x3);
+            MLA_TRACE_EV(gq, 21);
+            if (qc.j == qc.u.te - 1) ptx::mma_commit_pair(BAR(B_Q_FREE), 0x3);
+          }
+          __syncwarp();
+          if (qc.first) ++uq;
+          ++gq;
+          qc.advance();
+          progress = true;
+        }
+      }
+      if (progress) {
+        t_idle = 0;
+      } else {
+        if (t_idle == 0) t_idle = ptx::globaltimer();
+        if (*abort) goto role_done;
+        __nanosleep(32);
+        if (ptx::globaltimer() - t_idle > WAIT_LIMIT_NS) {
+          if (lane == 0) {
+            *abort = 1u;
+            ptx::st_cluster_u32(peer_abort, 1u);
+            raise_status(p.status, STATUS_TIMEOUT);
+          }
+          goto role_done;
+        }
+      }
     }
   }
 role_done:
-#undef MLA_WAIT
+#undef MLA_WAIT_WARP_CL
 #undef MLA_WAIT_WARP
-  // every tcgen05 op issued by the MMA thread has finished before TMEM is released
-  if (warp == 9 && lane == 0) {
-    ptx::mma_commit(S.bar(B_DRAIN));
+  // every pair MMA issued by CTA 0 has finished before TMEM is released
+  if (c == 0 && warp == MMA_WARP && lane == 0) {
+    ptx::mma_commit_pair(BAR(B_DRAIN), 0x1);
     const uint64_t t0 = ptx::globaltimer();
-    while (!ptx::mbar_try_wait(S.bar(B_DRAIN), 0) && ptx::globaltimer() - t0 < WAIT_LIMIT_NS) {}
+    while (!ptx::mbar_try_wait(BAR(B_DRAIN), 0) && ptx::globaltimer() - t0 < WAIT_LIMIT_NS) {}
   }
+#undef BAR
   ptx::tc_fence_before();
   __syncthreads();
-  ptx::cluster_sync();   // no DSMEM traffic targets a CTA that has exited
-  if (warp == 9) {
+  ptx::cluster_sync();   // no remote arrive or pair MMA targets a CTA that has exited
+  if (warp == MMA_WARP) {
     ptx::tc_fence_after();
-    ptx::tmem_dealloc(tbase, TMEM_COLS);
+    ptx::tmem_dealloc_pair(tbase, TMEM_COLS);
   }
 }
 
@@ -815,17 +993,17 @@ mla_combine_kernel(const __grid_constant__ DecodeParams p) {
 }
 
 // =============================================================================================
-// gather + dequant kernel (steps A and C alone): one CTA per (request, tile, dim half)
+// gather + dequant kernel (steps A and C alone): one CTA of 256 threads per (request, 64-key tile,
+// key half c).  Runs the decode's converter (load_tile + store_tile) and copies its K-half buffer
+// back out.
 // =============================================================================================
-constexpr int DQ_THREADS = 160;
-constexpr uint32_t DQ_SK = 0;                    // bf16 tile (SK_STRIDE bytes)
-constexpr uint32_t DQ_SF = SK_STRIDE;            // FP8 stage (SF_STRIDE bytes), 1024-aligned
-constexpr uint32_t DQ_BAR = DQ_SF + SF_STRIDE;
-constexpr uint32_t DQ_SMEM_ALLOC = DQ_BAR + 64 + 1024;
+constexpr int DQ_THREADS = CONV_THREADS;
+constexpr uint32_t DQ_SK = 0;
+constexpr uint32_t DQ_SV = SK_STRIDE;
+constexpr uint32_t DQ_SMEM_ALLOC = SK_STRIDE + SV_STRIDE + 1024;
 
 __global__ void __launch_bounds__(DQ_THREADS)
-mla_dequant_kernel(const __grid_constant__ DecodeParams p, const __grid_constant__ CUtensorMap tm_lat,
-                   const __grid_constant__ CUtensorMap tm_rope, const uint32_t* cache_lengths, int max_keys,
+mla_dequant_kernel(const __grid_constant__ DecodeParams p, const uint32_t* cache_lengths, int max_keys,
                    int tiles_per_req, uint16_t* out_k) {
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -834,42 +1012,17 @@ mla_dequant_kernel(const __grid_constant__ DecodeParams p, const __grid_constant
   const int j = blockIdx.x % tiles_per_req;
   const int c = blockIdx.y;
   const int n = min(static_cast<int>(min(cache_lengths[b], 0x3FFFFFFFu)) + p.T, max_keys);
-  if (j * BN >= n || b >= p.B) return;
-  const int nv = min(BN, n - j * BN);
-  const uint32_t full = base + DQ_BAR;
-  if (threadIdx.x == 0) {
-    ptx::mbar_init(full, 1);
-    ptx::fence_mbar_init();
-  }
+  if (j * BN + HALF_BN * c >= n || b >= p.B) return;
+  RawTile R;
+  if (!load_tile(p, c, threadIdx.x, b, n, j, R)) raise_status(p.status, STATUS_BOUNDS);
+  store_tile(c, threadIdx.x, R, base + DQ_SK, base + DQ_SV);
   __syncthreads();
-  if (threadIdx.x == 128) produce_tile(p, &tm_lat, &tm_rope, c, b, j * BN, nv, base + DQ_SF, full);
-  // bounded wait for the stage
-  {
-    const uint64_t t0 = ptx::globaltimer();
-    bool ok = false;
-    while (!(ok = ptx::mbar_try_wait(full, 0)) && ptx::globaltimer() - t0 < WAIT_LIMIT_NS) {}
-    if (!ok) {
-      if (threadIdx.x == 0) raise_status(p.status, STATUS_TIMEOUT);
-      return;
-    }
-  }
-  if (threadIdx.x < 128) convert_tile(threadIdx.x, base + DQ_SF, base + DQ_SK, nv);
-  __syncthreads();
-  // un-swizzle the tile back to row-major [row][576] bf16
-  for (int id = threadIdx.x; id < BN * 36; id += DQ_THREADS) {
-    const int row = id / 36, cc = id - row * 36;
+  const int nv = min(HALF_BN, n - (j * BN + HALF_BN * c));
+  for (int id = threadIdx.x; id < HALF_BN * 72; id += DQ_THREADS) {
+    const int row = id / 72, cc = id - row * 72;        // 72 units of 8 bf16 per key
     if (row >= nv) continue;
-    uint32_t src;
-    int col;
-    if (cc < 32) {
-      src = base + DQ_SK + (cc >> 3) * 8192 + sw128_off(row, cc & 7);
-      col = 256 * c + cc * 8;
-    } else {
-      src = base + DQ_SK + SK_ROPE + sw64_off(row, cc - 32);
-      col = 512 + 32 * c + (cc - 32) * 8;
-    }
-    const uint4 v = ptx::ld_shared_v4(src);
-    uint16_t* dst = out_k + (static_cast<size_t>(b) * max_keys + j * BN + row) * HEAD_DIM + col;
+    const uint4 v = ptx::ld_shared_v4(base + DQ_SK + (cc >> 3) * SK_ATOM + sw128_off(row, cc & 7));
+    uint16_t* dst = out_k + (static_cast<size_t>(b) * max_keys + j * BN + HALF_BN * c + row) * HEAD_DIM + cc * 8;
     *reinterpret_cast<uint4*>(dst) = v;
   }
 }

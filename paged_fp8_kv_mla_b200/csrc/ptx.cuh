@@ -36,6 +36,17 @@ __device__ __forceinline__ uint32_t nclusters_x() {
   return r;
 }
 
+// True on exactly one active lane of the (fully converged) warp.
+__device__ __forceinline__ bool elect_one() {
+  uint32_t pred = 0;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t.reg .b32 r;\n\t"
+      "elect.sync r|p, 0xffffffff;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(pred));
+  return pred != 0;
+}
+
 __device__ __forceinline__ void cluster_sync() {
   asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::: "memory");
 }
@@ -80,6 +91,28 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t addr, uint32_t parity) {
   return ok != 0;
 }
 
+// Same, letting the thread sleep up to `ns` nanoseconds for the phase (fewer polling issue slots).
+__device__ __forceinline__ bool mbar_try_wait_sleep(uint32_t addr, uint32_t parity, uint32_t ns) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok) : "r"(addr), "r"(parity), "r"(ns) : "memory");
+  return ok != 0;
+}
+
+// Non-blocking probe of a phase (cluster-scope acquire when it has completed).
+__device__ __forceinline__ bool mbar_test_wait_acq_cluster(uint32_t addr, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.test_wait.parity.acquire.cluster.shared::cta.b64 p, [%1], %2;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok) : "r"(addr), "r"(parity) : "memory");
+  return ok != 0;
+}
+
 // Poll without acquire semantics; the caller issues fence_acq_rel_cluster() once it succeeds.
 __device__ __forceinline__ bool mbar_try_wait_relaxed_cluster(uint32_t addr, uint32_t parity) {
   uint32_t ok;
@@ -88,6 +121,17 @@ __device__ __forceinline__ bool mbar_try_wait_relaxed_cluster(uint32_t addr, uin
       "mbarrier.try_wait.parity.relaxed.cluster.shared::cta.b64 p, [%1], %2;\n\t"
       "selp.u32 %0, 1, 0, p;\n\t}"
       : "=r"(ok) : "r"(addr), "r"(parity) : "memory");
+  return ok != 0;
+}
+
+// Poll with cluster-scope acquire (for barriers that other CTAs' threads arrive on).
+__device__ __forceinline__ bool mbar_try_wait_acq_cluster(uint32_t addr, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.try_wait.parity.acquire.cluster.shared::cta.b64 p, [%1], %2, %3;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok) : "r"(addr), "r"(parity), "r"(100000u) : "memory");
   return ok != 0;
 }
 
