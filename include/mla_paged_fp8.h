@@ -111,6 +111,29 @@ mla_status_t mla_decode_paged_fp8(
     const mla_paged_shape_t* shape, void* out, float* lse, cudaStream_t stream);
 
 /*
+ * mla_decode_paged_fp8_noalloc -- the same decode, for callers that cannot allocate device memory
+ * (for instance while a CUDA graph is being captured, under an allocator that owns the whole
+ * device, or in a service that forbids allocation once it is running).  The reference pages have
+ * no counterpart to this entry point.
+ *
+ * It takes exactly the arguments of mla_decode_paged_fp8 and produces the same results, but keeps
+ * its temporary data (split plan and split-KV partial results) in one fixed device array built into
+ * the library: about 42.5 MB on every GPU that loads the library, held until the process exits.
+ * It never calls cudaMalloc or cudaFree.  Limits: batch * max_prompt_length *
+ * ceil(num_q_heads / 128) <= 65536 (else MLA_ERR_UNSUPPORTED, with the reason in
+ * mla_last_error_string), and the keys are split over at most 80 two-CTA clusters.
+ * The first call on a device looks up the array's device address and sets kernel attributes; make
+ * that first call before any stream capture.  All calls share the array: calls whose GPU work
+ * overlaps (for example on two streams) race and corrupt each other's results, so serialise them.
+ * Nothing in the array needs to start at zero: each call writes everything it later reads.
+ */
+mla_status_t mla_decode_paged_fp8_noalloc(
+    const void* q, const void* blocks, const float* scales,
+    const uint32_t* cache_lengths, const uint32_t* lookup_table, const uint32_t* scales_lookup_table,
+    uint32_t max_prompt_length, uint32_t max_cache_length, uint32_t layer_idx, float softmax_scale,
+    const mla_paged_shape_t* shape, void* out, float* lse, cudaStream_t stream);
+
+/*
  * mla_gather_dequant_bf16 -- steps A and C of the decode on their own: gather every
  * stored key of every request through the page tables and dequantise it to bf16
  * with the per-token scale, K[t] = bf16_rn(f32_rn(e4m3 * s_t)).  Runs the same

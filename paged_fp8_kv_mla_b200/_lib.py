@@ -22,7 +22,7 @@ STATUS_NAMES = {0: "MLA_OK", 1: "MLA_ERR_INVALID_ARG", 2: "MLA_ERR_UNSUPPORTED",
 # every symbol include/mla_paged_fp8.h declares
 EXPORTED = ["mla_decode_paged_fp8", "mla_gather_dequant_bf16", "mla_set_num_clusters",
             "mla_get_num_clusters", "mla_last_error_string", "mla_get_device_status",
-            "mla_release_workspace", "mla_version", "mla_set_timing_events"]
+            "mla_release_workspace", "mla_version", "mla_set_timing_events", "mla_decode_paged_fp8_noalloc"]
 
 
 class MlaError(RuntimeError):
@@ -52,6 +52,9 @@ def load(path: str = LIB_PATH) -> ctypes.CDLL:
     lib.mla_decode_paged_fp8.argtypes = [vp, vp, vp, vp, vp, vp, u32, u32, u32, f32,
                                          ctypes.POINTER(PagedShape), vp, vp, vp]
     lib.mla_decode_paged_fp8.restype = ctypes.c_int
+    lib.mla_decode_paged_fp8_noalloc.argtypes = [vp, vp, vp, vp, vp, vp, u32, u32, u32, f32,
+                                                 ctypes.POINTER(PagedShape), vp, vp, vp]
+    lib.mla_decode_paged_fp8_noalloc.restype = ctypes.c_int
     lib.mla_gather_dequant_bf16.argtypes = [vp, vp, vp, vp, vp, u32, u32, u32,
                                             ctypes.POINTER(PagedShape), vp, u32, vp]
     lib.mla_gather_dequant_bf16.restype = ctypes.c_int
@@ -123,6 +126,24 @@ def decode(q, blocks, scales, cache_lengths, lookup_table, scales_lookup_table, 
                                   _ptr(scales_lookup_table), int(max_prompt_length), int(max_cache_length),
                                   int(layer_idx), float(softmax_scale), ctypes.byref(shp), _ptr(out), _ptr(lse),
                                   _stream(stream))
+    _check(st)
+    return out, lse
+
+
+def decode_noalloc(q, blocks, scales, cache_lengths, lookup_table, scales_lookup_table, max_prompt_length: int,
+                   max_cache_length: int, layer_idx: int, softmax_scale: float, out, lse, stream=None):
+    """mla_decode_paged_fp8_noalloc: the decode on the library's fixed scratch (no device allocation).
+
+    `out` and `lse` must be preallocated by the caller.
+    """
+    lib = load()
+    B, T, H, D = q.shape
+    _contig(q, blocks, scales, cache_lengths, lookup_table, scales_lookup_table, out, lse)
+    shp = paged_shape(B, H, blocks, scales, lookup_table)
+    st = lib.mla_decode_paged_fp8_noalloc(_ptr(q), _ptr(blocks), _ptr(scales), _ptr(cache_lengths),
+                                          _ptr(lookup_table), _ptr(scales_lookup_table), int(max_prompt_length),
+                                          int(max_cache_length), int(layer_idx), float(softmax_scale),
+                                          ctypes.byref(shp), _ptr(out), _ptr(lse), _stream(stream))
     _check(st)
     return out, lse
 

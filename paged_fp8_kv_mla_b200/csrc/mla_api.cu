@@ -180,6 +180,49 @@ unsigned int* status_ptr() {
 
 }  // namespace
 
+// ---------------------------------------------------------------- fixed scratch (no-allocation entry)
+// Some callers cannot allocate device memory while they run (CUDA graph capture, allocators that own
+// the whole device, real-time services that forbid allocation after start-up).  For them the decode
+// also runs on one statically sized device array instead of the lazily allocated workspace.
+namespace {
+
+constexpr int kNoAllocMaxItems = 65536;      // (request, query token, head group) triples per call
+constexpr int kNoAllocMaxClusters = 80;      // 2-CTA clusters the split is cut into (B200 default: 74)
+
+constexpr size_t noalloc_up(size_t v) { return (v + 255) / 256 * 256; }
+constexpr size_t kNoAllocBytes =
+    noalloc_up(64) + noalloc_up(sizeof(int32_t) * (kNoAllocMaxItems + 1)) + noalloc_up(sizeof(int32_t) * kNoAllocMaxItems) +
+    noalloc_up(sizeof(int32_t) * kNoAllocMaxClusters) + noalloc_up(sizeof(float) * 2 * kNoAllocMaxClusters * mla::MROWS) +
+    noalloc_up(sizeof(float) * 2 * kNoAllocMaxClusters * mla::MROWS * mla::V_DIM);
+
+std::mutex g_noalloc_mu;
+void* g_noalloc_ptr[kMaxDevices];
+
+}  // namespace
+
+// The scratch itself: about 42.5 MB of device memory on every GPU that loads this library, held
+// until the process exits.  Host code must not pass this symbol to a kernel (in host code it names
+// a host-side stand-in); it uses the device address cudaGetSymbolAddress returns.
+static __device__ __align__(256) unsigned char g_noalloc_scratch[kNoAllocBytes];
+
+namespace {
+
+// Device address of the scratch for the current device, looked up once per device.
+mla_status_t noalloc_scratch(int dev, void** out) {
+  std::lock_guard<std::mutex> lk(g_noalloc_mu);
+  if (!g_noalloc_ptr[dev]) {
+    void* ptr = nullptr;
+    cudaError_t e = cudaGetSymbolAddress(&ptr, g_noalloc_scratch);
+    if (e != cudaSuccess || !ptr)
+      return fail(MLA_ERR_CUDA, "cudaGetSymbolAddress of the fixed scratch failed: %s", cudaGetErrorString(e));
+    g_noalloc_ptr[dev] = ptr;
+  }
+  *out = g_noalloc_ptr[dev];
+  return MLA_OK;
+}
+
+}  // namespace
+
 extern "C" {
 
 const char* mla_version(void) { return "0.1.0"; }
@@ -325,6 +368,89 @@ mla_status_t mla_debug_set_trace(unsigned long long* buf) {
   return MLA_OK;
 }
 #endif
+
+// Same decode as mla_decode_paged_fp8, but on the fixed scratch: no device memory is allocated or
+// freed.  The first call on a device looks up the scratch address (and, like the regular entry,
+// sets the kernels' shared-memory attribute); make that first call before any stream capture.
+// Calls share the scratch, so two calls that overlap on the GPU (different streams or devices'
+// worth of work racing on one device) corrupt each other; serialise them.  Nothing in the scratch
+// has to start at zero: every call writes what it reads.
+mla_status_t mla_decode_paged_fp8_noalloc(const void* q, const void* blocks, const float* scales,
+                                          const uint32_t* cache_lengths, const uint32_t* lookup_table,
+                                          const uint32_t* scales_lookup_table, uint32_t max_prompt_length,
+                                          uint32_t max_cache_length, uint32_t layer_idx, float softmax_scale,
+                                          const mla_paged_shape_t* shape, void* out, float* lse,
+                                          cudaStream_t stream) {
+  mla::DecodeParams p{};
+  uint64_t rows = 0;
+  mla_status_t st = check_cache(blocks, scales, cache_lengths, lookup_table, max_prompt_length, max_cache_length,
+                                layer_idx, shape, &p, &rows);
+  if (st != MLA_OK) return st;
+  if (!q || !out) return fail(MLA_ERR_INVALID_ARG, "q and out must be non-NULL");
+  if (!aligned16(q) || !aligned16(out)) return fail(MLA_ERR_INVALID_ARG, "q and out must be 16-byte aligned");
+  if (!(softmax_scale == softmax_scale)) return fail(MLA_ERR_INVALID_ARG, "softmax_scale is NaN");
+  if (p.B == 0) return MLA_OK;
+  const int64_t items64 = static_cast<int64_t>(p.B) * p.T * p.G;
+  if (items64 > kNoAllocMaxItems)
+    return fail(MLA_ERR_UNSUPPORTED,
+                "batch * max_prompt_length * ceil(num_q_heads / 128) = %lld exceeds the fixed scratch limit of %d",
+                static_cast<long long>(items64), kNoAllocMaxItems);
+  p.items = static_cast<int>(items64);
+
+  int dev = 0;
+  MLA_CUDA(cudaGetDevice(&dev));
+  if (dev >= kMaxDevices) return fail(MLA_ERR_UNSUPPORTED, "device index too large");
+  int NC = 0;
+  st = device_setup(dev, &NC);
+  if (st != MLA_OK) return st;
+  if (NC > kNoAllocMaxClusters) NC = kNoAllocMaxClusters;
+  p.NC = NC;
+
+  void* ws = nullptr;
+  st = noalloc_scratch(dev, &ws);
+  if (st != MLA_OK) return st;
+  const WsLayout L = ws_layout(p.items, NC);
+  if (L.total > kNoAllocBytes) return fail(MLA_ERR_UNSUPPORTED, "problem needs more than the fixed scratch");
+  char* w = static_cast<char*>(ws);
+  p.hdr = reinterpret_cast<int32_t*>(w + L.hdr);
+  p.item_start = reinterpret_cast<int32_t*>(w + L.item_start);
+  p.item_nvis = reinterpret_cast<int32_t*>(w + L.item_nvis);
+  p.cluster_first = reinterpret_cast<int32_t*>(w + L.cluster_first);
+  p.part_lse = reinterpret_cast<float*>(w + L.part_lse);
+  p.part_o = reinterpret_cast<float*>(w + L.part_o);
+  p.q = static_cast<const uint16_t*>(q);
+  p.slut = scales_lookup_table;
+  p.out = static_cast<uint16_t*>(out);
+  p.lse = lse;
+  p.status = status_ptr();
+  if (!p.status) return fail(MLA_ERR_CUDA, "status word address unavailable");
+  p.scale_log2 = softmax_scale * 1.4426950408889634f;
+
+  mla::mla_plan_kernel<<<1, mla::PLAN_THREADS, 0, stream>>>(
+      cache_lengths, p.B, p.T, p.G, max_cache_length, NC, const_cast<int32_t*>(p.item_start),
+      const_cast<int32_t*>(p.item_nvis), const_cast<int32_t*>(p.cluster_first), const_cast<int32_t*>(p.hdr), p.status);
+  MLA_CUDA(cudaGetLastError());
+
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(2 * NC);
+  cfg.blockDim = dim3(mla::NUM_THREADS);
+  cfg.dynamicSmemBytes = mla::SMEM_ALLOC;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = 2;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  MLA_CUDA(cudaLaunchKernelEx(&cfg, mla::mla_decode_kernel, p));
+
+  const int per_item = mla::MROWS / mla::COMBINE_HEADS;
+  const int64_t cgrid = static_cast<int64_t>(p.items) * per_item;
+  mla::mla_combine_kernel<<<static_cast<unsigned>(cgrid), 32 * mla::COMBINE_HEADS, 0, stream>>>(p);
+  MLA_CUDA(cudaGetLastError());
+  return MLA_OK;
+}
 
 mla_status_t mla_get_device_status(cudaStream_t stream) {
   MLA_CUDA(cudaStreamSynchronize(stream));

@@ -1,0 +1,63 @@
+"""The no-allocation decode entry point, checked against the regular one.
+
+mla_decode_paged_fp8_noalloc exists for callers that may not allocate device memory while they run
+(a CUDA graph being captured, an allocator that owns the device, a service that forbids allocation
+after start-up).  It keeps its split plan and partial results in a fixed array built into the
+library instead of the lazily allocated workspace, so this test calls it twice in a row with
+different problems (the second call finds the first call's leftovers in the array) and compares each
+result with mla_decode_paged_fp8 on the same inputs, at the tolerances the parity tests use.
+
+The file name sorts last so that a run stopping at the first failure has run every other test
+first; the test also passes on its own in a fresh process.
+"""
+import numpy as np
+import pytest
+import torch
+
+import paged_fp8_kv_mla_b200 as M
+from oracle import mla_oracle as O
+from paged_fp8_kv_mla_b200 import _lib
+from paged_fp8_kv_mla_b200 import workloads as W
+
+pytestmark = pytest.mark.gpu
+
+OUT_RTOL = 2e-2
+OUT_ATOL = 1e-2
+LSE_ATOL = 1e-3
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _built():
+    from paged_fp8_kv_mla_b200 import build
+    build.build()
+    M.load()
+    M.set_num_clusters(0)
+    yield
+
+
+def _bf16_to_f64(t):
+    return O.bf16_bits_to_f64(t.detach().cpu().view(torch.int16).numpy().view(np.uint16))
+
+
+def _close(out_a, lse_a, out_b, lse_b):
+    a = _bf16_to_f64(out_a)
+    b = _bf16_to_f64(out_b)
+    assert np.isfinite(a).all() and np.isfinite(b).all()
+    tol = OUT_RTOL * np.abs(b).max() + OUT_ATOL
+    assert np.abs(a - b).max() <= tol
+    assert (lse_a - lse_b).abs().max().item() <= LSE_ATOL
+
+
+@pytest.mark.parametrize("first,second", [(1, 3), (0, 2)])
+def test_noalloc_matches_regular_entry_two_calls_in_a_row(first, second):
+    for cfg_i in (first, second):
+        inp = W.make_inputs(W.CONFIGS[cfg_i], device="cuda")
+        out_ref, lse_ref = M.decode_inputs(inp)
+        out = torch.full_like(out_ref, float("nan"))
+        lse = torch.full_like(lse_ref, float("nan"))
+        _lib.decode_noalloc(inp.q, inp.blocks, inp.scales, inp.cache_lengths, inp.lookup_table,
+                            inp.scales_lookup_table, inp.max_prompt_length, inp.max_cache_length,
+                            inp.layer_idx, inp.softmax_scale, out, lse)
+        torch.cuda.synchronize()
+        assert M.device_status() == 0
+        _close(out, lse, out_ref, lse_ref)
