@@ -281,11 +281,8 @@ struct LutVals {
   bool bad;
 };
 
-struct TilePtrs {
-  const uint8_t* ov;
-  const float* os;
-  const uint8_t* pv;
-  const float* ps;
+struct TilePtrs {                 // row indices into blocks / scales (both < 2^32, checked on the host)
+  uint32_t ov, os, pv, ps;
   bool own_ok, oth_ok;
 };
 
@@ -315,34 +312,37 @@ __device__ __forceinline__ TilePtrs lut_finish(const DecodeParams& p, const LutV
   T.oth_ok = V.oth_in && V.pb < static_cast<uint32_t>(p.NB) && V.psb < static_cast<uint32_t>(p.NSB);
   if (V.own_in && !T.own_ok) bad = true;
   if (V.oth_in && !T.oth_ok) bad = true;
-  const int oslot = V.otok % p.P, pslot = V.ptok % p.P;
-  const size_t lay = static_cast<size_t>(p.layer);
-  T.ov = p.blocks + (((static_cast<size_t>(V.ob) * p.KVD) * p.NL + lay) * p.P + oslot) * HEAD_DIM;
-  T.os = p.scales + ((static_cast<size_t>(V.osb) * p.KVD) * p.NL + lay) * p.P + oslot;
-  T.pv = p.blocks + (((static_cast<size_t>(V.pb) * p.KVD) * p.NL + lay) * p.P + pslot) * HEAD_DIM;
-  T.ps = p.scales + ((static_cast<size_t>(V.psb) * p.KVD) * p.NL + lay) * p.P + pslot;
+  const uint32_t oslot = static_cast<uint32_t>(V.otok % p.P), pslot = static_cast<uint32_t>(V.ptok % p.P);
+  const uint32_t per_blk = static_cast<uint32_t>(p.KVD * p.NL * p.P);
+  const uint32_t lay = static_cast<uint32_t>(p.layer * p.P);
+  T.ov = V.ob * per_blk + lay + oslot;
+  T.os = V.osb * per_blk + lay + oslot;
+  T.pv = V.pb * per_blk + lay + pslot;
+  T.ps = V.psb * per_blk + lay + pslot;
   return T;
 }
 
-__device__ __forceinline__ void fetch(const TilePtrs& T, int c, int t, RawTile& R) {
+__device__ __forceinline__ void fetch(const DecodeParams& p, const TilePtrs& T, int c, int t, RawTile& R) {
   const int q = t & 7;
   R.own_ok = T.own_ok;
   R.oth_ok = T.oth_ok;
   if (T.own_ok) {
-    R.so = __ldg(T.os);
+    const uint8_t* ov = p.blocks + static_cast<size_t>(T.ov) * HEAD_DIM;
+    R.so = __ldg(p.scales + T.os);
 #pragma unroll
     for (int k = 0; k < 5; ++k) {
       const int qq = q + 8 * k;
-      if (qq < 36) R.own[k] = ptx::ldg_stream_v4(T.ov + 16 * qq);
+      if (qq < 36) R.own[k] = ptx::ldg_stream_v4(ov + 16 * qq);
     }
   }
   if (T.oth_ok) {
-    R.sp = __ldg(T.ps);
+    const uint8_t* pv = p.blocks + static_cast<size_t>(T.pv) * HEAD_DIM;
+    R.sp = __ldg(p.scales + T.ps);
 #pragma unroll
     for (int k = 0; k < 2; ++k) {
       const int jc = q + 8 * k;                              // chunk index within D_c (0..15)
       const int qq = jc < 8 ? 8 * c + jc : 16 + 8 * c + (jc - 8);
-      R.oth[k] = ptx::ldg_stream_v4(T.pv + 16 * qq);
+      R.oth[k] = ptx::ldg_stream_v4(pv + 16 * qq);
     }
   }
 }
@@ -351,7 +351,7 @@ __device__ __forceinline__ void fetch(const TilePtrs& T, int c, int t, RawTile& 
 __device__ __forceinline__ bool load_tile(const DecodeParams& p, int c, int t, int b, int nvis, int j, RawTile& R) {
   bool bad;
   const TilePtrs T = lut_finish(p, lut_issue(p, c, t, b, nvis, j), bad);
-  fetch(T, c, t, R);
+  fetch(p, T, c, t, R);
   return !bad;
 }
 
@@ -392,6 +392,44 @@ __device__ __forceinline__ void store_tile(int c, int t, const RawTile& R, uint3
   }
 }
 
+// What the converter needs to know about one tile (request, query token and head group follow
+// from the item index).
+struct TileInfo {
+  int item, nvis, j;
+  bool first, valid;
+};
+
+// Produces the tile sequence of a cluster one TileInfo at a time (a lighter TileCursor).
+struct TileStream {
+  UnitWalker wk;
+  int item, nvis, j, te;
+  bool valid, first;
+  __device__ TileStream(const DecodeParams& p, int k) : wk(p, k) { next_unit(); }
+  __device__ void next_unit() {
+    Unit u;
+    valid = wk.next(u);
+    item = u.item;
+    nvis = u.nvis;
+    j = u.tb;
+    te = u.te;
+    first = true;
+  }
+  __device__ TileInfo take() {
+    TileInfo t;
+    t.item = item;
+    t.nvis = nvis;
+    t.j = j;
+    t.first = first;
+    t.valid = valid;
+    if (valid) {
+      ++j;
+      first = false;
+      if (j >= te) next_unit();
+    }
+    return t;
+  }
+};
+
 // Sequential cursor over the tiles a cluster processes (unit by unit).
 struct TileCursor {
   UnitWalker wk;
@@ -416,9 +454,9 @@ struct TileCursor {
 
 // Q rows 64c..64c+63 of an item's head group (all 576 dims) into the SW128 K-major layout, by the
 // 256 converter threads.  Rows whose head index is >= H are zero.
-__device__ __forceinline__ void load_q(const DecodeParams& p, const Unit& u, int c, int t, uint32_t sq) {
-  const uint16_t* qrow0 = p.q + (static_cast<size_t>(u.b) * p.T + u.i) * p.H * HEAD_DIM;
-  const int h0 = u.g * MROWS + HPC * c;
+__device__ __forceinline__ void load_q(const DecodeParams& p, int b, int i, int g, int c, int t, uint32_t sq) {
+  const uint16_t* qrow0 = p.q + (static_cast<size_t>(b) * p.T + i) * p.H * HEAD_DIM;
+  const int h0 = g * MROWS + HPC * c;
 #pragma unroll 1
   for (int batch = 0; batch < 2; ++batch) {
     uint4 v[9];
@@ -517,22 +555,21 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) mla_decode_kernel(const __grid
     const int t = threadIdx.x;
     const int cc = static_cast<int>(c);
     const uint32_t kv_full0 = ptx::mapa(BAR(B_KV_FULL), 0), q_full = ptx::mapa(BAR(B_Q_FULL), 0);
-    TileCursor cur(p, k);
+    TileStream ts(p, k);
+    TileInfo cur = ts.take();
     if (cur.valid) {
-      TileCursor n1 = cur;
-      n1.advance();
-      TileCursor n2 = n1;
-      if (n2.valid) n2.advance();
+      TileInfo n1 = ts.take();
+      TileInfo n2 = ts.take();
       RawTile ra, rb;
       bool bad = false;
       {
-        const TilePtrs t0 = lut_finish(p, lut_issue(p, cc, t, cur.u.b, cur.u.nvis, cur.j), bad);
+        const TilePtrs t0 = lut_finish(p, lut_issue(p, cc, t, cur.item / (p.G * p.T), cur.nvis, cur.j), bad);
         if (bad) raise_status(p.status, STATUS_BOUNDS);
-        fetch(t0, cc, t, ra);
+        fetch(p, t0, cc, t, ra);
       }
       TilePtrs t1{};
       if (n1.valid) {
-        t1 = lut_finish(p, lut_issue(p, cc, t, n1.u.b, n1.u.nvis, n1.j), bad);
+        t1 = lut_finish(p, lut_issue(p, cc, t, n1.item / (p.G * p.T), n1.nvis, n1.j), bad);
         if (bad) raise_status(p.status, STATUS_BOUNDS);
       }
       uint32_t g = 0, uu = 0;
@@ -542,23 +579,23 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) mla_decode_kernel(const __grid
         if (cur.first) {                                                                                 \
           MLA_WAIT_WARP(BAR(B_Q_FREE), (uu & 1) ^ 1);                                                    \
           if (t == 0) MLA_TRACE_EV(g, 3);                                                                \
-          load_q(p, cur.u, cc, t, base);                                                                 \
+          load_q(p, cur.item / (p.G * p.T), (cur.item / p.G) % p.T, cur.item % p.G, cc, t, base);         \
           ptx::fence_proxy_async_smem();                                                                 \
           __syncwarp();                                                                                  \
-          if (lane == 0) ptx::mbar_arrive_remote(q_full);                                                \
+          if (lane == 0) ptx::mbar_arrive_cluster(q_full);                                               \
           ++uu;                                                                                          \
         }                                                                                                \
         const uint32_t kb = g & 1;                                                                       \
         MLA_WAIT_WARP(BAR(B_PV_DONE + kb), ((g >> 1) & 1) ^ 1);                                          \
         if (t == 0) MLA_TRACE_EV(g, 1);                                                                  \
-        if (n1.valid) fetch(t1, cc, t, RNXT);                                                            \
+        if (n1.valid) fetch(p, t1, cc, t, RNXT);                                                         \
         LutVals v2{};                                                                                    \
-        if (n2.valid) v2 = lut_issue(p, cc, t, n2.u.b, n2.u.nvis, n2.j);                                 \
+        if (n2.valid) v2 = lut_issue(p, cc, t, n2.item / (p.G * p.T), n2.nvis, n2.j);                    \
         if (t == 0) MLA_TRACE_EV(g, 4);                                                                  \
         store_tile(cc, t, RCUR, base + SK0 + kb * SK_STRIDE, base + SV0 + kb * SV_STRIDE);               \
         ptx::fence_proxy_async_smem();                                                                   \
         __syncwarp();                                                                                    \
-        if (lane == 0) ptx::mbar_arrive_remote(kv_full0 + 8u * kb);                                      \
+        if (lane == 0) ptx::mbar_arrive_cluster(kv_full0 + 8u * kb);                                     \
         if (t == 0) {                                                                                    \
           *conv_tile = g + 1;                                                                            \
           MLA_TRACE_EV(g, 2);                                                                            \
@@ -574,12 +611,12 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) mla_decode_kernel(const __grid
         if (!n1.valid) break;
         cur = n1;
         n1 = n2;
-        if (n2.valid) n2.advance();
+        n2 = ts.take();
         MLA_CONV_STEP(rb, ra)
         if (!n1.valid) break;
         cur = n1;
         n1 = n2;
-        if (n2.valid) n2.advance();
+        n2 = ts.take();
       }
 #undef MLA_CONV_STEP
     }
@@ -671,7 +708,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) mla_decode_kernel(const __grid
         ptx::fence_proxy_async_smem();
         ptx::tc_fence_before();
         __syncwarp();
-        if (lane == 0) ptx::mbar_arrive_remote(p_full0 + 8u * sb);
+        if (lane == 0) ptx::mbar_arrive_cluster(p_full0 + 8u * sb);
         if (t == 0) MLA_TRACE_EV(g, 14);
       }
       // epilogue: O / l for this lane's 256 V dims of head row r
@@ -726,7 +763,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) mla_decode_kernel(const __grid
         }
         ptx::tc_fence_before();
         __syncwarp();
-        if (lane == 0) ptx::mbar_arrive_remote(o_free);
+        if (lane == 0) ptx::mbar_arrive_cluster(o_free);
         if (t == 0) MLA_TRACE_EV(g - 1, 15);
       }
       ++uu;
@@ -771,8 +808,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) mla_decode_kernel(const __grid
       if (gp < gq) {
         const uint32_t hb = gp & 1;
         const bool first = pc.first;
-        bool ready = ptx::mbar_test_wait_acq_cluster(BAR(B_P_FULL + hb), (gp >> 1) & 1);
-        if (ready && first) ready = ptx::mbar_test_wait_acq_cluster(BAR(B_O_FREE), (up & 1) ^ 1);
+        bool ready = ptx::mbar_test_wait(BAR(B_P_FULL + hb), (gp >> 1) & 1);
+        if (ready && first) ready = ptx::mbar_test_wait(BAR(B_O_FREE), (up & 1) ^ 1);
         if (__all_sync(0xffffffffu, ready)) {
           ptx::tc_fence_after();
           if (ptx::elect_one()) {
@@ -799,8 +836,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) mla_decode_kernel(const __grid
       // ---- Q.K^T of tile gq
       if (qc.valid && gq < gp + 2) {
         const uint32_t kb = gq & 1;
-        bool ready = ptx::mbar_test_wait_acq_cluster(BAR(B_KV_FULL + kb), (gq >> 1) & 1);
-        if (ready && qc.first) ready = ptx::mbar_test_wait_acq_cluster(BAR(B_Q_FULL), uq & 1);
+        bool ready = ptx::mbar_test_wait(BAR(B_KV_FULL + kb), (gq >> 1) & 1);
+        if (ready && qc.first) ready = ptx::mbar_test_wait(BAR(B_Q_FULL), uq & 1);
         if (__all_sync(0xffffffffu, ready)) {
           ptx::tc_fence_after();
           if (ptx::elect_one()) {
@@ -829,7 +866,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) mla_decode_kernel(const __grid
       } else {
         if (t_idle == 0) t_idle = ptx::globaltimer();
         if (*abort) goto role_done;
-        __nanosleep(32);
+        __nanosleep(128);
         if (ptx::globaltimer() - t_idle > WAIT_LIMIT_NS) {
           if (lane == 0) {
             *abort = 1u;

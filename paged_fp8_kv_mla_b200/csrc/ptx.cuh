@@ -81,6 +81,14 @@ __device__ __forceinline__ void mbar_arrive_remote(uint32_t cluster_addr) {
   asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" :: "r"(cluster_addr) : "memory");
 }
 
+// Arrive on a barrier of any CTA of the cluster with the default (CTA-scope release) semantics.
+// Used to publish shared-memory MMA operands: the writer first makes its writes visible to the
+// async proxy (fence.proxy.async), and the tensor core that reads them is ordered after the
+// barrier by the waiting thread's tcgen05 fence.
+__device__ __forceinline__ void mbar_arrive_cluster(uint32_t cluster_addr) {
+  asm volatile("mbarrier.arrive.shared::cluster.b64 _, [%0];" :: "r"(cluster_addr) : "memory");
+}
+
 __device__ __forceinline__ bool mbar_try_wait(uint32_t addr, uint32_t parity) {
   uint32_t ok;
   asm volatile(
@@ -99,6 +107,17 @@ __device__ __forceinline__ bool mbar_try_wait_sleep(uint32_t addr, uint32_t pari
       "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
       "selp.u32 %0, 1, 0, p;\n\t}"
       : "=r"(ok) : "r"(addr), "r"(parity), "r"(ns) : "memory");
+  return ok != 0;
+}
+
+// Non-blocking probe of a phase.
+__device__ __forceinline__ bool mbar_test_wait(uint32_t addr, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.test_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok) : "r"(addr), "r"(parity) : "memory");
   return ok != 0;
 }
 
