@@ -1,5 +1,6 @@
 // Host side of the C ABI declared in include/mla_paged_fp8.h: argument validation, the
 // per-device workspace, and the three launches (plan -> decode -> combine) on the caller's stream.
+#include <cuda.h>
 #include <cuda_runtime.h>
 
 #include <cstdarg>
@@ -121,6 +122,18 @@ mla_status_t device_setup(int dev, int* nc_out) {
   return MLA_OK;
 }
 
+// Multiplier and shifts of mla::FastDiv for divisor d >= 1 (l = ceil(log2 d), m = floor(2^32 (2^l - d) / d) + 1).
+mla::FastDiv make_fastdiv(uint32_t d) {
+  mla::FastDiv f{};
+  uint32_t l = 0;
+  while ((1ull << l) < d) ++l;
+  f.d = d;
+  f.m = static_cast<uint32_t>(((1ull << 32) * ((1ull << l) - d)) / d + 1);
+  f.s1 = l < 1 ? l : 1;
+  f.s2 = l > 0 ? l - 1 : 0;
+  return f;
+}
+
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
 // Shared validation of the cache description; fills the parts of DecodeParams that describe it.
@@ -168,7 +181,52 @@ mla_status_t check_cache(const void* blocks, const float* scales, const uint32_t
   p->NSB = s->num_scale_blocks;
   p->max_pages = s->max_pages;
   p->blocks = static_cast<const uint8_t*>(blocks);
+  p->divP = make_fastdiv(static_cast<uint32_t>(p->P));
+  p->divG = make_fastdiv(static_cast<uint32_t>(p->G));
+  p->divT = make_fastdiv(static_cast<uint32_t>(p->T));
   *rows = r;
+  return MLA_OK;
+}
+
+// ---------------------------------------------------------------- Q tensor map
+// cuTensorMapEncodeTiled comes from the driver through the runtime's entry-point query, so the
+// library needs no link-time dependency on libcuda.
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                  const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+mla_status_t get_encode_fn(EncodeTiledFn* fn) {
+  static std::mutex mu;
+  static EncodeTiledFn cached = nullptr;
+  std::lock_guard<std::mutex> lk(mu);
+  if (!cached) {
+    void* ptr = nullptr;
+    cudaDriverEntryPointQueryResult qr;
+    cudaError_t e = cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &qr);
+    if (e != cudaSuccess || qr != cudaDriverEntryPointSuccess || !ptr)
+      return fail(MLA_ERR_CUDA, "cuTensorMapEncodeTiled unavailable (%s)", cudaGetErrorString(e));
+    cached = reinterpret_cast<EncodeTiledFn>(ptr);
+  }
+  *fn = cached;
+  return MLA_OK;
+}
+
+// q [B*T][H][576] bf16 as a 3-D tensor (dims innermost); one box = 64 dims x 64 heads of one query
+// token, written in the 128-byte swizzle the MMA descriptors expect.  Heads past H read as zero.
+mla_status_t make_q_map(CUtensorMap* map, const void* q, int H, int BT) {
+  EncodeTiledFn enc = nullptr;
+  mla_status_t st = get_encode_fn(&enc);
+  if (st != MLA_OK) return st;
+  const cuuint64_t dims[3] = {static_cast<cuuint64_t>(mla::HEAD_DIM), static_cast<cuuint64_t>(H),
+                              static_cast<cuuint64_t>(BT)};
+  const cuuint64_t strides[2] = {static_cast<cuuint64_t>(mla::HEAD_DIM) * 2,
+                                 static_cast<cuuint64_t>(mla::HEAD_DIM) * 2 * static_cast<cuuint64_t>(H)};
+  const cuuint32_t box[3] = {64, static_cast<cuuint32_t>(mla::HPC), 1};
+  const cuuint32_t estr[3] = {1, 1, 1};
+  const CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(q), dims, strides, box, estr,
+                         CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                         CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) return fail(MLA_ERR_CUDA, "cuTensorMapEncodeTiled(q) failed (%d)", static_cast<int>(r));
   return MLA_OK;
 }
 
@@ -289,6 +347,8 @@ mla_status_t mla_decode_paged_fp8(const void* q, const void* blocks, const float
   p.part_lse = reinterpret_cast<float*>(w + L.part_lse);
   p.part_o = reinterpret_cast<float*>(w + L.part_o);
   p.q = static_cast<const uint16_t*>(q);
+  st = make_q_map(&p.tmap_q, q, p.H, p.B * p.T);
+  if (st != MLA_OK) return st;
   p.slut = scales_lookup_table;
   p.out = static_cast<uint16_t*>(out);
   p.lse = lse;
@@ -419,6 +479,8 @@ mla_status_t mla_decode_paged_fp8_noalloc(const void* q, const void* blocks, con
   p.part_lse = reinterpret_cast<float*>(w + L.part_lse);
   p.part_o = reinterpret_cast<float*>(w + L.part_o);
   p.q = static_cast<const uint16_t*>(q);
+  st = make_q_map(&p.tmap_q, q, p.H, p.B * p.T);
+  if (st != MLA_OK) return st;
   p.slut = scales_lookup_table;
   p.out = static_cast<uint16_t*>(out);
   p.lse = lse;

@@ -19,15 +19,17 @@
 //           itself (256 of their 576 bytes), so no converted data crosses between SMs.
 // Every KV byte is read from HBM once (the second CTA's partial reads hit L2).
 //
-// Warp roles per CTA (448 threads):
-//   warps 0-7   converter: Q tile at each unit start; FP8 -> bf16 dequant of the tile's keys into
-//               the UMMA K-major SWIZZLE_128B layout (K half and V operand buffers); the FP8 bytes
-//               of tile g+1 are loaded into registers while tile g is converted
+// Warp roles per CTA (480 threads):
+//   warps 0-7   converter: FP8 -> bf16 dequant of the tile's keys into the UMMA K-major
+//               SWIZZLE_128B layout, K half first (its buffer frees as soon as Q.K^T of the tile two
+//               back has finished), then the V operand (its buffer frees after P.V two back); the
+//               FP8 bytes of tile g+1 are loaded into registers while tile g is converted
 //   warps 8-11  softmax: online softmax of the CTA's 64 heads (two lanes per head row), P -> SMEM,
 //               lazy O rescale, epilogue
-//   warp 12     producer: L2 prefetch of upcoming page runs
-//   warp 13     MMA issuer (CTA 0 of the pair; one elected lane issues) and TMEM owner (pair
+//   warp 12     Q.K^T issuer (CTA 0 of the pair; one elected lane issues) and TMEM owner (pair
 //               allocation in both CTAs)
+//   warp 13     P.V issuer (CTA 0)
+//   warp 14     Q loader: one TMA tile load of the CTA's 64 heads x 576 dims per unit
 #pragma once
 #include <cuda_bf16.h>
 #include <cstdint>
@@ -41,13 +43,13 @@ constexpr int HEAD_DIM = 576;
 constexpr int V_DIM = 512;
 constexpr int MROWS = 128;      // query heads per item (pair MMA M)
 constexpr int HPC = 64;         // query heads per CTA
-constexpr int NUM_THREADS = 448;
+constexpr int NUM_THREADS = 480;
 constexpr int CONV_THREADS = 256;
 constexpr int CONV_WARPS = CONV_THREADS / 32;
 constexpr int SM_WARP0 = 8;     // first softmax warp (warps 8..11 reach TMEM lane quadrants 0..3)
-constexpr int PROD_WARP = 12;
-constexpr int MMA_WARP = 13;
-constexpr int PF_DIST = 4;      // tiles of L2 prefetch lead
+constexpr int QK_WARP = 12;     // Q.K^T issuer (CTA 0), TMEM owner (both CTAs)
+constexpr int PV_WARP = 13;     // P.V issuer (CTA 0)
+constexpr int Q_WARP = 14;      // Q tile loader
 
 // ---- shared memory map (offsets from a 1024-byte aligned base); all operands K-major SWIZZLE_128B,
 //      one "atom column" = 64 bf16 dims x rows at 128 B, 8-row groups 1024 B apart
@@ -67,21 +69,24 @@ constexpr uint32_t SMEM_USED = SBAR + 256;
 constexpr uint32_t SMEM_ALLOC = SMEM_USED + 1024;   // slack for aligning the base
 
 enum Bar : uint32_t {
-  B_KV_FULL = 0,   // [2] CTA 0: 16 warp arrivals (8 converter warps of each CTA)
-  B_PV_DONE = 2,   // [2] both CTAs: pair commit after P.V of a tile (its K/V/P buffers are free)
-  B_S_FULL = 4,    // [2] both CTAs: pair commit after Q.K^T of a tile
-  B_P_FULL = 6,    // [2] CTA 0: 8 warp arrivals (4 softmax warps of each CTA)
-  B_Q_FULL = 8,    // CTA 0: 16 warp arrivals (converter warps)
-  B_Q_FREE = 9,    // both CTAs: pair commit after the last Q.K^T of a unit
-  B_O_FREE = 10,   // CTA 0: 8 warp arrivals after each CTA's epilogue
-  B_DRAIN = 11,
-  B_RED = 12,      // [2] softmax warps of this CTA: row-max exchange of a tile (4 warp arrivals)
-  B_REDL = 14,     // softmax warps of this CTA: row-sum exchange at a unit's end (4 warp arrivals)
-  NUM_BARS = 15
+  B_K_FULL = 0,    // [2] CTA 0: 16 warp arrivals (8 converter warps of each CTA): K half converted
+  B_V_FULL = 2,    // [2] CTA 0: 16 warp arrivals: V operand converted
+  B_PV_DONE = 4,   // [2] both CTAs: pair commit after P.V of a tile (its V and P buffers are free)
+  B_S_FULL = 6,    // [2] both CTAs: pair commit after Q.K^T of a tile (its K buffer is free)
+  B_S_FREE = 8,    // [2] CTA 0: 8 warp arrivals (4 softmax warps of each CTA hold S in registers)
+  B_P_FULL = 10,   // [2] CTA 0: 8 warp arrivals
+  B_Q_FULL = 12,   // CTA 0: 2 arrivals (the Q loader of each CTA)
+  B_Q_FREE = 13,   // both CTAs: pair commit after the last Q.K^T of a unit
+  B_Q_LOCAL = 14,  // both CTAs: transaction barrier of this CTA's Q tile load
+  B_O_FREE = 15,   // CTA 0: 8 warp arrivals after each CTA's epilogue
+  B_DRAIN = 16,    // CTA 0: one commit from each issuer at exit
+  B_RED = 17,      // [2] softmax warps of this CTA: row-max exchange of a tile (4 warp arrivals)
+  B_REDL = 19,     // softmax warps of this CTA: row-sum exchange at a unit's end (4 warp arrivals)
+  NUM_BARS = 20
 };
-constexpr uint32_t S_TMEM_BASE = SBAR + 128;
-constexpr uint32_t S_ABORT = SBAR + 132;
-constexpr uint32_t S_CONV_TILE = SBAR + 136;
+static_assert(8 * NUM_BARS <= 192, "barrier block overlaps the scalars after it");
+constexpr uint32_t S_TMEM_BASE = SBAR + 192;
+constexpr uint32_t S_ABORT = SBAR + 196;
 
 // TMEM columns (pair layout)
 constexpr uint32_t T_O = 0;                      // P.V halves: cols 0..127 (dims 0..255), 128..255 (256..511)
@@ -100,7 +105,22 @@ constexpr uint64_t WAIT_LIMIT_NS = 2000000000ull;   // 2 s per wait
 constexpr int TRACE_TILES = 64;
 constexpr int TRACE_EVENTS = 32;
 
+// Unsigned 32-bit division by a divisor fixed for the launch, as a multiply-high and two shifts
+// (Granlund and Montgomery, "Division by invariant integers using multiplication", 1994, Fig. 4.1):
+// with l = ceil(log2 d) and m = floor(2^32 (2^l - d) / d) + 1,
+//   t = mulhi(m, n),  q = (t + ((n - t) >> min(l, 1))) >> max(l - 1, 0)
+// is exact for every 32-bit n.  The host fills the fields (make_fastdiv in the library).
+struct FastDiv {
+  uint32_t d, m, s1, s2;
+  __device__ __forceinline__ uint32_t div(uint32_t n) const {
+    const uint32_t t = __umulhi(n, m);
+    return (t + ((n - t) >> s1)) >> s2;
+  }
+  __device__ __forceinline__ uint32_t mod(uint32_t n) const { return n - div(n) * d; }
+};
+
 struct DecodeParams {
+  CUtensorMap tmap_q;              // q as [B*T][H][576] bf16, box 64 dims x 64 heads, SWIZZLE_128B
   unsigned long long* trace;       // null unless tracing
   const uint16_t* q;               // bf16 bits [B, T, H, 576]
   const uint8_t* blocks;           // e4m3 [NB, KVD, NL, P, 1, 576]
@@ -117,6 +137,7 @@ struct DecodeParams {
   float* part_lse;                 // [2 NC][128]
   unsigned int* status;
   int B, T, H, G, P, KVD, NL, layer, NB, NSB, max_pages, items, NC;
+  FastDiv divP, divG, divT;        // by the page size, the head-group count and the query length
   float scale_log2;                // softmax_scale * log2(e)
 };
 
@@ -142,9 +163,10 @@ struct UnitWalker {
     const int a = max(s, R0), z = min(e, R1);
     if (a >= z) return false;
     u.item = it;
-    u.g = it % p->G;
-    u.i = (it / p->G) % p->T;
-    u.b = it / (p->G * p->T);
+    const uint32_t bi = p->divG.div(it);       // it = (b * T + i) * G + g
+    u.g = it - static_cast<int>(bi) * p->G;
+    u.b = static_cast<int>(p->divT.div(bi));
+    u.i = static_cast<int>(bi) - u.b * p->T;
     u.nvis = p->item_nvis[it];
     u.tb = a - s;
     u.te = z - s;
@@ -170,59 +192,40 @@ __device__ __forceinline__ void raise_status(unsigned int* status, unsigned bits
 #else
 #define MLA_TRACE_EV(tile, ev) do {} while (0)
 #endif
+// Trace builds also record, per CTA, %globaltimer at entry, after setup and at exit, at
+// trace[2 * TRACE_TILES * TRACE_EVENTS + 4 * blockIdx.x + {0, 1, 2}].
+#ifdef MLA_TRACE
+#define MLA_TRACE_CTA(slot)                                                                           \
+  do {                                                                                                \
+    if (p.trace && threadIdx.x == 0)                                                                  \
+      p.trace[2 * TRACE_TILES * TRACE_EVENTS + 4 * blockIdx.x + (slot)] = ptx::globaltimer();         \
+  } while (0)
+#else
+#define MLA_TRACE_CTA(slot) do {} while (0)
+#endif
 
-// Bounded waits on an mbarrier phase.  wait_bar: CTA-scope acquire, for barriers arrived on by
-// this CTA's threads or by tcgen05 commits.  wait_bar_cl: cluster-scope acquire, for barriers the
-// other CTA's threads arrive on (their shared-memory writes must be visible afterwards).  Both
-// return false (and mark the CTA, its peer and the status word) when the wait gives up or another
-// role already gave up.
-template <bool CLUSTER>
-__device__ __noinline__ bool wait_bar_slow(uint32_t addr, uint32_t parity, volatile uint32_t* abort,
-                                           unsigned int* status, uint32_t peer_abort) {
-  const uint64_t t0 = ptx::globaltimer();
-  while (true) {
-    for (int i = 0; i < 16; ++i) {
-      if (CLUSTER ? ptx::mbar_try_wait_acq_cluster(addr, parity) : ptx::mbar_try_wait_sleep(addr, parity, 100000u))
-        return true;
-    }
-    if (*abort) return false;
-    if (ptx::globaltimer() - t0 > WAIT_LIMIT_NS) {
-      *abort = 1u;
-      if (peer_abort) ptx::st_cluster_u32(peer_abort, 1u);
-      raise_status(status, STATUS_TIMEOUT);
-      return false;
-    }
+// Bounded wait on an mbarrier phase (CTA-scope acquire; barriers arrived on by this CTA's threads,
+// by the peer CTA's threads through remote arrives, or by tcgen05 commits).  Returns false when the
+// wait gives up or another role already gave up; the first to give up marks the CTA, its peer and
+// the status word.  The loop is kept small (it is inlined at every wait) and the give-up path is
+// out of line.
+__device__ __noinline__ bool wait_gave_up(volatile uint32_t* abort, unsigned int* status, uint32_t peer_abort) {
+  if (!*abort) {
+    *abort = 1u;
+    if (peer_abort) ptx::st_cluster_u32(peer_abort, 1u);
+    raise_status(status, STATUS_TIMEOUT);
   }
+  return false;
 }
 
 __device__ __forceinline__ bool wait_bar(uint32_t addr, uint32_t parity, volatile uint32_t* abort,
                                          unsigned int* status, uint32_t peer_abort) {
   if (ptx::mbar_try_wait(addr, parity)) return true;
-  return wait_bar_slow<false>(addr, parity, abort, status, peer_abort);
-}
-
-__device__ __forceinline__ bool wait_bar_cl(uint32_t addr, uint32_t parity, volatile uint32_t* abort,
-                                            unsigned int* status, uint32_t peer_abort) {
-  if (ptx::mbar_try_wait_acq_cluster(addr, parity)) return true;
-  return wait_bar_slow<true>(addr, parity, abort, status, peer_abort);
-}
-
-// ---------------------------------------------------------------------------------------------
-// Page-table gather: where token `tok` of request b lives (value row and scale).  Out-of-range
-// page ids are reported (false) instead of being dereferenced.
-// ---------------------------------------------------------------------------------------------
-__device__ __forceinline__ bool row_source(const DecodeParams& p, int b, int tok, const uint8_t*& vptr,
-                                           const float*& sptr) {
-  const int page = tok / p.P;
-  const int slot = tok - page * p.P;
-  if (page >= p.max_pages) return false;
-  const uint32_t blk = __ldg(p.lut + static_cast<size_t>(b) * p.max_pages + page);
-  const uint32_t sblk = p.slut ? __ldg(p.slut + static_cast<size_t>(b) * p.max_pages + page) : blk;
-  if (blk >= static_cast<uint32_t>(p.NB) || sblk >= static_cast<uint32_t>(p.NSB)) return false;
-  const size_t row = ((static_cast<size_t>(blk) * p.KVD) * p.NL + p.layer) * p.P + slot;
-  const size_t srow = ((static_cast<size_t>(sblk) * p.KVD) * p.NL + p.layer) * p.P + slot;
-  vptr = p.blocks + row * HEAD_DIM;
-  sptr = p.scales + srow;
+  const uint64_t t0 = ptx::globaltimer();
+  while (!ptx::mbar_try_wait_sleep(addr, parity, 20000u)) {
+    if (*abort) return false;
+    if (ptx::globaltimer() - t0 > WAIT_LIMIT_NS) return wait_gave_up(abort, status, peer_abort);
+  }
   return true;
 }
 
@@ -257,11 +260,28 @@ __device__ __forceinline__ void st_chunk(uint32_t atom_base, int row, int u0, co
   ptx::st_shared_v4(atom_base + sw128_off(row, u0 + 1), w[4], w[5], w[6], w[7]);
 }
 
-// The FP8 bytes of one tile that one converter thread converts.  Thread t (of 256) owns row t >> 3
-// of both key halves and the 16-byte chunks (t & 7) + 8k:
+// Converter thread t (of 256) owns key row conv_row(t) (0..31) of both key halves and the 16-byte
+// chunks conv_q(t) + 8k of it.  Each group of 8 consecutive threads (one phase of a 16-byte shared
+// store) covers chunk slots 0..3 of two adjacent rows, so that its 8 stores land on 8 different
+// 16-byte positions of the 128-byte swizzle row (even rows on even positions, odd rows on odd
+// ones); each warp still reads 4 whole rows (coalesced).
+__device__ __forceinline__ int conv_row(int t) { return ((t >> 4) << 1) | ((t >> 2) & 1); }
+__device__ __forceinline__ int conv_q(int t) { return (t & 3) | (((t >> 3) & 1) << 2); }
+
+// The FP8 bytes of one tile that one converter thread converts: of row conv_row(t) and chunks
+// conv_q(t) + 8k,
 //   own key   32c + row    : the 36 chunks of its 576-byte row (576 dims) -> K half buffer; its D_c
 //                            chunks also -> V buffer
 //   other key 32(1-c) + row: the 16 chunks of D_c -> V buffer
+// Register slot s (0..4) of RawTile::own holds chunk conv_q(t) + 8 * own_k(s, c) of the own key:
+// slot 0 the chunk past dim 512 (k = 4; only threads with conv_q(t) < 4 have one), slots 1 and 2 the
+// two chunks outside D_c, slots 3 and 4 the two inside D_c (k = c and 2 + c).  With this order the
+// converter finds the V chunks in fixed registers whichever CTA of the pair it runs in, so both CTAs
+// run the same code.
+__device__ __forceinline__ int own_k(int s, int c) {
+  return s == 0 ? 4 : s == 1 ? 1 - c : s == 2 ? 3 - c : s == 3 ? c : 2 + c;
+}
+
 struct RawTile {
   uint4 own[5];
   uint4 oth[2];
@@ -287,14 +307,14 @@ struct TilePtrs {                 // row indices into blocks / scales (both < 2^
 };
 
 __device__ __forceinline__ LutVals lut_issue(const DecodeParams& p, int c, int t, int b, int nvis, int j) {
-  const int row = t >> 3;
+  const int row = conv_row(t);
   LutVals V;
   V.otok = j * BN + HALF_BN * c + row;
   V.ptok = j * BN + HALF_BN * (1 - c) + row;
   V.bad = false;
   const uint32_t* lrow = p.lut + static_cast<size_t>(b) * p.max_pages;
   const uint32_t* srow = p.slut ? p.slut + static_cast<size_t>(b) * p.max_pages : lrow;
-  const int opage = V.otok / p.P, ppage = V.ptok / p.P;
+  const int opage = static_cast<int>(p.divP.div(V.otok)), ppage = static_cast<int>(p.divP.div(V.ptok));
   V.own_in = V.otok < nvis;
   V.oth_in = V.ptok < nvis;
   if (V.own_in && opage >= p.max_pages) { V.own_in = false; V.bad = true; }
@@ -312,7 +332,7 @@ __device__ __forceinline__ TilePtrs lut_finish(const DecodeParams& p, const LutV
   T.oth_ok = V.oth_in && V.pb < static_cast<uint32_t>(p.NB) && V.psb < static_cast<uint32_t>(p.NSB);
   if (V.own_in && !T.own_ok) bad = true;
   if (V.oth_in && !T.oth_ok) bad = true;
-  const uint32_t oslot = static_cast<uint32_t>(V.otok % p.P), pslot = static_cast<uint32_t>(V.ptok % p.P);
+  const uint32_t oslot = p.divP.mod(V.otok), pslot = p.divP.mod(V.ptok);
   const uint32_t per_blk = static_cast<uint32_t>(p.KVD * p.NL * p.P);
   const uint32_t lay = static_cast<uint32_t>(p.layer * p.P);
   T.ov = V.ob * per_blk + lay + oslot;
@@ -323,16 +343,16 @@ __device__ __forceinline__ TilePtrs lut_finish(const DecodeParams& p, const LutV
 }
 
 __device__ __forceinline__ void fetch(const DecodeParams& p, const TilePtrs& T, int c, int t, RawTile& R) {
-  const int q = t & 7;
+  const int q = conv_q(t);
   R.own_ok = T.own_ok;
   R.oth_ok = T.oth_ok;
   if (T.own_ok) {
     const uint8_t* ov = p.blocks + static_cast<size_t>(T.ov) * HEAD_DIM;
     R.so = __ldg(p.scales + T.os);
 #pragma unroll
-    for (int k = 0; k < 5; ++k) {
-      const int qq = q + 8 * k;
-      if (qq < 36) R.own[k] = ptx::ldg_stream_v4(ov + 16 * qq);
+    for (int sl = 0; sl < 5; ++sl) {
+      const int qq = q + 8 * own_k(sl, c);
+      if (qq < 36) R.own[sl] = ptx::ldg_stream_v4(ov + 16 * qq);
     }
   }
   if (T.oth_ok) {
@@ -357,24 +377,23 @@ __device__ __forceinline__ bool load_tile(const DecodeParams& p, int c, int t, i
 
 // Dequantises thread t's part of a loaded tile into the K half buffer `sk` and the V buffer `sv`.
 __device__ __forceinline__ void store_tile(int c, int t, const RawTile& R, uint32_t sk, uint32_t sv) {
-  const int row = t >> 3, q = t & 7;
+  const int row = conv_row(t), q = conv_q(t);
   const int vrow_own = HALF_BN * c + row;
   const int vrow_oth = HALF_BN * (1 - c) + row;
 #pragma unroll
-  for (int k = 0; k < 5; ++k) {
-    const int qq = q + 8 * k;                                // chunk of the 576-byte row
+  for (int sl = 0; sl < 5; ++sl) {
+    const int qq = q + 8 * own_k(sl, c);                     // chunk of the 576-byte row
     if (qq >= 36) continue;
     uint32_t w[8];
     if (R.own_ok) {
-      dequant16(R.own[k], R.so, w);
+      dequant16(R.own[sl], R.so, w);
     } else {
 #pragma unroll
       for (int x = 0; x < 8; ++x) w[x] = 0u;
     }
     st_chunk(sk + (qq >> 2) * SK_ATOM, row, (qq & 3) * 2, w);
-    const int blk128 = qq >> 3;                              // 128-dim block of the latent
-    if (blk128 == c || blk128 == 2 + c) {
-      const int jc = (qq & 7) + (blk128 >= 2 ? 8 : 0);
+    if (sl >= 3) {                                           // D_c chunk: V chunk q (slot 3) or q + 8 (slot 4)
+      const int jc = q + (sl == 4 ? 8 : 0);
       st_chunk(sv + (jc >> 2) * SV_ATOM, vrow_own, (jc & 3) * 2, w);
     }
   }
@@ -390,6 +409,63 @@ __device__ __forceinline__ void store_tile(int c, int t, const RawTile& R, uint3
     }
     st_chunk(sv + (jc >> 2) * SV_ATOM, vrow_oth, (jc & 3) * 2, w);
   }
+}
+
+// The decode's converter writes the two operands of a tile at different times: the K half as soon
+// as its buffer is free (store_k), the V operand once P.V two tiles back has finished (store_v).
+// store_k keeps the two chunks of the own key that also belong to the V operand (slots 3 and 4:
+// V chunks q and q + 8) so that store_v need not convert them again; they come last so that they
+// occupy registers only once the other chunks are done.
+__device__ __forceinline__ void store_k(int c, int t, const RawTile& R, uint32_t sk, uint32_t (&keep0)[8],
+                                        uint32_t (&keep1)[8]) {
+  const int row = conv_row(t), q = conv_q(t);
+#pragma unroll
+  for (int sl = 0; sl < 5; ++sl) {
+    const int qq = q + 8 * own_k(sl, c);
+    if (qq >= 36) continue;
+    uint32_t w[8];
+    if (R.own_ok) {
+      dequant16(R.own[sl], R.so, w);
+    } else {
+#pragma unroll
+      for (int x = 0; x < 8; ++x) w[x] = 0u;
+    }
+    st_chunk(sk + (qq >> 2) * SK_ATOM, row, (qq & 3) * 2, w);
+    if (sl == 3) {
+#pragma unroll
+      for (int x = 0; x < 8; ++x) keep0[x] = w[x];
+    }
+    if (sl == 4) {
+#pragma unroll
+      for (int x = 0; x < 8; ++x) keep1[x] = w[x];
+    }
+  }
+}
+
+__device__ __forceinline__ void store_v(int c, int t, const RawTile& R, const uint32_t (&keep0)[8],
+                                        const uint32_t (&keep1)[8], uint32_t sv) {
+  const int row = conv_row(t), q = conv_q(t);
+  const int vrow_own = HALF_BN * c + row;
+  const int vrow_oth = HALF_BN * (1 - c) + row;
+  st_chunk(sv + (q >> 2) * SV_ATOM, vrow_own, (q & 3) * 2, keep0);
+  st_chunk(sv + ((q + 8) >> 2) * SV_ATOM, vrow_own, (q & 3) * 2, keep1);
+#pragma unroll
+  for (int k = 0; k < 2; ++k) {
+    const int jc = q + 8 * k;
+    uint32_t w[8];
+    if (R.oth_ok) {
+      dequant16(R.oth[k], R.sp, w);
+    } else {
+#pragma unroll
+      for (int x = 0; x < 8; ++x) w[x] = 0u;
+    }
+    st_chunk(sv + (jc >> 2) * SV_ATOM, vrow_oth, (jc & 3) * 2, w);
+  }
+}
+
+// Request index of an item (items are ordered (b, i, g)).
+__device__ __forceinline__ int item_b(const DecodeParams& p, int item) {
+  return static_cast<int>(p.divT.div(p.divG.div(item)));
 }
 
 // What the converter needs to know about one tile (request, query token and head group follow
@@ -452,49 +528,89 @@ struct TileCursor {
   }
 };
 
-// Q rows 64c..64c+63 of an item's head group (all 576 dims) into the SW128 K-major layout, by the
-// 256 converter threads.  Rows whose head index is >= H are zero.
-__device__ __forceinline__ void load_q(const DecodeParams& p, int b, int i, int g, int c, int t, uint32_t sq) {
-  const uint16_t* qrow0 = p.q + (static_cast<size_t>(b) * p.T + i) * p.H * HEAD_DIM;
-  const int h0 = g * MROWS + HPC * c;
-#pragma unroll 1
-  for (int batch = 0; batch < 2; ++batch) {
-    uint4 v[9];
-#pragma unroll
-    for (int k = 0; k < 9; ++k) {
-      const int id = (batch * 9 + k) * CONV_THREADS + t;   // 64 rows x 72 chunks of 8 bf16
-      const int row = id / 72, cc = id - row * 72;
-      v[k] = make_uint4(0, 0, 0, 0);
-      if (h0 + row < p.H)
-        v[k] = __ldg(reinterpret_cast<const uint4*>(qrow0 + static_cast<size_t>(h0 + row) * HEAD_DIM + cc * 8));
-    }
-#pragma unroll
-    for (int k = 0; k < 9; ++k) {
-      const int id = (batch * 9 + k) * CONV_THREADS + t;
-      const int row = id / 72, cc = id - row * 72;
-      ptx::st_shared_v4(sq + SQ + (cc >> 3) * SQ_ATOM + sw128_off(row, cc & 7), v[k].x, v[k].y, v[k].z, v[k].w);
-    }
+// =============================================================================================
+// converter role (warps 0-7); the same code in both CTAs of the pair (c = rank).
+// Software pipeline over the tile sequence: while tile g is converted, the FP8 bytes of tile g+1 are
+// in flight and the page-table entries of tile g+2 are being read.  Buffers alternate by tile
+// parity; the K half of tile g waits for Q.K^T(g-2) (S_FULL), the V operand for P.V(g-2).
+// Returns early (with the abort flag set by the failing wait) when a wait gives up.
+// =============================================================================================
+__device__ __forceinline__ void converter_role(const DecodeParams& p, int k, uint32_t base, int lane,
+                                               volatile uint32_t* abort, uint32_t peer_abort, uint32_t c) {
+  const int C = static_cast<int>(c);
+  const int t = threadIdx.x;
+#define BAR(i) (base + SBAR + 8u * (i))
+#define MLA_WAIT_RET(b_, parity)                                                               \
+  if (!__all_sync(0xffffffffu, wait_bar((b_), (parity), abort, p.status, peer_abort))) return;
+  const uint32_t k_full0 = ptx::mapa(BAR(B_K_FULL), 0), v_full0 = ptx::mapa(BAR(B_V_FULL), 0);
+  TileStream ts(p, k);
+  TileInfo cur = ts.take();
+  if (!cur.valid) return;
+  TileInfo n1 = ts.take();
+  TileInfo n2 = ts.take();
+  RawTile ra, rb;
+  bool bad = false;
+  {
+    const TilePtrs t0 = lut_finish(p, lut_issue(p, C, t, item_b(p, cur.item), cur.nvis, cur.j), bad);
+    if (bad) raise_status(p.status, STATUS_BOUNDS);
+    fetch(p, t0, C, t, ra);
   }
-}
-
-// L2 prefetch of the value rows and scales of CTA c's own keys of tile j (whole page runs).
-__device__ __forceinline__ void prefetch_tile(const DecodeParams& p, int c, int b, int nvis, int j) {
-  const int first = j * BN + HALF_BN * c;
-  int tok = first;
-  const int end = min(first + HALF_BN, nvis);
-  while (tok < end) {
-    const int page = tok / p.P;
-    const int slot = tok - page * p.P;
-    const int run = min(end - tok, p.P - slot);
-    const uint8_t* vptr;
-    const float* sptr;
-    if (row_source(p, b, tok, vptr, sptr)) {
-      ptx::prefetch_l2(vptr, static_cast<uint32_t>(run) * HEAD_DIM);
-      // the whole page's scale run (P * 4 bytes, 64-byte aligned because P % 16 == 0)
-      if (slot == 0 || tok == first) ptx::prefetch_l2(sptr - slot, static_cast<uint32_t>(p.P) * 4);
-    }
-    tok += run;
+  TilePtrs t1{};
+  if (n1.valid) {
+    t1 = lut_finish(p, lut_issue(p, C, t, item_b(p, n1.item), n1.nvis, n1.j), bad);
+    if (bad) raise_status(p.status, STATUS_BOUNDS);
   }
+  uint32_t g = 0;
+  // One tile: convert RCUR while RNXT (the next tile) is being fetched.
+#define MLA_CONV_STEP(RCUR, RNXT)                                                                        \
+  {                                                                                                      \
+    const uint32_t kb = g & 1, free_par = ((g >> 1) & 1) ^ 1;                                           \
+    MLA_WAIT_RET(BAR(B_S_FULL + kb), free_par);                                                          \
+    if (t == 0) MLA_TRACE_EV(g, 1);                                                                      \
+    if (t == 224) MLA_TRACE_EV(g, 26);                                                                   \
+    if (n1.valid) fetch(p, t1, C, t, RNXT);                                                              \
+    if (t == 0) MLA_TRACE_EV(g, 16);                                                                     \
+    LutVals v2{};                                                                                        \
+    if (n2.valid) v2 = lut_issue(p, C, t, item_b(p, n2.item), n2.nvis, n2.j);                         \
+    if (t == 0) MLA_TRACE_EV(g, 4);                                                                      \
+    if (t == 224) MLA_TRACE_EV(g, 27);                                                                   \
+    uint32_t keep0[8], keep1[8];                                                                         \
+    store_k(C, t, RCUR, base + SK0 + kb * SK_STRIDE, keep0, keep1);                                      \
+    ptx::fence_proxy_async_smem();                                                                       \
+    __syncwarp();                                                                                        \
+    if (lane == 0) ptx::mbar_arrive_cluster(k_full0 + 8u * kb);                                          \
+    if (t == 0) MLA_TRACE_EV(g, 5);                                                                      \
+    if (t == 224) MLA_TRACE_EV(g, 28);                                                                   \
+    MLA_WAIT_RET(BAR(B_PV_DONE + kb), free_par);                                                         \
+    if (t == 0) MLA_TRACE_EV(g, 6);                                                                      \
+    if (t == 224) MLA_TRACE_EV(g, 29);                                                                   \
+    store_v(C, t, RCUR, keep0, keep1, base + SV0 + kb * SV_STRIDE);                                      \
+    ptx::fence_proxy_async_smem();                                                                       \
+    __syncwarp();                                                                                        \
+    if (lane == 0) ptx::mbar_arrive_cluster(v_full0 + 8u * kb);                                          \
+    if (t == 0) MLA_TRACE_EV(g, 2);                                                                      \
+    if (t == 224) MLA_TRACE_EV(g, 30);                                                                   \
+    if (n2.valid) {                                                                                      \
+      t1 = lut_finish(p, v2, bad);                                                                       \
+      if (bad) raise_status(p.status, STATUS_BOUNDS);                                                    \
+    }                                                                                                    \
+    if (t == 0) MLA_TRACE_EV(g, 7);                                                                      \
+    if (t == 224) MLA_TRACE_EV(g, 31);                                                                   \
+    ++g;                                                                                                 \
+  }
+  // Rolled loop (one copy of the step keeps the hot code small): the next tile's bytes move from
+  // rb to ra at the end of a step, when they have normally arrived.
+  while (true) {
+    MLA_CONV_STEP(ra, rb)
+    if (!n1.valid) break;
+    ra = rb;
+    cur = n1;
+    n1 = n2;
+    n2 = ts.take();
+  }
+#undef MLA_CONV_STEP
+#undef MLA_WAIT_RET
+#undef BAR
 }
 
 // =============================================================================================
@@ -509,29 +625,30 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) mla_decode_kernel(const __grid
   const uint32_t peer = c ^ 1u;
   const int k = static_cast<int>(ptx::cluster_id_x());
   volatile uint32_t* abort = reinterpret_cast<volatile uint32_t*>(smem + S_ABORT);
-  volatile uint32_t* conv_tile = reinterpret_cast<volatile uint32_t*>(smem + S_CONV_TILE);
   const uint32_t peer_abort = ptx::mapa(base + S_ABORT, peer);
 #define BAR(i) (base + SBAR + 8u * (i))
+  MLA_TRACE_CTA(0);
 
   if (threadIdx.x == 0) {
     for (uint32_t i = 0; i < 2; ++i) {
-      ptx::mbar_init(BAR(B_KV_FULL + i), 2 * CONV_WARPS);
+      ptx::mbar_init(BAR(B_K_FULL + i), 2 * CONV_WARPS);
+      ptx::mbar_init(BAR(B_V_FULL + i), 2 * CONV_WARPS);
       ptx::mbar_init(BAR(B_PV_DONE + i), 1);
       ptx::mbar_init(BAR(B_S_FULL + i), 1);
+      ptx::mbar_init(BAR(B_S_FREE + i), 8);
       ptx::mbar_init(BAR(B_P_FULL + i), 8);
+      ptx::mbar_init(BAR(B_RED + i), 4);
     }
-    ptx::mbar_init(BAR(B_Q_FULL), 2 * CONV_WARPS);
+    ptx::mbar_init(BAR(B_Q_FULL), 2);
     ptx::mbar_init(BAR(B_Q_FREE), 1);
+    ptx::mbar_init(BAR(B_Q_LOCAL), 1);
     ptx::mbar_init(BAR(B_O_FREE), 8);
-    ptx::mbar_init(BAR(B_DRAIN), 1);
-    ptx::mbar_init(BAR(B_RED + 0), 4);
-    ptx::mbar_init(BAR(B_RED + 1), 4);
+    ptx::mbar_init(BAR(B_DRAIN), 2);
     ptx::mbar_init(BAR(B_REDL), 4);
     *abort = 0u;
-    *conv_tile = 0u;
     ptx::fence_mbar_init();
   }
-  if (warp == MMA_WARP) {
+  if (warp == QK_WARP) {
     ptx::tmem_alloc_pair(base + S_TMEM_BASE, TMEM_COLS);
     ptx::tmem_relinquish_pair();
   }
@@ -540,93 +657,24 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) mla_decode_kernel(const __grid
   ptx::cluster_sync();   // the peer's barriers exist before any remote arrive
   ptx::tc_fence_after();
   const uint32_t tbase = *reinterpret_cast<volatile uint32_t*>(smem + S_TMEM_BASE);
+  MLA_TRACE_CTA(1);
 
 // Whole-warp roles bail out together so that the warp-collective instructions after a wait never
 // run on a partial warp.
 #define MLA_WAIT_WARP(b_, parity)                                                              \
   if (!__all_sync(0xffffffffu, wait_bar((b_), (parity), abort, p.status, peer_abort))) goto role_done;
-#define MLA_WAIT_WARP_CL(b_, parity)                                                           \
-  if (!__all_sync(0xffffffffu, wait_bar_cl((b_), (parity), abort, p.status, peer_abort))) goto role_done;
 
   if (warp < CONV_WARPS) {
     // ------------------------------------------------------------------ converter
-    // Software pipeline over the tile sequence: while tile g is converted, the FP8 bytes of tile g+1
-    // are in flight and the page-table entries of tile g+2 are being read.
-    const int t = threadIdx.x;
-    const int cc = static_cast<int>(c);
-    const uint32_t kv_full0 = ptx::mapa(BAR(B_KV_FULL), 0), q_full = ptx::mapa(BAR(B_Q_FULL), 0);
-    TileStream ts(p, k);
-    TileInfo cur = ts.take();
-    if (cur.valid) {
-      TileInfo n1 = ts.take();
-      TileInfo n2 = ts.take();
-      RawTile ra, rb;
-      bool bad = false;
-      {
-        const TilePtrs t0 = lut_finish(p, lut_issue(p, cc, t, cur.item / (p.G * p.T), cur.nvis, cur.j), bad);
-        if (bad) raise_status(p.status, STATUS_BOUNDS);
-        fetch(p, t0, cc, t, ra);
-      }
-      TilePtrs t1{};
-      if (n1.valid) {
-        t1 = lut_finish(p, lut_issue(p, cc, t, n1.item / (p.G * p.T), n1.nvis, n1.j), bad);
-        if (bad) raise_status(p.status, STATUS_BOUNDS);
-      }
-      uint32_t g = 0, uu = 0;
-      // One tile.  Unrolled twice below so that the two register sets alternate statically.
-#define MLA_CONV_STEP(RCUR, RNXT)                                                                        \
-      {                                                                                                  \
-        if (cur.first) {                                                                                 \
-          MLA_WAIT_WARP(BAR(B_Q_FREE), (uu & 1) ^ 1);                                                    \
-          if (t == 0) MLA_TRACE_EV(g, 3);                                                                \
-          load_q(p, cur.item / (p.G * p.T), (cur.item / p.G) % p.T, cur.item % p.G, cc, t, base);         \
-          ptx::fence_proxy_async_smem();                                                                 \
-          __syncwarp();                                                                                  \
-          if (lane == 0) ptx::mbar_arrive_cluster(q_full);                                               \
-          ++uu;                                                                                          \
-        }                                                                                                \
-        const uint32_t kb = g & 1;                                                                       \
-        MLA_WAIT_WARP(BAR(B_PV_DONE + kb), ((g >> 1) & 1) ^ 1);                                          \
-        if (t == 0) MLA_TRACE_EV(g, 1);                                                                  \
-        if (n1.valid) fetch(p, t1, cc, t, RNXT);                                                         \
-        LutVals v2{};                                                                                    \
-        if (n2.valid) v2 = lut_issue(p, cc, t, n2.item / (p.G * p.T), n2.nvis, n2.j);                    \
-        if (t == 0) MLA_TRACE_EV(g, 4);                                                                  \
-        store_tile(cc, t, RCUR, base + SK0 + kb * SK_STRIDE, base + SV0 + kb * SV_STRIDE);               \
-        ptx::fence_proxy_async_smem();                                                                   \
-        __syncwarp();                                                                                    \
-        if (lane == 0) ptx::mbar_arrive_cluster(kv_full0 + 8u * kb);                                     \
-        if (t == 0) {                                                                                    \
-          *conv_tile = g + 1;                                                                            \
-          MLA_TRACE_EV(g, 2);                                                                            \
-        }                                                                                                \
-        if (n2.valid) {                                                                                  \
-          t1 = lut_finish(p, v2, bad);                                                                   \
-          if (bad) raise_status(p.status, STATUS_BOUNDS);                                                \
-        }                                                                                                \
-        ++g;                                                                                             \
-      }
-      while (true) {
-        MLA_CONV_STEP(ra, rb)
-        if (!n1.valid) break;
-        cur = n1;
-        n1 = n2;
-        n2 = ts.take();
-        MLA_CONV_STEP(rb, ra)
-        if (!n1.valid) break;
-        cur = n1;
-        n1 = n2;
-        n2 = ts.take();
-      }
-#undef MLA_CONV_STEP
-    }
+    converter_role(p, k, base, lane, abort, peer_abort, c);
   } else if (warp < SM_WARP0 + 4) {
     // ------------------------------------------------------------------ softmax / epilogue
     const int t = threadIdx.x - 32 * SM_WARP0;
     const int quad = warp - SM_WARP0;
     const int r = t & 63, hh = t >> 6;             // head row within the CTA, key half of the tile
     const uint32_t lane_base = tbase + (static_cast<uint32_t>(quad * 32) << 16);
-    const uint32_t p_full0 = ptx::mapa(BAR(B_P_FULL), 0), o_free = ptx::mapa(BAR(B_O_FREE), 0);
+    const uint32_t p_full0 = ptx::mapa(BAR(B_P_FULL), 0), s_free0 = ptx::mapa(BAR(B_S_FREE), 0);
+    const uint32_t o_free = ptx::mapa(BAR(B_O_FREE), 0);
     volatile float* red_max = reinterpret_cast<volatile float*>(smem + SRED);
     volatile float* red_l = reinterpret_cast<volatile float*>(smem + SRED + 1024);
     UnitWalker wk(p, k);
@@ -647,6 +695,10 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) mla_decode_kernel(const __grid
 #pragma unroll
           for (int q = 0; q < 32; ++q) x[q] = __uint_as_float(rr[q]);
         }
+        // S buffer sb may be overwritten by Q.K^T(g + 2) from here on
+        ptx::tc_fence_before();
+        __syncwarp();
+        if (lane == 0) ptx::mbar_arrive_cluster(s_free0 + 8u * sb);
         if (t == 0) MLA_TRACE_EV(g, 9);
         const int nv = min(BN, u.nvis - j * BN) - HALF_BN * hh;   // valid keys in this lane's half
         float mt = -INFINITY;
@@ -681,6 +733,9 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) mla_decode_kernel(const __grid
         }
         l += lsum;
         if (t == 0) MLA_TRACE_EV(g, 11);
+        // P buffer sb is free once P.V(g - 2) has finished
+        MLA_WAIT_WARP(BAR(B_PV_DONE + sb), ((g >> 1) & 1) ^ 1);
+        if (t == 0) MLA_TRACE_EV(g, 13);
         {
           const uint32_t sp = base + SP0 + sb * SP_STRIDE;
 #pragma unroll
@@ -768,121 +823,111 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) mla_decode_kernel(const __grid
       }
       ++uu;
     }
-  } else if (warp == PROD_WARP) {
-    // ------------------------------------------------------------------ producer: L2 prefetch
+  } else if (warp == Q_WARP) {
+    // ------------------------------------------------------------------ Q loader (both CTAs)
+    // Per unit: wait until the last Q.K^T of the previous unit has finished, then one TMA load per
+    // 64-dim atom column of the CTA's 64 heads (heads past H read as zero).
     if (lane == 0) {
+      const uint32_t q_full = ptx::mapa(BAR(B_Q_FULL), 0);
+      ptx::prefetch_tmap(&p.tmap_q);
       UnitWalker wk(p, k);
       Unit u;
-      uint32_t g = 0;
-      bool ok = true;
-      const uint64_t t0 = ptx::globaltimer();
-      while (ok && wk.next(u)) {
-        for (int j = u.tb; j < u.te && ok; ++j, ++g) {
-          while (g >= *conv_tile + PF_DIST) {
-            if (*abort || ptx::globaltimer() - t0 > 8 * WAIT_LIMIT_NS) {
-              ok = false;
-              break;
-            }
-            __nanosleep(256);
-          }
-          if (ok) prefetch_tile(p, static_cast<int>(c), u.b, u.nvis, j);
-        }
+      uint32_t uu = 0;
+      while (wk.next(u)) {
+        if (!wait_bar(BAR(B_Q_FREE), (uu & 1) ^ 1, abort, p.status, peer_abort)) break;
+        if (uu < 2 && c == 0) MLA_TRACE_EV(uu, 24);
+        ptx::mbar_arrive_expect_tx(BAR(B_Q_LOCAL), 9 * SQ_ATOM);
+#pragma unroll 1
+        for (int a = 0; a < 9; ++a)
+          ptx::tma_load_3d(base + SQ + a * SQ_ATOM, &p.tmap_q, 64 * a, u.g * MROWS + HPC * static_cast<int>(c),
+                           u.b * p.T + u.i, BAR(B_Q_LOCAL));
+        if (!wait_bar(BAR(B_Q_LOCAL), uu & 1, abort, p.status, peer_abort)) break;
+        if (uu < 2 && c == 0) MLA_TRACE_EV(uu, 25);
+        ptx::mbar_arrive_cluster(q_full);
+        ++uu;
       }
     }
-  } else if (c == 0) {
-    // ------------------------------------------------------------------ MMA issuer (CTA 0 of the pair)
+  } else if (warp == QK_WARP) {
+    // ------------------------------------------------------------------ Q.K^T issuer (CTA 0)
     // The whole warp runs the loop (descriptors stay warp-uniform); one elected lane issues.
-    // Greedy order: P.V(h) as soon as both CTAs' P(h) is in shared memory; Q.K^T(g) as soon as both
-    // CTAs' K/V tile g is converted and P.V(g - 2) (which frees score buffer g & 1) was issued.
-    TileCursor qc(p, k), pc(p, k);
-    uint32_t gq = 0, gp = 0, uq = 0, up = 0;
-    // descriptor bases; per K step only the start-address field (bits 0..13, bytes >> 4) moves
-    const uint64_t dq0 = ptx::smem_desc(base + SQ, 16, 1024, ptx::SW_128B);
-    const uint64_t dk0 = ptx::smem_desc(base + SK0, 16, 1024, ptx::SW_128B);
-    const uint64_t dp0 = ptx::smem_desc(base + SP0, 16, 1024, ptx::SW_128B);
-    const uint64_t dv0 = ptx::smem_desc(base + SV0, SV_ATOM, 1024, ptx::SW_128B);
-    uint64_t t_idle = 0;
-    while (pc.valid) {
-      bool progress = false;
-      // ---- P.V of tile gp
-      if (gp < gq) {
-        const uint32_t hb = gp & 1;
+    if (c == 0) {
+      TileCursor qc(p, k);
+      uint32_t g = 0, uq = 0;
+      // descriptor bases; per K step only the start-address field (bits 0..13, bytes >> 4) moves
+      const uint64_t dq0 = ptx::smem_desc(base + SQ, 16, 1024, ptx::SW_128B);
+      const uint64_t dk0 = ptx::smem_desc(base + SK0, 16, 1024, ptx::SW_128B);
+      while (qc.valid) {
+        const uint32_t kb = g & 1;
+        if (qc.first) {
+          MLA_WAIT_WARP(BAR(B_Q_FULL), uq & 1);
+          ++uq;
+        }
+        MLA_WAIT_WARP(BAR(B_K_FULL + kb), (g >> 1) & 1);
+        MLA_WAIT_WARP(BAR(B_S_FREE + kb), ((g >> 1) & 1) ^ 1);
+        ptx::tc_fence_after();
+        if (ptx::elect_one()) {
+          MLA_TRACE_EV(g, 20);
+          const uint32_t dS = tbase + T_S + 32 * kb;
+          // 9 atom columns of 64 dims x 4 K steps of 16 dims
+          uint64_t ad = dq0, bd = dk0 + ((kb * SK_STRIDE) >> 4);
+#pragma unroll 1
+          for (int a = 0; a < 9; ++a) {
+#pragma unroll
+            for (int kk = 0; kk < 4; ++kk)
+              ptx::mma_pair_ss(dS, ad + kk * 2, bd + kk * 2, IDESC_QK, (a | kk) != 0 ? 1u : 0u);
+            ad += SQ_ATOM >> 4;
+            bd += SK_ATOM >> 4;
+          }
+          ptx::mma_commit_pair(BAR(B_S_FULL + kb), 0x3);
+          MLA_TRACE_EV(g, 21);
+          if (qc.j == qc.u.te - 1) ptx::mma_commit_pair(BAR(B_Q_FREE), 0x3);
+        }
+        __syncwarp();
+        ++g;
+        qc.advance();
+      }
+    }
+  } else if (warp == PV_WARP) {
+    // ------------------------------------------------------------------ P.V issuer (CTA 0)
+    if (c == 0) {
+      TileCursor pc(p, k);
+      uint32_t g = 0, up = 0;
+      const uint64_t dp0 = ptx::smem_desc(base + SP0, 16, 1024, ptx::SW_128B);
+      const uint64_t dv0 = ptx::smem_desc(base + SV0, SV_ATOM, 1024, ptx::SW_128B);
+      while (pc.valid) {
+        const uint32_t hb = g & 1;
         const bool first = pc.first;
-        bool ready = ptx::mbar_test_wait(BAR(B_P_FULL + hb), (gp >> 1) & 1);
-        if (ready && first) ready = ptx::mbar_test_wait(BAR(B_O_FREE), (up & 1) ^ 1);
-        if (__all_sync(0xffffffffu, ready)) {
-          ptx::tc_fence_after();
-          if (ptx::elect_one()) {
-            MLA_TRACE_EV(gp, 22);
+        MLA_WAIT_WARP(BAR(B_V_FULL + hb), (g >> 1) & 1);
+        MLA_WAIT_WARP(BAR(B_P_FULL + hb), (g >> 1) & 1);
+        if (first) {
+          MLA_WAIT_WARP(BAR(B_O_FREE), (up & 1) ^ 1);
+          ++up;
+        }
+        ptx::tc_fence_after();
+        if (ptx::elect_one()) {
+          MLA_TRACE_EV(g, 22);
 #pragma unroll
-            for (int jv = 0; jv < 2; ++jv) {
+          for (int jv = 0; jv < 2; ++jv) {
 #pragma unroll
-              for (int kk = 0; kk < 4; ++kk) {
-                const uint64_t ad = dp0 + ((hb * SP_STRIDE + kk * 32) >> 4);
-                const uint64_t bd = dv0 + ((hb * SV_STRIDE + 2 * jv * SV_ATOM + kk * 2048) >> 4);
-                ptx::mma_pair_ss(tbase + T_O + 128 * jv, ad, bd, IDESC_PV, (first && kk == 0) ? 0u : 1u);
-              }
+            for (int kk = 0; kk < 4; ++kk) {
+              const uint64_t ad = dp0 + ((hb * SP_STRIDE + kk * 32) >> 4);
+              const uint64_t bd = dv0 + ((hb * SV_STRIDE + 2 * jv * SV_ATOM + kk * 2048) >> 4);
+              ptx::mma_pair_ss(tbase + T_O + 128 * jv, ad, bd, IDESC_PV, (first && kk == 0) ? 0u : 1u);
             }
-            ptx::mma_commit_pair(BAR(B_PV_DONE + hb), 0x3);
-            MLA_TRACE_EV(gp, 23);
           }
-          __syncwarp();
-          if (first) ++up;
-          ++gp;
-          pc.advance();
-          progress = true;
+          ptx::mma_commit_pair(BAR(B_PV_DONE + hb), 0x3);
+          MLA_TRACE_EV(g, 23);
         }
-      }
-      // ---- Q.K^T of tile gq
-      if (qc.valid && gq < gp + 2) {
-        const uint32_t kb = gq & 1;
-        bool ready = ptx::mbar_test_wait(BAR(B_KV_FULL + kb), (gq >> 1) & 1);
-        if (ready && qc.first) ready = ptx::mbar_test_wait(BAR(B_Q_FULL), uq & 1);
-        if (__all_sync(0xffffffffu, ready)) {
-          ptx::tc_fence_after();
-          if (ptx::elect_one()) {
-            MLA_TRACE_EV(gq, 20);
-            const uint32_t dS = tbase + T_S + 32 * kb;
-#pragma unroll
-            for (int ks = 0; ks < 36; ++ks) {
-              const uint32_t off = (ks & 3) * 32;
-              const uint64_t ad = dq0 + (((ks >> 2) * SQ_ATOM + off) >> 4);
-              const uint64_t bd = dk0 + ((kb * SK_STRIDE + (ks >> 2) * SK_ATOM + off) >> 4);
-              ptx::mma_pair_ss(dS, ad, bd, IDESC_QK, ks > 0 ? 1u : 0u);
-            }
-            ptx::mma_commit_pair(BAR(B_S_FULL + kb), 0x3);
-            MLA_TRACE_EV(gq, 21);
-            if (qc.j == qc.u.te - 1) ptx::mma_commit_pair(BAR(B_Q_FREE), 0x3);
-          }
-          __syncwarp();
-          if (qc.first) ++uq;
-          ++gq;
-          qc.advance();
-          progress = true;
-        }
-      }
-      if (progress) {
-        t_idle = 0;
-      } else {
-        if (t_idle == 0) t_idle = ptx::globaltimer();
-        if (*abort) goto role_done;
-        __nanosleep(128);
-        if (ptx::globaltimer() - t_idle > WAIT_LIMIT_NS) {
-          if (lane == 0) {
-            *abort = 1u;
-            ptx::st_cluster_u32(peer_abort, 1u);
-            raise_status(p.status, STATUS_TIMEOUT);
-          }
-          goto role_done;
-        }
+        __syncwarp();
+        ++g;
+        pc.advance();
       }
     }
   }
 role_done:
-#undef MLA_WAIT_WARP_CL
 #undef MLA_WAIT_WARP
   // every pair MMA issued by CTA 0 has finished before TMEM is released
-  if (c == 0 && warp == MMA_WARP && lane == 0) {
+  if (c == 0 && (warp == QK_WARP || warp == PV_WARP) && lane == 0) {
     ptx::mma_commit_pair(BAR(B_DRAIN), 0x1);
     const uint64_t t0 = ptx::globaltimer();
     while (!ptx::mbar_try_wait(BAR(B_DRAIN), 0) && ptx::globaltimer() - t0 < WAIT_LIMIT_NS) {}
@@ -890,13 +935,13 @@ role_done:
 #undef BAR
   ptx::tc_fence_before();
   __syncthreads();
+  MLA_TRACE_CTA(2);
   ptx::cluster_sync();   // no remote arrive or pair MMA targets a CTA that has exited
-  if (warp == MMA_WARP) {
+  if (warp == QK_WARP) {
     ptx::tc_fence_after();
     ptx::tmem_dealloc_pair(tbase, TMEM_COLS);
   }
 }
-
 // =============================================================================================
 // plan kernel: per-item visible keys and tile prefix, per-cluster first item (1 CTA)
 // =============================================================================================
@@ -991,7 +1036,8 @@ mla_combine_kernel(const __grid_constant__ DecodeParams p) {
   if (k0 == k1) return;
   const int w = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int h = hc * COMBINE_HEADS + w;
-  const int g = it % p.G, i = (it / p.G) % p.T, b = it / (p.G * p.T);
+  const int bi = static_cast<int>(p.divG.div(it));
+  const int g = it - bi * p.G, b = static_cast<int>(p.divT.div(bi)), i = bi - b * p.T;
   const int head = g * MROWS + h;
   if (head >= p.H) return;
   float mx = -INFINITY;

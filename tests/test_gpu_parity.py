@@ -196,6 +196,7 @@ def _custom(B, T, H, P, lengths, layers=1, layer_idx=0, kv_dim=1, seed=5, separa
     dict(B=2, T=1, H=128, P=256, lengths=(1000, 4000), layers=3, layer_idx=2, kv_dim=2),
     dict(B=4, T=1, H=128, P=16, lengths=(1, 2, 3, 4), separate=True),
     dict(B=1, T=1, H=1, P=64, lengths=(5000,)),
+    dict(B=2, T=2, H=256, P=80, lengths=(300, 77)),                 # G = 2 and T = 2 together, page size 80
 ])
 def test_edge_cases(case):
     inp = _custom(**case)
