@@ -236,6 +236,50 @@ unsigned int* status_ptr() {
   return p;
 }
 
+// The three launches of one decode call on `stream`: plan -> decode -> combine.  The decode and
+// combine kernels are launched as programmatic dependents of the kernel before them, so their
+// launch and (for the decode kernel) prologue overlap the previous kernel; each waits for its
+// predecessor's results with griddepcontrol.wait.  With timing events set, the events bracket the
+// decode launch (the event between plan and decode then serialises the two).
+mla_status_t launch_path(const mla::DecodeParams& p, int NC, const uint32_t* cache_lengths, uint32_t max_cache_length,
+                         cudaStream_t stream, bool timing) {
+  mla::mla_plan_kernel<<<1, mla::PLAN_THREADS, 0, stream>>>(
+      cache_lengths, p.B, p.T, p.G, max_cache_length, NC, const_cast<int32_t*>(p.item_start),
+      const_cast<int32_t*>(p.item_nvis), const_cast<int32_t*>(p.cluster_first), const_cast<int32_t*>(p.hdr), p.status);
+  MLA_CUDA(cudaGetLastError());
+
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(2 * NC);
+  cfg.blockDim = dim3(mla::NUM_THREADS);
+  cfg.dynamicSmemBytes = mla::SMEM_ALLOC;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[2];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = 2;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[1].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 2;
+  if (timing) MLA_CUDA(cudaEventRecord(g_ev_before, stream));
+  MLA_CUDA(cudaLaunchKernelEx(&cfg, mla::mla_decode_kernel, p));
+  if (timing) MLA_CUDA(cudaEventRecord(g_ev_after, stream));
+
+  const int per_item = mla::MROWS / mla::COMBINE_HEADS;
+  const int64_t cgrid = static_cast<int64_t>(p.items) * per_item;
+  if (cgrid > 0x7FFFFFFF) return fail(MLA_ERR_UNSUPPORTED, "combine grid too large");
+  cudaLaunchConfig_t ccfg = {};
+  ccfg.gridDim = dim3(static_cast<unsigned>(cgrid));
+  ccfg.blockDim = dim3(32 * mla::COMBINE_HEADS);
+  ccfg.dynamicSmemBytes = 0;
+  ccfg.stream = stream;
+  ccfg.attrs = &attr[1];
+  ccfg.numAttrs = 1;
+  MLA_CUDA(cudaLaunchKernelEx(&ccfg, mla::mla_combine_kernel, p));
+  return MLA_OK;
+}
+
 }  // namespace
 
 // ---------------------------------------------------------------- fixed scratch (no-allocation entry)
@@ -359,33 +403,7 @@ mla_status_t mla_decode_paged_fp8(const void* q, const void* blocks, const float
   p.trace = g_trace;
 #endif
 
-  mla::mla_plan_kernel<<<1, mla::PLAN_THREADS, 0, stream>>>(
-      cache_lengths, p.B, p.T, p.G, max_cache_length, NC, const_cast<int32_t*>(p.item_start),
-      const_cast<int32_t*>(p.item_nvis), const_cast<int32_t*>(p.cluster_first), const_cast<int32_t*>(p.hdr), p.status);
-  MLA_CUDA(cudaGetLastError());
-
-  cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3(2 * NC);
-  cfg.blockDim = dim3(mla::NUM_THREADS);
-  cfg.dynamicSmemBytes = mla::SMEM_ALLOC;
-  cfg.stream = stream;
-  cudaLaunchAttribute attr[1];
-  attr[0].id = cudaLaunchAttributeClusterDimension;
-  attr[0].val.clusterDim.x = 2;
-  attr[0].val.clusterDim.y = 1;
-  attr[0].val.clusterDim.z = 1;
-  cfg.attrs = attr;
-  cfg.numAttrs = 1;
-  if (g_ev_before && g_ev_after) MLA_CUDA(cudaEventRecord(g_ev_before, stream));
-  MLA_CUDA(cudaLaunchKernelEx(&cfg, mla::mla_decode_kernel, p));
-  if (g_ev_before && g_ev_after) MLA_CUDA(cudaEventRecord(g_ev_after, stream));
-
-  const int per_item = mla::MROWS / mla::COMBINE_HEADS;
-  const int64_t cgrid = static_cast<int64_t>(p.items) * per_item;
-  if (cgrid > 0x7FFFFFFF) return fail(MLA_ERR_UNSUPPORTED, "combine grid too large");
-  mla::mla_combine_kernel<<<static_cast<unsigned>(cgrid), 32 * mla::COMBINE_HEADS, 0, stream>>>(p);
-  MLA_CUDA(cudaGetLastError());
-  return MLA_OK;
+  return launch_path(p, NC, cache_lengths, max_cache_length, stream, g_ev_before && g_ev_after);
 }
 
 mla_status_t mla_gather_dequant_bf16(const void* blocks, const float* scales, const uint32_t* cache_lengths,
@@ -425,6 +443,18 @@ mla_status_t mla_gather_dequant_bf16(const void* blocks, const float* scales, co
 // (2 * TRACE_TILES * TRACE_EVENTS uint64 values).
 mla_status_t mla_debug_set_trace(unsigned long long* buf) {
   g_trace = buf;
+  return MLA_OK;
+}
+
+// Trace builds only: copies the %globaltimer marks of the last decode call (plan end, first decode
+// CTA entry, last decode CTA exit, first combine CTA entry) to out8 and, if reset, re-arms them.
+mla_status_t mla_debug_marks(unsigned long long* out8, int reset) {
+  MLA_CUDA(cudaDeviceSynchronize());
+  MLA_CUDA(cudaMemcpyFromSymbol(out8, mla::g_trace_marks, 8 * sizeof(unsigned long long)));
+  if (reset) {
+    const unsigned long long init[8] = {0ull, ~0ull, 0ull, ~0ull, 0ull, 0ull, 0ull, 0ull};
+    MLA_CUDA(cudaMemcpyToSymbol(mla::g_trace_marks, init, sizeof(init)));
+  }
   return MLA_OK;
 }
 #endif
@@ -488,30 +518,7 @@ mla_status_t mla_decode_paged_fp8_noalloc(const void* q, const void* blocks, con
   if (!p.status) return fail(MLA_ERR_CUDA, "status word address unavailable");
   p.scale_log2 = softmax_scale * 1.4426950408889634f;
 
-  mla::mla_plan_kernel<<<1, mla::PLAN_THREADS, 0, stream>>>(
-      cache_lengths, p.B, p.T, p.G, max_cache_length, NC, const_cast<int32_t*>(p.item_start),
-      const_cast<int32_t*>(p.item_nvis), const_cast<int32_t*>(p.cluster_first), const_cast<int32_t*>(p.hdr), p.status);
-  MLA_CUDA(cudaGetLastError());
-
-  cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3(2 * NC);
-  cfg.blockDim = dim3(mla::NUM_THREADS);
-  cfg.dynamicSmemBytes = mla::SMEM_ALLOC;
-  cfg.stream = stream;
-  cudaLaunchAttribute attr[1];
-  attr[0].id = cudaLaunchAttributeClusterDimension;
-  attr[0].val.clusterDim.x = 2;
-  attr[0].val.clusterDim.y = 1;
-  attr[0].val.clusterDim.z = 1;
-  cfg.attrs = attr;
-  cfg.numAttrs = 1;
-  MLA_CUDA(cudaLaunchKernelEx(&cfg, mla::mla_decode_kernel, p));
-
-  const int per_item = mla::MROWS / mla::COMBINE_HEADS;
-  const int64_t cgrid = static_cast<int64_t>(p.items) * per_item;
-  mla::mla_combine_kernel<<<static_cast<unsigned>(cgrid), 32 * mla::COMBINE_HEADS, 0, stream>>>(p);
-  MLA_CUDA(cudaGetLastError());
-  return MLA_OK;
+  return launch_path(p, NC, cache_lengths, max_cache_length, stream, false);
 }
 
 mla_status_t mla_get_device_status(cudaStream_t stream) {

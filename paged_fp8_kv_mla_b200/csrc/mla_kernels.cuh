@@ -82,7 +82,8 @@ enum Bar : uint32_t {
   B_DRAIN = 16,    // CTA 0: one commit from each issuer at exit
   B_RED = 17,      // [2] softmax warps of this CTA: row-max exchange of a tile (4 warp arrivals)
   B_REDL = 19,     // softmax warps of this CTA: row-sum exchange at a unit's end (4 warp arrivals)
-  NUM_BARS = 20
+  B_EXIT = 20,     // both CTAs: the peer has finished (1 remote arrival)
+  NUM_BARS = 21
 };
 static_assert(8 * NUM_BARS <= 192, "barrier block overlaps the scalars after it");
 constexpr uint32_t S_TMEM_BASE = SBAR + 192;
@@ -195,6 +196,16 @@ __device__ __forceinline__ void raise_status(unsigned int* status, unsigned bits
 // Trace builds also record, per CTA, %globaltimer at entry, after setup and at exit, at
 // trace[2 * TRACE_TILES * TRACE_EVENTS + 4 * blockIdx.x + {0, 1, 2}].
 #ifdef MLA_TRACE
+// Trace builds: %globaltimer marks of one decode call: [0] plan end, [1] first decode CTA entry,
+// [2] last decode CTA exit, [3] first combine CTA entry, [4] last combine CTA exit.
+__device__ unsigned long long g_trace_marks[8];
+#define MLA_MARK_MIN(i) atomicMin(&g_trace_marks[i], static_cast<unsigned long long>(ptx::globaltimer()))
+#define MLA_MARK_MAX(i) atomicMax(&g_trace_marks[i], static_cast<unsigned long long>(ptx::globaltimer()))
+#else
+#define MLA_MARK_MIN(i) do {} while (0)
+#define MLA_MARK_MAX(i) do {} while (0)
+#endif
+#ifdef MLA_TRACE
 #define MLA_TRACE_CTA(slot)                                                                           \
   do {                                                                                                \
     if (p.trace && threadIdx.x == 0)                                                                  \
@@ -223,6 +234,21 @@ __device__ __forceinline__ bool wait_bar(uint32_t addr, uint32_t parity, volatil
   if (ptx::mbar_try_wait(addr, parity)) return true;
   const uint64_t t0 = ptx::globaltimer();
   while (!ptx::mbar_try_wait_sleep(addr, parity, 20000u)) {
+    if (*abort) return false;
+    if (ptx::globaltimer() - t0 > WAIT_LIMIT_NS) return wait_gave_up(abort, status, peer_abort);
+  }
+  return true;
+}
+
+// The same bound, polling instead of suspending in try_wait: the MMA issuers use it because a
+// suspended thread resumes hundreds of cycles after the phase completes, and the issuers sit on
+// the critical path of every tile.
+__device__ __forceinline__ bool poll_bar(uint32_t addr, uint32_t parity, volatile uint32_t* abort,
+                                         unsigned int* status, uint32_t peer_abort) {
+  if (ptx::mbar_test_wait(addr, parity)) return true;
+  const uint64_t t0 = ptx::globaltimer();
+  while (!ptx::mbar_test_wait(addr, parity)) {
+    __nanosleep(32);
     if (*abort) return false;
     if (ptx::globaltimer() - t0 > WAIT_LIMIT_NS) return wait_gave_up(abort, status, peer_abort);
   }
@@ -617,6 +643,8 @@ __device__ __forceinline__ void converter_role(const DecodeParams& p, int k, uin
 // decode kernel
 // =============================================================================================
 __global__ void __launch_bounds__(NUM_THREADS, 1) mla_decode_kernel(const __grid_constant__ DecodeParams p) {
+  if (threadIdx.x == 0) MLA_MARK_MIN(1);
+  ptx::griddep_launch_dependents();   // the combine kernel may start launching (it waits for this grid)
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   const uint32_t base = ptx::smem_u32(smem);
@@ -645,6 +673,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) mla_decode_kernel(const __grid
     ptx::mbar_init(BAR(B_O_FREE), 8);
     ptx::mbar_init(BAR(B_DRAIN), 2);
     ptx::mbar_init(BAR(B_REDL), 4);
+    ptx::mbar_init(BAR(B_EXIT), 1);
     *abort = 0u;
     ptx::fence_mbar_init();
   }
@@ -657,12 +686,14 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) mla_decode_kernel(const __grid
   ptx::cluster_sync();   // the peer's barriers exist before any remote arrive
   ptx::tc_fence_after();
   const uint32_t tbase = *reinterpret_cast<volatile uint32_t*>(smem + S_TMEM_BASE);
-  MLA_TRACE_CTA(1);
+  ptx::griddep_wait();   // the split plan (previous kernel of the stream) is complete and visible
 
 // Whole-warp roles bail out together so that the warp-collective instructions after a wait never
 // run on a partial warp.
 #define MLA_WAIT_WARP(b_, parity)                                                              \
   if (!__all_sync(0xffffffffu, wait_bar((b_), (parity), abort, p.status, peer_abort))) goto role_done;
+#define MLA_POLL_WARP(b_, parity)                                                              \
+  if (!__all_sync(0xffffffffu, poll_bar((b_), (parity), abort, p.status, peer_abort))) goto role_done;
 
   if (warp < CONV_WARPS) {
     // ------------------------------------------------------------------ converter
@@ -769,6 +800,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) mla_decode_kernel(const __grid
       // epilogue: O / l for this lane's 256 V dims of head row r
       {
         const uint32_t gl = g - 1;
+        if (gl > 0) MLA_WAIT_WARP(BAR(B_PV_DONE + ((gl - 1) & 1)), ((gl - 1) >> 1) & 1);
         MLA_WAIT_WARP(BAR(B_PV_DONE + (gl & 1)), (gl >> 1) & 1);
         ptx::tc_fence_after();
         red_l[t] = l;
@@ -780,34 +812,54 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) mla_decode_kernel(const __grid
         const int head = u.g * MROWS + HPC * static_cast<int>(c) + r;
         const bool row_ok = head < p.H;
         const float lse_v = (m_ref + ptx::lg2_approx(l_row)) * 0.69314718055994530942f;
+        // O / l goes out through a per-warp 4 KB staging block in the (now idle) P buffers: each
+        // thread writes its row's 32 values of a chunk, then the warp stores whole 64- or 128-byte
+        // row segments (16-byte positions swizzled by row, so both passes are conflict-free).
+        const uint32_t stage = base + SP0 + static_cast<uint32_t>(quad) * 4096u;
+        const int row0 = HPC * static_cast<int>(c) + 32 * (quad & 1);   // CTA row of this warp's lane 0
 #pragma unroll 1
         for (int ch = 0; ch < 8; ++ch) {
           uint32_t rr[32];
           ptx::tmem_ld32(lane_base + T_O + 32 * ch, rr);
           ptx::tmem_wait_ld();
-          if (!row_ok) continue;
           const int dv = (ch < 4 ? 0 : 256) + 128 * hh + 32 * (ch & 3);
           if (u.slot < 0) {
-            uint16_t* dst = p.out + ((static_cast<size_t>(u.b) * p.T + u.i) * p.H + head) * V_DIM + dv;
+            // bf16: 32 rows x 64 B; 16-byte chunk j of row x at x * 64 + 16 * (j ^ ((x >> 1) & 3))
 #pragma unroll
             for (int v = 0; v < 4; ++v) {
-              uint4 w;
-              w.x = ptx::pack_bf16x2(__uint_as_float(rr[8 * v + 0]) * inv_l, __uint_as_float(rr[8 * v + 1]) * inv_l);
-              w.y = ptx::pack_bf16x2(__uint_as_float(rr[8 * v + 2]) * inv_l, __uint_as_float(rr[8 * v + 3]) * inv_l);
-              w.z = ptx::pack_bf16x2(__uint_as_float(rr[8 * v + 4]) * inv_l, __uint_as_float(rr[8 * v + 5]) * inv_l);
-              w.w = ptx::pack_bf16x2(__uint_as_float(rr[8 * v + 6]) * inv_l, __uint_as_float(rr[8 * v + 7]) * inv_l);
-              reinterpret_cast<uint4*>(dst)[v] = w;
+              const uint32_t w0 = ptx::pack_bf16x2(__uint_as_float(rr[8 * v + 0]) * inv_l, __uint_as_float(rr[8 * v + 1]) * inv_l);
+              const uint32_t w1 = ptx::pack_bf16x2(__uint_as_float(rr[8 * v + 2]) * inv_l, __uint_as_float(rr[8 * v + 3]) * inv_l);
+              const uint32_t w2 = ptx::pack_bf16x2(__uint_as_float(rr[8 * v + 4]) * inv_l, __uint_as_float(rr[8 * v + 5]) * inv_l);
+              const uint32_t w3 = ptx::pack_bf16x2(__uint_as_float(rr[8 * v + 6]) * inv_l, __uint_as_float(rr[8 * v + 7]) * inv_l);
+              ptx::st_shared_v4(stage + lane * 64 + 16 * (v ^ ((lane >> 1) & 3)), w0, w1, w2, w3);
+            }
+            __syncwarp();
+#pragma unroll
+            for (int it = 0; it < 4; ++it) {
+              const int x = it * 8 + (lane >> 2), j = lane & 3;
+              const uint4 w = ptx::ld_shared_v4(stage + x * 64 + 16 * (j ^ ((x >> 1) & 3)));
+              const int hd = u.g * MROWS + row0 + x;
+              if (hd < p.H)
+                *reinterpret_cast<uint4*>(p.out + ((static_cast<size_t>(u.b) * p.T + u.i) * p.H + hd) * V_DIM + dv + 8 * j) = w;
             }
           } else {
-            float* dst = p.part_o + (static_cast<size_t>(u.slot) * MROWS + HPC * c + r) * V_DIM + dv;
+            // fp32: 32 rows x 128 B; 16-byte chunk j of row x at x * 128 + 16 * (j ^ (x & 7))
 #pragma unroll
-            for (int v = 0; v < 8; ++v) {
-              const float4 w = make_float4(__uint_as_float(rr[4 * v]) * inv_l, __uint_as_float(rr[4 * v + 1]) * inv_l,
-                                           __uint_as_float(rr[4 * v + 2]) * inv_l,
-                                           __uint_as_float(rr[4 * v + 3]) * inv_l);
-              reinterpret_cast<float4*>(dst)[v] = w;
+            for (int v = 0; v < 8; ++v)
+              ptx::st_shared_v4(stage + lane * 128 + 16 * (v ^ (lane & 7)),
+                                __float_as_uint(__uint_as_float(rr[4 * v + 0]) * inv_l),
+                                __float_as_uint(__uint_as_float(rr[4 * v + 1]) * inv_l),
+                                __float_as_uint(__uint_as_float(rr[4 * v + 2]) * inv_l),
+                                __float_as_uint(__uint_as_float(rr[4 * v + 3]) * inv_l));
+            __syncwarp();
+#pragma unroll
+            for (int it = 0; it < 8; ++it) {
+              const int x = it * 4 + (lane >> 3), j = lane & 7;
+              const uint4 w = ptx::ld_shared_v4(stage + x * 128 + 16 * (j ^ (x & 7)));
+              *reinterpret_cast<uint4*>(p.part_o + (static_cast<size_t>(u.slot) * MROWS + row0 + x) * V_DIM + dv + 4 * j) = w;
             }
           }
+          __syncwarp();
         }
         if (hh == 0 && row_ok) {
           if (u.slot < 0) {
@@ -846,6 +898,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) mla_decode_kernel(const __grid
         ptx::mbar_arrive_cluster(q_full);
         ++uu;
       }
+      // drain: the last unit's Q_FREE commit lands in this CTA before it exits
+      if (uu > 0) wait_bar(BAR(B_Q_FREE), (uu & 1) ^ 1, abort, p.status, peer_abort);
     }
   } else if (warp == QK_WARP) {
     // ------------------------------------------------------------------ Q.K^T issuer (CTA 0)
@@ -859,11 +913,11 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) mla_decode_kernel(const __grid
       while (qc.valid) {
         const uint32_t kb = g & 1;
         if (qc.first) {
-          MLA_WAIT_WARP(BAR(B_Q_FULL), uq & 1);
+          MLA_POLL_WARP(BAR(B_Q_FULL), uq & 1);
           ++uq;
         }
-        MLA_WAIT_WARP(BAR(B_K_FULL + kb), (g >> 1) & 1);
-        MLA_WAIT_WARP(BAR(B_S_FREE + kb), ((g >> 1) & 1) ^ 1);
+        MLA_POLL_WARP(BAR(B_K_FULL + kb), (g >> 1) & 1);
+        MLA_POLL_WARP(BAR(B_S_FREE + kb), ((g >> 1) & 1) ^ 1);
         ptx::tc_fence_after();
         if (ptx::elect_one()) {
           MLA_TRACE_EV(g, 20);
@@ -886,6 +940,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) mla_decode_kernel(const __grid
         ++g;
         qc.advance();
       }
+      // drain: the S_FREE arrivals of the last two tiles (nothing else waits for them)
+      for (uint32_t gd = (g >= 2 ? g - 2 : 0); gd < g; ++gd) MLA_POLL_WARP(BAR(B_S_FREE + (gd & 1)), (gd >> 1) & 1);
     }
   } else if (warp == PV_WARP) {
     // ------------------------------------------------------------------ P.V issuer (CTA 0)
@@ -897,10 +953,10 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) mla_decode_kernel(const __grid
       while (pc.valid) {
         const uint32_t hb = g & 1;
         const bool first = pc.first;
-        MLA_WAIT_WARP(BAR(B_V_FULL + hb), (g >> 1) & 1);
-        MLA_WAIT_WARP(BAR(B_P_FULL + hb), (g >> 1) & 1);
+        MLA_POLL_WARP(BAR(B_V_FULL + hb), (g >> 1) & 1);
+        MLA_POLL_WARP(BAR(B_P_FULL + hb), (g >> 1) & 1);
         if (first) {
-          MLA_WAIT_WARP(BAR(B_O_FREE), (up & 1) ^ 1);
+          MLA_POLL_WARP(BAR(B_O_FREE), (up & 1) ^ 1);
           ++up;
         }
         ptx::tc_fence_after();
@@ -922,9 +978,12 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) mla_decode_kernel(const __grid
         ++g;
         pc.advance();
       }
+      // drain: the last unit's O_FREE arrivals (both CTAs' epilogues)
+      if (up > 0) MLA_POLL_WARP(BAR(B_O_FREE), (up - 1) & 1);
     }
   }
 role_done:
+#undef MLA_POLL_WARP
 #undef MLA_WAIT_WARP
   // every pair MMA issued by CTA 0 has finished before TMEM is released
   if (c == 0 && (warp == QK_WARP || warp == PV_WARP) && lane == 0) {
@@ -932,14 +991,31 @@ role_done:
     const uint64_t t0 = ptx::globaltimer();
     while (!ptx::mbar_try_wait(BAR(B_DRAIN), 0) && ptx::globaltimer() - t0 < WAIT_LIMIT_NS) {}
   }
-#undef BAR
   ptx::tc_fence_before();
   __syncthreads();
   MLA_TRACE_CTA(2);
-  ptx::cluster_sync();   // no remote arrive or pair MMA targets a CTA that has exited
+  // Exit handshake.  Every cross-CTA arrival and pair-MMA commit has been waited for above, so no
+  // remote access can reach a CTA that has exited; the two CTAs still tell each other that they are
+  // done (one remote arrive each) before the pair's TMEM is released.  The wait polls: a thread
+  // suspended in try_wait (or in a cluster barrier) measured ~7 us to resume after the peer's
+  // remote arrival on B200, even with both CTAs arriving together.
+  if (threadIdx.x == 0) {
+    ptx::mbar_arrive_remote_relaxed(ptx::mapa(BAR(B_EXIT), peer));
+#ifdef MLA_TRACE
+    if (p.trace) p.trace[2 * TRACE_TILES * TRACE_EVENTS + 4 * blockIdx.x + 1] = ptx::globaltimer();
+#endif
+    const uint64_t t0 = ptx::globaltimer();
+    while (!ptx::mbar_test_wait(BAR(B_EXIT), 0) && ptx::globaltimer() - t0 < WAIT_LIMIT_NS) __nanosleep(32);
+  }
+  __syncthreads();
+#undef BAR
   if (warp == QK_WARP) {
     ptx::tc_fence_after();
     ptx::tmem_dealloc_pair(tbase, TMEM_COLS);
+    if (lane == 0) MLA_MARK_MAX(2);
+#ifdef MLA_TRACE
+    if (lane == 0 && p.trace) p.trace[2 * TRACE_TILES * TRACE_EVENTS + 4 * blockIdx.x + 3] = ptx::globaltimer();
+#endif
   }
 }
 // =============================================================================================
@@ -951,6 +1027,7 @@ __global__ void __launch_bounds__(PLAN_THREADS)
 mla_plan_kernel(const uint32_t* __restrict__ cache_lengths, int B, int T, int G, uint32_t max_cache_length,
                 int NC, int32_t* item_start, int32_t* item_nvis, int32_t* cluster_first, int32_t* hdr,
                 unsigned int* status) {
+  ptx::griddep_launch_dependents();   // the decode kernel may launch and run its prologue meanwhile
   __shared__ int warp_sums[32];
   __shared__ int carry;
   const int items = B * T * G;
@@ -1017,6 +1094,8 @@ mla_plan_kernel(const uint32_t* __restrict__ cache_lengths, int B, int T, int G,
     }
     cluster_first[kk] = first;
   }
+  __syncthreads();
+  if (t == 0) MLA_MARK_MAX(0);
 }
 
 // =============================================================================================
@@ -1026,6 +1105,8 @@ constexpr int COMBINE_HEADS = 8;
 
 __global__ void __launch_bounds__(32 * COMBINE_HEADS)
 mla_combine_kernel(const __grid_constant__ DecodeParams p) {
+  ptx::griddep_wait();   // the decode kernel's partials are complete and visible
+  if (threadIdx.x == 0) MLA_MARK_MIN(3);
   const int per_item = MROWS / COMBINE_HEADS;
   const int it = blockIdx.x / per_item;
   const int hc = blockIdx.x % per_item;

@@ -51,6 +51,18 @@ __device__ __forceinline__ void cluster_sync() {
   asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::: "memory");
 }
 
+// Cluster barrier whose arrive orders nothing: for the exit of a CTA that has no memory access
+// left for the peer to observe (a release arrive would first wait for every outstanding global
+// store of the thread).
+__device__ __forceinline__ void cluster_sync_relaxed() {
+  asm volatile("barrier.cluster.arrive.relaxed.aligned;\n\tbarrier.cluster.wait.aligned;" ::: "memory");
+}
+
+// Programmatic dependent launch: let the next kernel of the stream start launching (its own
+// griddepcontrol.wait still waits for this grid to finish), and wait for the previous kernel.
+__device__ __forceinline__ void griddep_launch_dependents() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
+__device__ __forceinline__ void griddep_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+
 // Address of the same shared-memory location in CTA `rank` of the cluster.
 __device__ __forceinline__ uint32_t mapa(uint32_t addr, uint32_t rank) {
   uint32_t r;
@@ -79,6 +91,12 @@ __device__ __forceinline__ void mbar_arrive_expect_tx(uint32_t addr, uint32_t tx
 // ordering this thread's earlier cluster-shared writes before the arrival.
 __device__ __forceinline__ void mbar_arrive_remote(uint32_t cluster_addr) {
   asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" :: "r"(cluster_addr) : "memory");
+}
+
+// Arrive on a barrier of another CTA without ordering any earlier memory access (the caller has
+// nothing left for the peer to observe).
+__device__ __forceinline__ void mbar_arrive_remote_relaxed(uint32_t cluster_addr) {
+  asm volatile("mbarrier.arrive.relaxed.cluster.shared::cluster.b64 _, [%0];" :: "r"(cluster_addr) : "memory");
 }
 
 // Arrive on a barrier of any CTA of the cluster with the default (CTA-scope release) semantics.
@@ -196,10 +214,11 @@ __device__ __forceinline__ void prefetch_l2(const void* src, uint32_t bytes) {
   asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" :: "l"(reinterpret_cast<uint64_t>(src)), "r"(bytes) : "memory");
 }
 
-// 16-byte global load that bypasses L1 allocation (streamed KV bytes).
+// 16-byte global load of streamed KV bytes (plain cached load: measured faster here than the
+// non-coherent no-allocate form).
 __device__ __forceinline__ uint4 ldg_stream_v4(const void* p) {
   uint4 v;
-  asm volatile("ld.global.nc.L1::no_allocate.v4.u32 {%0, %1, %2, %3}, [%4];"
+  asm volatile("ld.global.v4.u32 {%0, %1, %2, %3}, [%4];"
                : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w) : "l"(p));
   return v;
 }
