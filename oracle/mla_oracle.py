@@ -27,6 +27,15 @@ What it computes, step by step, in the order the pages lay out the data:
    new tokens are already in the cache); query i of request b sees keys
    t <= cache_lengths[b] + i (causal among the new tokens).
 
+4. The KV-store step that produces this path's input (the data-generation
+   recipe of the pages' config 0: per-token scale f32(amax) / 448, e4m3 codes
+   with round-to-nearest and saturation).  For new token i of request b, at
+   position t = cache_lengths[b] + i (reading R1), with x the 576 bf16 values:
+   scale = f32(max_d |x_d|) / 448 rounded to fp32 (1.0 for an all-zero row),
+   code_d = e4m3_rn_sat(f32_rn(x_d / scale)), written to blocks[blk, 0,
+   layer_idx, t % page_size, 0, :] and scale to the same slot of scales, with
+   blk (and the scale block) from the page tables as in step 1.
+
 Everything after the e4m3 decode is float64 (the dequantised bf16 values are
 exact in float64).  Points the pages leave open and the reading taken here:
 cache_lengths count only tokens cached before this step (R1); query i sees
@@ -111,6 +120,73 @@ def dequant_rows(codes, scale) -> np.ndarray:
     with np.errstate(over="ignore", invalid="ignore"):
         p32 = prod.astype(np.float32)
     return bf16_round_f32(p32)
+
+
+def e4m3_encode_rn_sat(y) -> np.ndarray:
+    """e4m3 byte nearest to each finite float32 value y, ties to even mantissa, saturated to +-448.
+
+    Written from the format: |y| is clamped to 448, then for |y| >= 2^-6 (normal range) the
+    exponent is e = floor(log2 |y|) and the mantissa steps are 2^(e-3); below 2^-6 the steps are
+    the subnormal 2^-9.  A mantissa that rounds up to 8 carries into the exponent.  The sign bit is
+    kept (so -0.0 -> 0x80).  Scaling by powers of two is exact in float64, so the rounding here is
+    the single round-to-nearest-even of the format.
+    """
+    y = np.asarray(y, dtype=np.float32).astype(np.float64)
+    sign = (np.signbit(y)).astype(np.int64)
+    a = np.minimum(np.abs(y), 448.0)
+    code = np.zeros(a.shape, dtype=np.int64)
+    normal = a >= 2.0 ** -6
+    # subnormal range: value = m * 2^-9, m in 0..8 (8 carries into the smallest normal)
+    m_sub = np.rint(a * 2.0 ** 9).astype(np.int64)            # rint: round half to even
+    code = np.where(~normal, m_sub, code)                     # m_sub == 8 -> 0x08 = 2^-6, correct
+    # normal range
+    with np.errstate(divide="ignore"):
+        e = np.floor(np.log2(np.where(normal, a, 1.0))).astype(np.int64)
+    # guard against log2 rounding at exact powers of two
+    e = np.where(np.ldexp(1.0, e) > a, e - 1, e)
+    e = np.where(np.ldexp(1.0, e + 1) <= a, e + 1, e)
+    m = np.rint((a / np.ldexp(1.0, e) - 1.0) * 8.0).astype(np.int64)
+    carry = m == 8
+    e = np.where(carry, e + 1, e)
+    m = np.where(carry, 0, m)
+    code_n = ((e + 7) << 3) | m
+    code = np.where(normal, code_n, code)
+    return ((sign << 7) | code).astype(np.uint8)
+
+
+def quantize_token(x_bf16_bits):
+    """(codes [576] uint8, scale float32) of one token's latent given as bf16 bit patterns."""
+    x = bf16_bits_to_f64(x_bf16_bits).astype(np.float32)       # exact
+    amax = np.float32(np.max(np.abs(x))) if x.size else np.float32(0)
+    scale = np.float32(amax / np.float32(448.0)) if amax > 0 else np.float32(1.0)
+    y = (x / scale).astype(np.float32)                         # IEEE fp32 division, RN
+    return e4m3_encode_rn_sat(y), scale
+
+
+def kv_store(latent_bits, cache_lengths, lookup_table, scales_lookup_table, layer_idx, blocks, scales):
+    """Write the new tokens' codes and scales into copies of blocks / scales; returns the copies.
+
+    latent_bits: bf16 bit patterns [B, T, 576]; token i of request b goes to position
+    cache_lengths[b] + i.  Only kv_dim 0 and scale column 0 are written.
+    """
+    lat = np.asarray(latent_bits, dtype=np.uint16)
+    B, T, _ = lat.shape
+    blocks = np.array(blocks, copy=True)
+    scales = np.array(scales, copy=True)
+    L = np.asarray(cache_lengths, dtype=np.int64)
+    lut = np.asarray(lookup_table, dtype=np.uint32)
+    slut = None if scales_lookup_table is None else np.asarray(scales_lookup_table, dtype=np.uint32)
+    P = blocks.shape[3]
+    for b in range(B):
+        for i in range(T):
+            t = int(L[b]) + i
+            page, slot = t // P, t % P
+            blk = int(lut[b, page])
+            sblk = int(slut[b, page]) if slut is not None else blk
+            codes, sc = quantize_token(lat[b, i])
+            blocks[blk, 0, layer_idx, slot, 0, :] = codes
+            scales[sblk, 0, layer_idx, slot, 0, 0] = sc
+    return blocks, scales
 
 
 # ----------------------------------------------------------------------------
