@@ -40,6 +40,8 @@ def parse():
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--config", type=int, default=1)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--op", choices=["decode", "kv_store"], default="decode",
+                    help="decode (the default contract line) or the KV-store step that fills the cache")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=12.0, help="budget of the oracle CPU baseline")
@@ -59,7 +61,7 @@ def load_peaks():
 
 def kernel_source_sha():
     h = hashlib.sha256()
-    for f in ("ptx.cuh", "mla_kernels.cuh", "mla_api.cu"):
+    for f in ("ptx.cuh", "mla_kernels.cuh", "mla_api.cu", "mla_kv_store.cuh"):
         with open(os.path.join(ROOT, "paged_fp8_kv_mla_b200", "csrc", f), "rb") as fh:
             h.update(fh.read())
     return h.hexdigest()[:16]
@@ -200,10 +202,111 @@ def run_reference(args):
     return 0
 
 
+STORE_WORKLOAD = dict(batch=64, new_tokens=1024, page_size=64, max_cached=4096, seed=3001)
+
+
+def run_kv_store(args):
+    """KV-store step (quantise + scatter) on a prefill-sized chunk: 64 requests x 1024 new tokens.
+
+    HBM-bound: per token 1152 B of bf16 read, 576 B of e4m3 and a 4 B scale written.  One GPU.
+    """
+    import paged_fp8_kv_mla_b200 as M
+    from paged_fp8_kv_mla_b200 import workloads as W
+    torch.cuda.set_device(0)
+    M.load()
+    w = STORE_WORKLOAD
+    si = W.make_store_inputs(w["batch"], w["new_tokens"], w["page_size"], w["max_cached"], w["seed"], device="cuda")
+    nbytes = si.algorithmic_bytes()
+    tokens = w["batch"] * w["new_tokens"]
+    l2 = torch.cuda.get_device_properties(0).L2_cache_size
+    flush = torch.empty(max(2 * l2, 256 << 20), dtype=torch.uint8, device="cuda")
+    stream = torch.cuda.current_stream()
+
+    def step():
+        M.kv_store(si.latent, si.cache_lengths, si.lookup_table, si.scales_lookup_table, si.layer_idx,
+                   si.blocks, si.scales, stream=stream)
+
+    for _ in range(max(3, args.warmup)):
+        flush.zero_()
+        step()
+    torch.cuda.synchronize()
+    if M.device_status() != 0:
+        raise RuntimeError("device status error during warm-up")
+    K = args.steps
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(K)]
+    clocks = ClockSampler(0)
+    clocks.start()
+    torch.cuda.synchronize()
+    for a, b in ev:
+        flush.zero_()
+        a.record(stream)
+        step()
+        b.record(stream)
+    torch.cuda.synchronize()
+    clk = clocks.stop()
+    ms = sum(a.elapsed_time(b) for a, b in ev) / K
+    if M.device_status() != 0:
+        raise RuntimeError("device status error in the timed region")
+
+    e2e = None
+    if not args.no_e2e:
+        hl = si.latent.cpu().pin_memory()
+        dl = torch.empty_like(si.latent)
+        Ke = min(K, 50)
+        eev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(Ke)]
+        for a, b in eev:
+            flush.zero_()
+            a.record(stream)
+            dl.copy_(hl, non_blocking=True)
+            M.kv_store(dl, si.cache_lengths, si.lookup_table, si.scales_lookup_table, si.layer_idx,
+                       si.blocks, si.scales, stream=stream)
+            b.record(stream)
+        torch.cuda.synchronize()
+        e_ms = sum(a.elapsed_time(b) for a, b in eev) / Ke
+        e2e = {"value": nbytes / (e_ms * 1e-3) / 1e9, "unit": "GB/s", "h2d_bytes_per_step": hl.numel() * 2,
+               "d2h_bytes_per_step": 0, "ms_per_step": e_ms}
+
+    cpu = None
+    if not args.no_cpu_baseline:
+        import numpy as np
+        from oracle import mla_oracle as O
+        lat = si.latent[:1].cpu().view(torch.int16).numpy().view(np.uint16)
+        t0 = time.perf_counter()
+        n = 0
+        while time.perf_counter() - t0 < min(args.cpu_seconds, 10.0) and n < lat.shape[1]:
+            O.quantize_token(lat[0, n])
+            n += 1
+        dt = time.perf_counter() - t0
+        cpu = {"value": n * (2 * 576 + 576 + 4) / dt / 1e9, "unit": "GB/s", "cores": 1, "kind": "oracle",
+               "sample": f"{n} tokens of request 0 quantised by the float64 oracle (scatter not timed)"}
+    peaks = load_peaks()
+    gbs = nbytes / (ms * 1e-3) / 1e9
+    line = {
+        "metric": "KV-store GB/s (bf16 latent read + e4m3 row and fp32 scale written)", "value": gbs, "unit": "GB/s",
+        "n_gpus": 1, "steps": K, "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "bf16 in, e4m3 + fp32 out", "data": "synthetic",
+        "tokens_per_s": tokens / (ms * 1e-3),
+        "config": {"workload": "kv_store_prefill_b64_t1024_p64", "batch": w["batch"], "new_tokens": w["new_tokens"],
+                   "page_size": w["page_size"], "bytes_per_step": nbytes,
+                   "l2": "flushed before every timed step (write of %d MB)" % (flush.numel() >> 20)},
+        "roofline": {"kernel": "mla_kv_store_kernel", "bound": "hbm", "achieved": gbs, "peak": peaks["hbm_gbs"],
+                     "unit": "GB/s", "frac": gbs / peaks["hbm_gbs"], "peak_source": peaks["source"] + " copy",
+                     "traffic": None, "kernel_ms": ms},
+        "gpu_launches": K,
+        "clocks": clk,
+        "e2e": e2e,
+        "cpu_baseline": cpu,
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
 def main():
     args = parse()
     if args.impl == "reference":
         return run_reference(args)
+    if args.op == "kv_store":
+        return run_kv_store(args)
 
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))

@@ -151,6 +151,38 @@ mla_status_t mla_gather_dequant_bf16(
     const mla_paged_shape_t* shape, void* out_k, uint32_t max_keys, cudaStream_t stream);
 
 /*
+ * mla_kv_store_fp8 -- the KV-store step that produces the cache the decode reads: quantise the
+ * step's new tokens' latent to e4m3 with one fp32 scale per token and scatter each row into its
+ * page.  The quantiser is the pages' data recipe (per-token scale amax / 448, e4m3 round to
+ * nearest with saturation); the placement is the page-table layout of
+ * generic_get_paged_cache_with_scales.
+ *
+ * For new token i of request b, at position t = cache_lengths[b] + i (the step's tokens follow
+ * the cached ones), with x its 576 bf16 values:
+ *   scale = f32(max |x|) / 448 rounded to fp32 (1.0 when the row is all zero),
+ *   code_d = e4m3 of f32(x_d / scale), round to nearest even, saturated to +-448,
+ * written to blocks[lookup_table[b][t / P], 0, layer_idx, t % P, 0, :] and the scale to the same
+ * slot of scales in block scales_lookup_table[b][t / P] when that table is given, else in the value
+ * block.  Non-finite inputs are not supported.
+ *
+ *   latent          bf16 [batch, num_new_tokens, 576], contiguous, 16-byte aligned, device memory.
+ *   cache_lengths   uint32 [batch] device; positions must satisfy t / P < max_pages.
+ *   lookup_table, scales_lookup_table   as for mla_decode_paged_fp8; the pages must already be
+ *                   assigned (this call writes into them, it does not allocate pages).
+ *   blocks, scales  the cache, written in place (only the rows of the new tokens, kv_dim 0).
+ *   shape           as for mla_decode_paged_fp8 (head_dim 576, num_kv_heads 1,
+ *                   head_dim_granularity 1; num_q_heads, v_dim and max_prompt_length are not used).
+ * Asynchronous on `stream`.  A page id past the pool or a position past max_pages is skipped on
+ * the device and reported by mla_get_device_status as MLA_ERR_DEVICE_BOUNDS.  Two new tokens that
+ * map to the same slot race (the caller's tables must not do that).  batch = 0 or
+ * num_new_tokens = 0 is a no-op.
+ */
+mla_status_t mla_kv_store_fp8(
+    const void* latent, const uint32_t* cache_lengths, const uint32_t* lookup_table,
+    const uint32_t* scales_lookup_table, uint32_t num_new_tokens, uint32_t layer_idx,
+    const mla_paged_shape_t* shape, void* blocks, float* scales, cudaStream_t stream);
+
+/*
  * mla_set_num_clusters -- test and tuning hook: fix the number of 2-CTA clusters
  * the decode splits the keys over (0 restores the default, one per resident
  * cluster slot of the device).  Process-wide.  Smaller values make fewer, longer

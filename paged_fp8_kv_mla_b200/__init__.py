@@ -5,6 +5,6 @@ include/mla_paged_fp8.h; this package holds its Python binding (`_lib`), the
 build step (`build`) and the seeded workload generators (`workloads`).
 """
 from ._lib import (  # noqa: F401
-    MlaError, decode, decode_inputs, gather_dequant, set_num_clusters, get_num_clusters, device_status,
+    MlaError, decode, decode_inputs, gather_dequant, kv_store, set_num_clusters, get_num_clusters, device_status,
     release_workspace, version, set_timing_events, load, LIB_PATH, EXPORTED,
 )

@@ -22,7 +22,8 @@ STATUS_NAMES = {0: "MLA_OK", 1: "MLA_ERR_INVALID_ARG", 2: "MLA_ERR_UNSUPPORTED",
 # every symbol include/mla_paged_fp8.h declares
 EXPORTED = ["mla_decode_paged_fp8", "mla_gather_dequant_bf16", "mla_set_num_clusters",
             "mla_get_num_clusters", "mla_last_error_string", "mla_get_device_status",
-            "mla_release_workspace", "mla_version", "mla_set_timing_events", "mla_decode_paged_fp8_noalloc"]
+            "mla_release_workspace", "mla_version", "mla_set_timing_events", "mla_decode_paged_fp8_noalloc",
+            "mla_kv_store_fp8"]
 
 
 class MlaError(RuntimeError):
@@ -58,6 +59,8 @@ def load(path: str = LIB_PATH) -> ctypes.CDLL:
     lib.mla_gather_dequant_bf16.argtypes = [vp, vp, vp, vp, vp, u32, u32, u32,
                                             ctypes.POINTER(PagedShape), vp, u32, vp]
     lib.mla_gather_dequant_bf16.restype = ctypes.c_int
+    lib.mla_kv_store_fp8.argtypes = [vp, vp, vp, vp, u32, u32, ctypes.POINTER(PagedShape), vp, vp, vp]
+    lib.mla_kv_store_fp8.restype = ctypes.c_int
     lib.mla_set_num_clusters.argtypes = [i32]
     lib.mla_set_num_clusters.restype = ctypes.c_int
     lib.mla_get_num_clusters.argtypes = []
@@ -128,6 +131,20 @@ def decode(q, blocks, scales, cache_lengths, lookup_table, scales_lookup_table, 
                                   _stream(stream))
     _check(st)
     return out, lse
+
+
+def kv_store(latent, cache_lengths, lookup_table, scales_lookup_table, layer_idx: int, blocks, scales,
+             stream=None):
+    """mla_kv_store_fp8 on torch tensors: quantise latent bf16 [B, T, 576] and write it in place into
+    blocks / scales at positions cache_lengths[b] + i (page tables as for decode)."""
+    lib = load()
+    B, T, D = latent.shape
+    _contig(latent, blocks, scales, cache_lengths, lookup_table, scales_lookup_table)
+    shp = paged_shape(B, 0, blocks, scales, lookup_table)
+    st = lib.mla_kv_store_fp8(_ptr(latent), _ptr(cache_lengths), _ptr(lookup_table), _ptr(scales_lookup_table),
+                              int(T), int(layer_idx), ctypes.byref(shp), _ptr(blocks), _ptr(scales), _stream(stream))
+    _check(st)
+    return blocks, scales
 
 
 def decode_noalloc(q, blocks, scales, cache_lengths, lookup_table, scales_lookup_table, max_prompt_length: int,

@@ -17,8 +17,11 @@ import sys
 PKG = os.path.dirname(os.path.abspath(__file__))
 ROOT = os.path.dirname(PKG)
 SRC = [os.path.join(PKG, "csrc", "mla_api.cu")]
-DEPS = [os.path.join(PKG, "csrc", f) for f in ("mla_kernels.cuh", "ptx.cuh", "mla_api.cu")] + \
-       [os.path.join(ROOT, "include", "mla_paged_fp8.h")]
+def _deps():
+    """Every source the library is built from (all of csrc/ and the public header)."""
+    d = os.path.join(PKG, "csrc")
+    return sorted(os.path.join(d, f) for f in os.listdir(d) if f.endswith((".cu", ".cuh"))) + \
+        [os.path.join(ROOT, "include", "mla_paged_fp8.h")]
 LIB = os.path.join(PKG, "libmla_paged_fp8.so")
 
 
@@ -33,7 +36,7 @@ def needs_build(out: str = LIB) -> bool:
     if not os.path.exists(out):
         return True
     t = os.path.getmtime(out)
-    return any(os.path.getmtime(d) > t for d in DEPS + [__file__])
+    return any(os.path.getmtime(d) > t for d in _deps() + [__file__])
 
 
 def build(debug: bool = False, verbose_ptxas: bool = False, force: bool = False, out: str = LIB) -> str:

@@ -11,6 +11,7 @@
 #include <vector>
 
 #include "mla_kernels.cuh"
+#include "mla_kv_store.cuh"
 #include "mla_paged_fp8.h"
 
 namespace {
@@ -434,6 +435,55 @@ mla_status_t mla_gather_dequant_bf16(const void* blocks, const float* scales, co
   if (gx > 0x7FFFFFFF) return fail(MLA_ERR_UNSUPPORTED, "grid too large");
   mla::mla_dequant_kernel<<<dim3(static_cast<unsigned>(gx), 2), mla::DQ_THREADS, mla::DQ_SMEM_ALLOC, stream>>>(
       p, cache_lengths, static_cast<int>(max_keys), tiles, static_cast<uint16_t*>(out_k));
+  MLA_CUDA(cudaGetLastError());
+  return MLA_OK;
+}
+
+mla_status_t mla_kv_store_fp8(const void* latent, const uint32_t* cache_lengths, const uint32_t* lookup_table,
+                              const uint32_t* scales_lookup_table, uint32_t num_new_tokens, uint32_t layer_idx,
+                              const mla_paged_shape_t* s, void* blocks, float* scales, cudaStream_t stream) {
+  if (!s) return fail(MLA_ERR_INVALID_ARG, "shape is NULL");
+  if (!latent || !cache_lengths || !lookup_table || !blocks || !scales)
+    return fail(MLA_ERR_INVALID_ARG, "latent, cache_lengths, lookup_table, blocks and scales must be non-NULL");
+  if (s->batch < 0 || s->num_blocks < 1 || s->kv_dim < 1 || s->num_layers < 1 || s->page_size < 1 ||
+      s->num_kv_heads < 1 || s->num_scale_blocks < 1 || s->head_dim_granularity < 1 || s->max_pages < 1)
+    return fail(MLA_ERR_INVALID_ARG, "non-positive dimension in shape");
+  if (s->head_dim != mla::HEAD_DIM) return fail(MLA_ERR_UNSUPPORTED, "head_dim must be 576 (got %d)", s->head_dim);
+  if (s->num_kv_heads != 1) return fail(MLA_ERR_UNSUPPORTED, "num_kv_heads must be 1 (MLA latent cache)");
+  if (s->head_dim_granularity != 1)
+    return fail(MLA_ERR_UNSUPPORTED, "only one scale per token (head_dim_granularity 1) is implemented");
+  if (layer_idx >= static_cast<uint32_t>(s->num_layers))
+    return fail(MLA_ERR_INVALID_ARG, "layer_idx %u >= num_layers %d", layer_idx, s->num_layers);
+  if (!aligned16(latent) || !aligned16(blocks) || !aligned16(scales))
+    return fail(MLA_ERR_INVALID_ARG, "latent, blocks and scales must be 16-byte aligned");
+  const uint64_t r = static_cast<uint64_t>(s->num_blocks) * s->kv_dim * s->num_layers * s->page_size;
+  const uint64_t sr = static_cast<uint64_t>(s->num_scale_blocks) * s->kv_dim * s->num_layers * s->page_size;
+  if (r >= (1ull << 40) || sr >= (1ull << 40)) return fail(MLA_ERR_UNSUPPORTED, "block pool too large");
+  const uint64_t tokens = static_cast<uint64_t>(s->batch) * num_new_tokens;
+  if (tokens == 0) return MLA_OK;
+  if (tokens >= (1ull << 31)) return fail(MLA_ERR_UNSUPPORTED, "too many new tokens (%llu)", static_cast<unsigned long long>(tokens));
+  mla::KvStoreParams p{};
+  p.latent = static_cast<const uint16_t*>(latent);
+  p.cache_lengths = cache_lengths;
+  p.lut = lookup_table;
+  p.slut = scales_lookup_table;
+  p.blocks = static_cast<uint8_t*>(blocks);
+  p.scales = scales;
+  p.status = status_ptr();
+  if (!p.status) return fail(MLA_ERR_CUDA, "status word address unavailable");
+  p.B = s->batch;
+  p.T = static_cast<int>(num_new_tokens);
+  p.P = s->page_size;
+  p.KVD = s->kv_dim;
+  p.NL = s->num_layers;
+  p.layer = static_cast<int>(layer_idx);
+  p.NB = s->num_blocks;
+  p.NSB = s->num_scale_blocks;
+  p.max_pages = s->max_pages;
+  p.divT = make_fastdiv(num_new_tokens);
+  const uint64_t per_cta = 32 * mla::KVS_WARPS / mla::KVS_LANES;     // tokens per CTA
+  const uint64_t grid = (tokens + per_cta - 1) / per_cta;
+  mla::mla_kv_store_kernel<<<static_cast<unsigned>(grid), 32 * mla::KVS_WARPS, 0, stream>>>(p);
   MLA_CUDA(cudaGetLastError());
   return MLA_OK;
 }

@@ -168,6 +168,50 @@ def quantize_rows_e4m3(x: torch.Tensor):
     return codes.view(torch.uint8), scale
 
 
+@dataclass
+class StoreInputs:
+    """Tensors of one KV-store call: new tokens' latent and the (pre-assigned) pages they go to."""
+    latent: torch.Tensor            # bf16 [B, T, 576]
+    cache_lengths: torch.Tensor     # int32 view of uint32 [B]
+    lookup_table: torch.Tensor      # int32 view of uint32 [B, max_pages]
+    scales_lookup_table: Optional[torch.Tensor]
+    blocks: torch.Tensor            # uint8 [NB, 1, L, P, 1, 576]
+    scales: torch.Tensor            # fp32 [NSB, 1, L, P, 1, 1]
+    layer_idx: int
+
+    def algorithmic_bytes(self) -> int:
+        """bf16 latent read (1152 B) + e4m3 row (576 B) + fp32 scale (4 B) written, per token."""
+        B, T, _ = self.latent.shape
+        return B * T * (2 * HEAD_DIM + HEAD_DIM + 4)
+
+
+def make_store_inputs(batch: int, new_tokens: int, page_size: int, max_cached: int, seed: int, device="cpu",
+                      num_layers: int = 1, layer_idx: int = 0) -> StoreInputs:
+    """Seeded inputs of the KV-store step: cached lengths uniform in [0, max_cached], every page a
+    request needs for its cached plus new tokens assigned from a randomly permuted pool, latent
+    N(0, 1) in bf16.  The pool's bytes start as zeros (the store writes the new rows)."""
+    gc = torch.Generator()
+    gc.manual_seed(seed)
+    L = torch.randint(0, max_cached + 1, (batch,), generator=gc)
+    pages = (L + new_tokens + page_size - 1) // page_size
+    max_pages = int(pages.max().item())
+    nb = int(pages.sum().item())
+    perm = torch.randperm(nb, generator=gc).to(torch.int64)
+    lut = torch.full((batch, max_pages), INVALID_PAGE, dtype=torch.int64)
+    k = 0
+    for b in range(batch):
+        n = int(pages[b])
+        lut[b, :n] = perm[k:k + n]
+        k += n
+    g = torch.Generator(device=torch.device(device))
+    g.manual_seed(seed + 1)
+    latent = torch.randn((batch, new_tokens, HEAD_DIM), generator=g, device=device).to(torch.bfloat16)
+    blocks = torch.zeros((nb, 1, num_layers, page_size, 1, HEAD_DIM), dtype=torch.uint8, device=device)
+    scales = torch.zeros((nb, 1, num_layers, page_size, 1, 1), dtype=torch.float32, device=device)
+    return StoreInputs(latent=latent, cache_lengths=u32_as_i32(L).to(device), lookup_table=u32_as_i32(lut).to(device),
+                       scales_lookup_table=None, blocks=blocks, scales=scales, layer_idx=layer_idx)
+
+
 def make_inputs(cfg: DecodeConfig, device="cpu", *, poison: bool = False,
                 lengths: Optional[torch.Tensor] = None, seed: Optional[int] = None,
                 q_zero: bool = False, chunk_tokens: int = 1 << 20) -> DecodeInputs:

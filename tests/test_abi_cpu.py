@@ -65,6 +65,25 @@ def test_host_validation_rejects_null_and_misaligned(lib):
     assert _call(lib, _shape(), T=0) == 1
 
 
+def _store(lib, shape, latent=FAKE, lens=FAKE, lut=FAKE, slut=None, T=1, layer=0, blocks=FAKE, scales=FAKE):
+    return lib.mla_kv_store_fp8(latent, lens, lut, slut, T, layer,
+                                ctypes.byref(shape) if shape is not None else None, blocks, scales, None)
+
+
+def test_kv_store_host_validation(lib):
+    assert _store(lib, None) == 1
+    assert _store(lib, _shape(), latent=None) == 1
+    assert _store(lib, _shape(), blocks=None) == 1
+    assert _store(lib, _shape(), latent=ctypes.c_void_p(0x10008)) == 1
+    assert _store(lib, _shape(), layer=1) == 1
+    assert _store(lib, _shape(head_dim=512)) == 2
+    assert _store(lib, _shape(head_dim_granularity=9)) == 2
+    assert _store(lib, _shape(num_kv_heads=2)) == 2
+    # no new tokens: nothing to launch, nothing dereferenced
+    assert _store(lib, _shape(), T=0) == 0
+    assert _store(lib, _shape(batch=0)) == 0
+
+
 def test_set_num_clusters_range(lib):
     assert lib.mla_set_num_clusters(-1) == 1
     assert lib.mla_set_num_clusters(0) == 0
