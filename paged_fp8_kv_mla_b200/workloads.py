@@ -61,6 +61,7 @@ class DecodeConfig:
     kv_dim: int = 1
     seed: int = 1000
     softmax_scale: float = SOFTMAX_SCALE
+    scale_blocks: int = 1             # scales per token (head_dim_granularity); each covers 576 / g dims
 
     @property
     def head_dim(self) -> int:
@@ -158,14 +159,18 @@ def _lengths(cfg: DecodeConfig, g: torch.Generator) -> torch.Tensor:
     raise ValueError(cfg.length_kind)
 
 
-def quantize_rows_e4m3(x: torch.Tensor):
-    """Per-row amax/448 fp32 scale and saturating RNE e4m3 codes (data generation only)."""
+def quantize_rows_e4m3(x: torch.Tensor, blocks: int = 1):
+    """amax/448 fp32 scales (one per row, or one per each of `blocks` equal slices of a row) and
+    saturating RNE e4m3 codes (data generation only).  Returns (codes uint8 like x, scales [..., blocks]
+    or [...] when blocks == 1)."""
     xf = x.to(torch.float32)
-    amax = xf.abs().amax(dim=-1)
+    xb = xf.reshape(*xf.shape[:-1], blocks, xf.shape[-1] // blocks)
+    amax = xb.abs().amax(dim=-1)
     scale = amax / E4M3_MAX
     scale = torch.where(amax > 0, scale, torch.ones_like(scale))
-    codes = (xf / scale[..., None]).clamp(-E4M3_MAX, E4M3_MAX).to(torch.float8_e4m3fn)
-    return codes.view(torch.uint8), scale
+    codes = (xb / scale[..., None]).clamp(-E4M3_MAX, E4M3_MAX).to(torch.float8_e4m3fn)
+    codes = codes.reshape(xf.shape).view(torch.uint8)
+    return codes, (scale[..., 0] if blocks == 1 else scale)
 
 
 @dataclass
@@ -261,12 +266,13 @@ def make_inputs(cfg: DecodeConfig, device="cpu", *, poison: bool = False,
 
     KVD, NL, li = cfg.kv_dim, cfg.num_layers, cfg.layer_idx
     D = HEAD_DIM
+    SG = cfg.scale_blocks
     if poison:
         blocks = torch.full((NB, KVD, NL, P, 1, D), 0x7F, dtype=torch.uint8, device=dev)
-        scales = torch.full((NSB, KVD, NL, P, 1, 1), float("nan"), dtype=torch.float32, device=dev)
+        scales = torch.full((NSB, KVD, NL, P, 1, SG), float("nan"), dtype=torch.float32, device=dev)
     else:
         blocks = torch.empty((NB, KVD, NL, P, 1, D), dtype=torch.uint8, device=dev)
-        scales = torch.empty((NSB, KVD, NL, P, 1, 1), dtype=torch.float32, device=dev)
+        scales = torch.empty((NSB, KVD, NL, P, 1, SG), dtype=torch.float32, device=dev)
         # every slot gets real random data (other layers, spare pages, tails)
         flat_b = blocks.view(-1, D)
         flat_s = scales.view(-1)
@@ -293,9 +299,9 @@ def make_inputs(cfg: DecodeConfig, device="cpu", *, poison: bool = False,
         if cfg.outlier_rate > 0:
             m = torch.rand((s1 - s0,), generator=g, device=dev) < cfg.outlier_rate
             x = torch.where(m[:, None], x * cfg.outlier_mult, x)
-        c, s = quantize_rows_e4m3(x.to(torch.bfloat16))
+        c, s = quantize_rows_e4m3(x.to(torch.bfloat16), SG)
         blocks[blk_d[s0:s1], 0, li, slot_d[s0:s1], 0, :] = c
-        scales[sblk_d[s0:s1], 0, li, slot_d[s0:s1], 0, 0] = s
+        scales[sblk_d[s0:s1], 0, li, slot_d[s0:s1], 0, :] = s.reshape(s1 - s0, SG)
 
     if q_zero:
         q = torch.zeros((B, T, H, D), dtype=torch.bfloat16, device=dev)
