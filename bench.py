@@ -40,6 +40,8 @@ def parse():
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--config", type=int, default=1)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--scale-blocks", type=int, default=1,
+                    help="decode with g scales per token (head_dim_granularity), each over 576/g dims")
     ap.add_argument("--op", choices=["decode", "kv_store"], default="decode",
                     help="decode (the default contract line) or the KV-store step that fills the cache")
     ap.add_argument("--no-cpu-baseline", action="store_true")
@@ -322,6 +324,9 @@ def main():
     from paged_fp8_kv_mla_b200 import workloads as W
     M.load()
     cfg = W.CONFIGS[args.config]
+    if args.scale_blocks > 1:
+        from dataclasses import replace
+        cfg = replace(cfg, name=f"{cfg.name}_g{args.scale_blocks}", scale_blocks=args.scale_blocks)
     seed = cfg.seed + 7919 * rank
     inp = W.make_inputs(cfg, device="cuda", seed=seed)
     kv_bytes = inp.kv_scale_bytes()

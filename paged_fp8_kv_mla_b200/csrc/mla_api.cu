@@ -96,9 +96,13 @@ mla_status_t ensure_workspace(int dev, size_t bytes, void** out) {
 mla_status_t device_setup(int dev, int* nc_out) {
   std::lock_guard<std::mutex> lk(g_mu);
   if (!g_attr_set[dev]) {
-    MLA_CUDA(cudaFuncSetAttribute(mla::mla_decode_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+    MLA_CUDA(cudaFuncSetAttribute(mla::mla_decode_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                   static_cast<int>(mla::SMEM_ALLOC)));
-    MLA_CUDA(cudaFuncSetAttribute(mla::mla_dequant_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+    MLA_CUDA(cudaFuncSetAttribute(mla::mla_decode_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                  static_cast<int>(mla::SMEM_ALLOC)));
+    MLA_CUDA(cudaFuncSetAttribute(mla::mla_dequant_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                  static_cast<int>(mla::DQ_SMEM_ALLOC)));
+    MLA_CUDA(cudaFuncSetAttribute(mla::mla_dequant_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                   static_cast<int>(mla::DQ_SMEM_ALLOC)));
     g_attr_set[dev] = true;
   }
@@ -114,8 +118,10 @@ mla_status_t device_setup(int dev, int* nc_out) {
     attr[0].val.clusterDim.z = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
-    int n = 0;
-    MLA_CUDA(cudaOccupancyMaxActiveClusters(&n, mla::mla_decode_kernel, &cfg));
+    int n = 0, n_bs = 0;
+    MLA_CUDA(cudaOccupancyMaxActiveClusters(&n, mla::mla_decode_kernel<false>, &cfg));
+    MLA_CUDA(cudaOccupancyMaxActiveClusters(&n_bs, mla::mla_decode_kernel<true>, &cfg));
+    n = n < n_bs ? n : n_bs;
     if (n <= 0) return fail(MLA_ERR_UNSUPPORTED, "no 2-CTA cluster of the decode kernel fits on this device");
     g_default_nc[dev] = n;
   }
@@ -151,8 +157,11 @@ mla_status_t check_cache(const void* blocks, const float* scales, const uint32_t
   if (s->head_dim != mla::HEAD_DIM || s->v_dim != mla::V_DIM)
     return fail(MLA_ERR_UNSUPPORTED, "head_dim must be 576 and v_dim 512 (got %d, %d)", s->head_dim, s->v_dim);
   if (s->num_kv_heads != 1) return fail(MLA_ERR_UNSUPPORTED, "num_kv_heads must be 1 (MLA latent cache)");
-  if (s->head_dim_granularity != 1)
-    return fail(MLA_ERR_UNSUPPORTED, "only one scale per token (head_dim_granularity 1) is implemented");
+  const int g = s->head_dim_granularity;
+  if (mla::HEAD_DIM % g != 0 || (mla::HEAD_DIM / g) % 16 != 0)
+    return fail(MLA_ERR_UNSUPPORTED,
+                "head_dim_granularity %d: each scale must cover a multiple of 16 of the 576 dims "
+                "(1, 2, 3, 4, 6, 9, 12, 18 or 36)", g);
   if (s->page_size % 16 != 0) return fail(MLA_ERR_UNSUPPORTED, "page_size must be a multiple of 16");
   if (layer_idx >= static_cast<uint32_t>(s->num_layers))
     return fail(MLA_ERR_INVALID_ARG, "layer_idx %u >= num_layers %d", layer_idx, s->num_layers);
@@ -183,6 +192,8 @@ mla_status_t check_cache(const void* blocks, const float* scales, const uint32_t
   p->max_pages = s->max_pages;
   p->blocks = static_cast<const uint8_t*>(blocks);
   p->divP = make_fastdiv(static_cast<uint32_t>(p->P));
+  p->SG = s->head_dim_granularity;
+  p->divCPB = make_fastdiv(static_cast<uint32_t>(mla::HEAD_DIM / 16 / s->head_dim_granularity));
   p->divG = make_fastdiv(static_cast<uint32_t>(p->G));
   p->divT = make_fastdiv(static_cast<uint32_t>(p->T));
   *rows = r;
@@ -264,7 +275,11 @@ mla_status_t launch_path(const mla::DecodeParams& p, int NC, const uint32_t* cac
   cfg.attrs = attr;
   cfg.numAttrs = 2;
   if (timing) MLA_CUDA(cudaEventRecord(g_ev_before, stream));
-  MLA_CUDA(cudaLaunchKernelEx(&cfg, mla::mla_decode_kernel, p));
+  if (p.SG > 1) {
+    MLA_CUDA(cudaLaunchKernelEx(&cfg, mla::mla_decode_kernel<true>, p));
+  } else {
+    MLA_CUDA(cudaLaunchKernelEx(&cfg, mla::mla_decode_kernel<false>, p));
+  }
   if (timing) MLA_CUDA(cudaEventRecord(g_ev_after, stream));
 
   const int per_item = mla::MROWS / mla::COMBINE_HEADS;
@@ -433,8 +448,13 @@ mla_status_t mla_gather_dequant_bf16(const void* blocks, const float* scales, co
   const int tiles = static_cast<int>((static_cast<uint64_t>(max_keys) + mla::BN - 1) / mla::BN);
   const int64_t gx = static_cast<int64_t>(p.B) * tiles;
   if (gx > 0x7FFFFFFF) return fail(MLA_ERR_UNSUPPORTED, "grid too large");
-  mla::mla_dequant_kernel<<<dim3(static_cast<unsigned>(gx), 2), mla::DQ_THREADS, mla::DQ_SMEM_ALLOC, stream>>>(
-      p, cache_lengths, static_cast<int>(max_keys), tiles, static_cast<uint16_t*>(out_k));
+  if (p.SG > 1) {
+    mla::mla_dequant_kernel<true><<<dim3(static_cast<unsigned>(gx), 2), mla::DQ_THREADS, mla::DQ_SMEM_ALLOC, stream>>>(
+        p, cache_lengths, static_cast<int>(max_keys), tiles, static_cast<uint16_t*>(out_k));
+  } else {
+    mla::mla_dequant_kernel<false><<<dim3(static_cast<unsigned>(gx), 2), mla::DQ_THREADS, mla::DQ_SMEM_ALLOC, stream>>>(
+        p, cache_lengths, static_cast<int>(max_keys), tiles, static_cast<uint16_t*>(out_k));
+  }
   MLA_CUDA(cudaGetLastError());
   return MLA_OK;
 }

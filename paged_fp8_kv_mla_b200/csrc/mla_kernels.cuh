@@ -139,6 +139,8 @@ struct DecodeParams {
   unsigned int* status;
   int B, T, H, G, P, KVD, NL, layer, NB, NSB, max_pages, items, NC;
   FastDiv divP, divG, divT;        // by the page size, the head-group count and the query length
+  int SG;                          // scales per token (head_dim_granularity): 1, or g with 576 / g % 16 == 0
+  FastDiv divCPB;                  // 16-byte chunks per scale block (36 / g)
   float scale_log2;                // softmax_scale * log2(e)
 };
 
@@ -308,10 +310,13 @@ __device__ __forceinline__ int own_k(int s, int c) {
   return s == 0 ? 4 : s == 1 ? 1 - c : s == 2 ? 3 - c : s == 3 ? c : 2 + c;
 }
 
+// With per-token scales (BS = false) only so[0] and sp[0] are used; with block scales (BS = true,
+// head_dim_granularity g > 1) each register slot carries the scale of its chunk's block, scale
+// index = chunk / (36 / g).
 struct RawTile {
   uint4 own[5];
   uint4 oth[2];
-  float so, sp;
+  float so[5], sp[2];
   bool own_ok, oth_ok;
 };
 
@@ -371,50 +376,58 @@ __device__ __forceinline__ TilePtrs lut_finish(const DecodeParams& p, const LutV
 // scale), and the other key's chunks (with its scale).  The converter issues the next tile's slots
 // 0-2 before converting the current tile's own key and the rest after it, which keeps fewer
 // registers live at once (measured: the decode runs ~20% faster than with one fetch up front).
-template <int S0, int S1>
+template <int S0, int S1, bool BS>
 __device__ __forceinline__ void fetch_own_part(const DecodeParams& p, const TilePtrs& T, int c, int t, RawTile& R) {
   const int q = conv_q(t);
   R.own_ok = T.own_ok;
   if (T.own_ok) {
     const uint8_t* ov = p.blocks + static_cast<size_t>(T.ov) * HEAD_DIM;
-    if (S0 == 0) R.so = __ldg(p.scales + T.os);
+    if (!BS && S0 == 0) R.so[0] = __ldg(p.scales + T.os);
 #pragma unroll
     for (int sl = S0; sl < S1; ++sl) {
       const int qq = q + 8 * own_k(sl, c);
-      if (qq < 36) R.own[sl] = ptx::ldg_stream_v4(ov + 16 * qq);
+      if (qq < 36) {
+        R.own[sl] = ptx::ldg_stream_v4(ov + 16 * qq);
+        if (BS) R.so[sl] = __ldg(p.scales + static_cast<size_t>(T.os) * p.SG + p.divCPB.div(qq));
+      }
     }
   }
 }
 
+template <bool BS>
 __device__ __forceinline__ void fetch_oth(const DecodeParams& p, const TilePtrs& T, int c, int t, RawTile& R) {
   const int q = conv_q(t);
   R.oth_ok = T.oth_ok;
   if (T.oth_ok) {
     const uint8_t* pv = p.blocks + static_cast<size_t>(T.pv) * HEAD_DIM;
-    R.sp = __ldg(p.scales + T.ps);
+    if (!BS) R.sp[0] = __ldg(p.scales + T.ps);
 #pragma unroll
     for (int k = 0; k < 2; ++k) {
       const int jc = q + 8 * k;                              // chunk index within D_c (0..15)
       const int qq = jc < 8 ? 8 * c + jc : 16 + 8 * c + (jc - 8);
       R.oth[k] = ptx::ldg_stream_v4(pv + 16 * qq);
+      if (BS) R.sp[k] = __ldg(p.scales + static_cast<size_t>(T.ps) * p.SG + p.divCPB.div(qq));
     }
   }
 }
 
+template <bool BS>
 __device__ __forceinline__ void fetch(const DecodeParams& p, const TilePtrs& T, int c, int t, RawTile& R) {
-  fetch_own_part<0, 5>(p, T, c, t, R);
-  fetch_oth(p, T, c, t, R);
+  fetch_own_part<0, 5, BS>(p, T, c, t, R);
+  fetch_oth<BS>(p, T, c, t, R);
 }
 
 // All three phases at once (for callers with nothing to overlap).  Returns false on a bad page id.
+template <bool BS>
 __device__ __forceinline__ bool load_tile(const DecodeParams& p, int c, int t, int b, int nvis, int j, RawTile& R) {
   bool bad;
   const TilePtrs T = lut_finish(p, lut_issue(p, c, t, b, nvis, j), bad);
-  fetch(p, T, c, t, R);
+  fetch<BS>(p, T, c, t, R);
   return !bad;
 }
 
 // Dequantises thread t's part of a loaded tile into the K half buffer `sk` and the V buffer `sv`.
+template <bool BS>
 __device__ __forceinline__ void store_tile(int c, int t, const RawTile& R, uint32_t sk, uint32_t sv) {
   const int row = conv_row(t), q = conv_q(t);
   const int vrow_own = HALF_BN * c + row;
@@ -425,7 +438,7 @@ __device__ __forceinline__ void store_tile(int c, int t, const RawTile& R, uint3
     if (qq >= 36) continue;
     uint32_t w[8];
     if (R.own_ok) {
-      dequant16(R.own[sl], R.so, w);
+      dequant16(R.own[sl], R.so[BS ? sl : 0], w);
     } else {
 #pragma unroll
       for (int x = 0; x < 8; ++x) w[x] = 0u;
@@ -441,7 +454,7 @@ __device__ __forceinline__ void store_tile(int c, int t, const RawTile& R, uint3
     const int jc = q + 8 * k;
     uint32_t w[8];
     if (R.oth_ok) {
-      dequant16(R.oth[k], R.sp, w);
+      dequant16(R.oth[k], R.sp[BS ? k : 0], w);
     } else {
 #pragma unroll
       for (int x = 0; x < 8; ++x) w[x] = 0u;
@@ -455,6 +468,7 @@ __device__ __forceinline__ void store_tile(int c, int t, const RawTile& R, uint3
 // store_k keeps the two chunks of the own key that also belong to the V operand (slots 3 and 4:
 // V chunks q and q + 8) so that store_v need not convert them again; they come last so that they
 // occupy registers only once the other chunks are done.
+template <bool BS>
 __device__ __forceinline__ void store_k(int c, int t, const RawTile& R, uint32_t sk, uint32_t (&keep0)[8],
                                         uint32_t (&keep1)[8]) {
   const int row = conv_row(t), q = conv_q(t);
@@ -464,7 +478,7 @@ __device__ __forceinline__ void store_k(int c, int t, const RawTile& R, uint32_t
     if (qq >= 36) continue;
     uint32_t w[8];
     if (R.own_ok) {
-      dequant16(R.own[sl], R.so, w);
+      dequant16(R.own[sl], R.so[BS ? sl : 0], w);
     } else {
 #pragma unroll
       for (int x = 0; x < 8; ++x) w[x] = 0u;
@@ -481,6 +495,7 @@ __device__ __forceinline__ void store_k(int c, int t, const RawTile& R, uint32_t
   }
 }
 
+template <bool BS>
 __device__ __forceinline__ void store_v(int c, int t, const RawTile& R, const uint32_t (&keep0)[8],
                                         const uint32_t (&keep1)[8], uint32_t sv) {
   const int row = conv_row(t), q = conv_q(t);
@@ -493,7 +508,7 @@ __device__ __forceinline__ void store_v(int c, int t, const RawTile& R, const ui
     const int jc = q + 8 * k;
     uint32_t w[8];
     if (R.oth_ok) {
-      dequant16(R.oth[k], R.sp, w);
+      dequant16(R.oth[k], R.sp[BS ? k : 0], w);
     } else {
 #pragma unroll
       for (int x = 0; x < 8; ++x) w[x] = 0u;
@@ -574,6 +589,7 @@ struct TileCursor {
 // parity; the K half of tile g waits for Q.K^T(g-2) (S_FULL), the V operand for P.V(g-2).
 // Returns early (with the abort flag set by the failing wait) when a wait gives up.
 // =============================================================================================
+template <bool BS>
 __device__ __forceinline__ void converter_role(const DecodeParams& p, int k, uint32_t base, int lane,
                                                volatile uint32_t* abort, uint32_t peer_abort, uint32_t c) {
   const int C = static_cast<int>(c);
@@ -592,7 +608,7 @@ __device__ __forceinline__ void converter_role(const DecodeParams& p, int k, uin
   {
     const TilePtrs t0 = lut_finish(p, lut_issue(p, C, t, item_b(p, cur.item), cur.nvis, cur.j), bad);
     if (bad) raise_status(p.status, STATUS_BOUNDS);
-    fetch(p, t0, C, t, ra);
+    fetch<BS>(p, t0, C, t, ra);
   }
   TilePtrs t1{};
   if (n1.valid) {
@@ -607,13 +623,13 @@ __device__ __forceinline__ void converter_role(const DecodeParams& p, int k, uin
     MLA_WAIT_RET(BAR(B_S_FULL + kb), free_par);                                                          \
     if (t == 0) MLA_TRACE_EV(g, 1);                                                                      \
     if (t == 224) MLA_TRACE_EV(g, 26);                                                                   \
-    if (n1.valid) fetch_own_part<0, 3>(p, t1, C, t, RNXT);                                                          \
+    if (n1.valid) fetch_own_part<0, 3, BS>(p, t1, C, t, RNXT);                                                          \
     if (t == 0) MLA_TRACE_EV(g, 16);                                                                     \
     uint32_t keep0[8], keep1[8];                                                                         \
-    store_k(C, t, RCUR, base + SK0 + kb * SK_STRIDE, keep0, keep1);                                      \
+    store_k<BS>(C, t, RCUR, base + SK0 + kb * SK_STRIDE, keep0, keep1);                                      \
     if (n1.valid) {                                                                                     \
-      fetch_own_part<3, 5>(p, t1, C, t, RNXT);                                                           \
-      fetch_oth(p, t1, C, t, RNXT);                                                                      \
+      fetch_own_part<3, 5, BS>(p, t1, C, t, RNXT);                                                           \
+      fetch_oth<BS>(p, t1, C, t, RNXT);                                                                      \
     }                                                          \
     LutVals v2{};                                                                                        \
     if (n2.valid) v2 = lut_issue(p, C, t, item_b(p, n2.item), n2.nvis, n2.j);                         \
@@ -627,7 +643,7 @@ __device__ __forceinline__ void converter_role(const DecodeParams& p, int k, uin
     MLA_WAIT_RET(BAR(B_PV_DONE + kb), free_par);                                                         \
     if (t == 0) MLA_TRACE_EV(g, 6);                                                                      \
     if (t == 224) MLA_TRACE_EV(g, 29);                                                                   \
-    store_v(C, t, RCUR, keep0, keep1, base + SV0 + kb * SV_STRIDE);                                      \
+    store_v<BS>(C, t, RCUR, keep0, keep1, base + SV0 + kb * SV_STRIDE);                                      \
     ptx::fence_proxy_async_smem();                                                                       \
     __syncwarp();                                                                                        \
     if (lane == 0) ptx::mbar_arrive_cluster(v_full0 + 8u * kb);                                          \
@@ -659,6 +675,8 @@ __device__ __forceinline__ void converter_role(const DecodeParams& p, int k, uin
 // =============================================================================================
 // decode kernel
 // =============================================================================================
+// BS: block scales (head_dim_granularity > 1) instead of one scale per token.
+template <bool BS>
 __global__ void __launch_bounds__(NUM_THREADS, 1) mla_decode_kernel(const __grid_constant__ DecodeParams p) {
   if (threadIdx.x == 0) MLA_MARK_MIN(1);
   ptx::griddep_launch_dependents();   // the combine kernel may start launching (it waits for this grid)
@@ -714,7 +732,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) mla_decode_kernel(const __grid
 
   if (warp < CONV_WARPS) {
     // ------------------------------------------------------------------ converter
-    converter_role(p, k, base, lane, abort, peer_abort, c);
+    converter_role<BS>(p, k, base, lane, abort, peer_abort, c);
   } else if (warp < SM_WARP0 + 4) {
     // ------------------------------------------------------------------ softmax / epilogue
     const int t = threadIdx.x - 32 * SM_WARP0;
@@ -1183,6 +1201,7 @@ constexpr uint32_t DQ_SK = 0;
 constexpr uint32_t DQ_SV = SK_STRIDE;
 constexpr uint32_t DQ_SMEM_ALLOC = SK_STRIDE + SV_STRIDE + 1024;
 
+template <bool BS>
 __global__ void __launch_bounds__(DQ_THREADS)
 mla_dequant_kernel(const __grid_constant__ DecodeParams p, const uint32_t* cache_lengths, int max_keys,
                    int tiles_per_req, uint16_t* out_k) {
@@ -1195,8 +1214,8 @@ mla_dequant_kernel(const __grid_constant__ DecodeParams p, const uint32_t* cache
   const int n = min(static_cast<int>(min(cache_lengths[b], 0x3FFFFFFFu)) + p.T, max_keys);
   if (j * BN + HALF_BN * c >= n || b >= p.B) return;
   RawTile R;
-  if (!load_tile(p, c, threadIdx.x, b, n, j, R)) raise_status(p.status, STATUS_BOUNDS);
-  store_tile(c, threadIdx.x, R, base + DQ_SK, base + DQ_SV);
+  if (!load_tile<BS>(p, c, threadIdx.x, b, n, j, R)) raise_status(p.status, STATUS_BOUNDS);
+  store_tile<BS>(c, threadIdx.x, R, base + DQ_SK, base + DQ_SV);
   __syncthreads();
   const int nv = min(HALF_BN, n - (j * BN + HALF_BN * c));
   for (int id = threadIdx.x; id < HALF_BN * 72; id += DQ_THREADS) {

@@ -49,7 +49,8 @@ def _call(lib, shape, q=FAKE, blocks=FAKE, scales=FAKE, lens=FAKE, lut=FAKE, slu
 
 @pytest.mark.parametrize("kw,want", [
     (dict(head_dim=512), 2), (dict(v_dim=256), 2), (dict(num_kv_heads=2), 2),
-    (dict(head_dim_granularity=9), 2), (dict(page_size=24), 2), (dict(num_layers=0), 1),
+    (dict(head_dim_granularity=72), 2), (dict(head_dim_granularity=5), 2), (dict(page_size=24), 2),
+    (dict(num_layers=0), 1),
     (dict(max_pages=2), 1),
 ])
 def test_host_validation_rejects_bad_shapes(lib, kw, want):
