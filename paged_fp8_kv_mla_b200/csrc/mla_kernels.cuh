@@ -264,16 +264,16 @@ __device__ __forceinline__ bool poll_bar(uint32_t addr, uint32_t parity, volatil
 // ---------------------------------------------------------------------------------------------
 __device__ __forceinline__ void dequant16(uint4 raw, float s, uint32_t (&w)[8]) {
   const uint32_t in[4] = {raw.x, raw.y, raw.z, raw.w};
+  const float2 ss = make_float2(s, s);
 #pragma unroll
   for (int k = 0; k < 4; ++k) {
     const uint32_t h0 = ptx::e4m3x2_to_f16x2(static_cast<uint16_t>(in[k] & 0xFFFFu));
     const uint32_t h1 = ptx::e4m3x2_to_f16x2(static_cast<uint16_t>(in[k] >> 16));
-    const float f0 = ptx::mul_rn(ptx::f16_lo_to_f32(h0), s);
-    const float f1 = ptx::mul_rn(ptx::f16_hi_to_f32(h0), s);
-    const float f2 = ptx::mul_rn(ptx::f16_lo_to_f32(h1), s);
-    const float f3 = ptx::mul_rn(ptx::f16_hi_to_f32(h1), s);
-    w[2 * k] = ptx::pack_bf16x2(f0, f1);
-    w[2 * k + 1] = ptx::pack_bf16x2(f2, f3);
+    // packed fp32 multiply (two round-to-nearest products per instruction)
+    const float2 p0 = __fmul2_rn(make_float2(ptx::f16_lo_to_f32(h0), ptx::f16_hi_to_f32(h0)), ss);
+    const float2 p1 = __fmul2_rn(make_float2(ptx::f16_lo_to_f32(h1), ptx::f16_hi_to_f32(h1)), ss);
+    w[2 * k] = ptx::pack_bf16x2(p0.x, p0.y);
+    w[2 * k + 1] = ptx::pack_bf16x2(p1.x, p1.y);
   }
 }
 
