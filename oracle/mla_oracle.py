@@ -36,6 +36,12 @@ What it computes, step by step, in the order the pages lay out the data:
    layer_idx, t % page_size, 0, :] and scale to the same slot of scales, with
    blk (and the scale block) from the page tables as in step 1.
 
+5. The scale-folding variant (per-token scales): the same gather and attention, with the
+   key and value elements left as the exact e4m3 values and the per-token scale applied to
+   score column t and to weight column t instead (attend_scale_folded).  Exactly, this is
+   attention over the unrounded products e4m3 * s_t; it differs from step 2's rounded keys by
+   the fp32 and bf16 roundings of the dequant (reading R18).
+
 Everything after the e4m3 decode is float64 (the dequantised bf16 values are
 exact in float64).  Points the pages leave open and the reading taken here:
 cache_lengths count only tokens cached before this step (R1); query i sees
@@ -276,6 +282,63 @@ def decode(q, blocks, scales, cache_lengths, lookup_table, scales_lookup_table,
                 weights[(b, i)] = r[2]
     if return_weights:
         return out, lse, weights
+    return out, lse
+
+
+# ----------------------------------------------------------------------------
+# scale-folding variant (per-token scales only)
+# ----------------------------------------------------------------------------
+def attend_scale_folded(q, codes, scale, softmax_scale):
+    """Attention with the per-token scale folded out of the keys and values.
+
+    The key and value elements stay the exact e4m3 values C[t, d]; the scale s_t multiplies
+    column t of the scores and column t of the softmax weights instead:
+      x[t] = f32(softmax_scale) * s_t * sum_d q[d] C[t, d],
+      lse = log sum_t exp(x[t]),  w[t] = exp(x[t] - lse),
+      out[v] = sum_t (w[t] s_t) C[t, v]   (v < 512).
+    In exact arithmetic this is attention over the unrounded keys K[t, d] = s_t C[t, d] (no fp32
+    or bf16 rounding of the dequantised values), which the tests check.
+    """
+    q = np.asarray(q, dtype=np.float64)
+    C = e4m3_decode(codes)                             # [n, 576], exact
+    s = np.asarray(scale, dtype=np.float32).astype(np.float64).reshape(-1)
+    ss = float(np.float32(softmax_scale))
+    x = ss * (q @ C.T) * s[None, :]                    # score columns scaled by s_t
+    mx = x.max(axis=1, keepdims=True)
+    lse = (mx + np.log(np.exp(x - mx).sum(axis=1, keepdims=True)))[:, 0]
+    w = np.exp(x - lse[:, None])
+    out = (w * s[None, :]) @ C[:, :V_DIM]              # weight columns scaled by s_t
+    return out, lse
+
+
+def decode_scale_folded(q, blocks, scales, cache_lengths, lookup_table, scales_lookup_table,
+                        max_prompt_length, layer_idx, softmax_scale, requests=None, heads=None):
+    """decode() with the scale-folding variant's arithmetic (one fp32 scale per token).
+
+    Same gather and visibility rules as decode(); rows not computed are NaN.
+    """
+    q = np.asarray(q)
+    if q.dtype == np.uint16:
+        q = bf16_bits_to_f64(q)
+    q = q.astype(np.float64)
+    B, T, H, D = q.shape
+    assert D == HEAD_DIM
+    if np.asarray(scales).shape[-1] != 1:
+        raise ValueError("the scale-folding variant takes one scale per token")
+    T = int(max_prompt_length)
+    L = np.asarray(cache_lengths).astype(np.int64) & 0xFFFFFFFF
+    n_all = num_keys(L, T)
+    out = np.full((B, T, H, V_DIM), np.nan)
+    lse = np.full((B, T, H), np.nan)
+    reqs = range(B) if requests is None else requests
+    hs = np.arange(H) if heads is None else np.asarray(heads)
+    for b in reqs:
+        codes, sc = gather_request(blocks, scales, lookup_table, scales_lookup_table, b, int(n_all[b]), layer_idx)
+        for i in range(T):
+            vis = int(L[b]) + i + 1
+            r = attend_scale_folded(q[b, i, hs], codes[:vis], sc[:vis, 0], softmax_scale)
+            out[b, i, hs] = r[0]
+            lse[b, i, hs] = r[1]
     return out, lse
 
 
