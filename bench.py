@@ -42,6 +42,8 @@ def parse():
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--scale-blocks", type=int, default=1,
                     help="decode with g scales per token (head_dim_granularity), each over 576/g dims")
+    ap.add_argument("--fold-scales", action="store_true",
+                    help="time the scale-folding decode (per-token scale on score and weight columns)")
     ap.add_argument("--op", choices=["decode", "kv_store"], default="decode",
                     help="decode (the default contract line) or the KV-store step that fills the cache")
     ap.add_argument("--no-cpu-baseline", action="store_true")
@@ -132,7 +134,7 @@ class ClockSampler:
         return {"sm_mhz": sm[len(sm) // 2], "sm_max_mhz": mx, "reasons": reasons, "samples": len(rows)}
 
 
-def cpu_oracle_baseline(inp, budget_s, rank_requests=None):
+def cpu_oracle_baseline(inp, budget_s, rank_requests=None, fold=False):
     """The float64 oracle, as it stands, on whole requests of the same workload until ~budget_s."""
     import numpy as np
     from oracle import mla_oracle as O
@@ -147,9 +149,10 @@ def cpu_oracle_baseline(inp, budget_s, rank_requests=None):
     order = rank_requests if rank_requests is not None else list(range(len(n)))
     done, nbytes = [], 0
     t0 = time.perf_counter()
+    fn = O.decode_scale_folded if fold else O.decode
     for b in order:
-        O.decode(a["q"], a["blocks"], a["scales"], a["cache_lengths"], a["lookup_table"],
-                 a["scales_lookup_table"], a["max_prompt_length"], a["layer_idx"], a["softmax_scale"], requests=[b])
+        fn(a["q"], a["blocks"], a["scales"], a["cache_lengths"], a["lookup_table"],
+           a["scales_lookup_table"], a["max_prompt_length"], a["layer_idx"], a["softmax_scale"], requests=[b])
         done.append(b)
         nbytes += int(n[b]) * 580
         if time.perf_counter() - t0 > budget_s:
@@ -327,6 +330,10 @@ def main():
     if args.scale_blocks > 1:
         from dataclasses import replace
         cfg = replace(cfg, name=f"{cfg.name}_g{args.scale_blocks}", scale_blocks=args.scale_blocks)
+    fold = bool(args.fold_scales)
+    if fold:
+        from dataclasses import replace
+        cfg = replace(cfg, name=f"{cfg.name}_scale_folded")
     seed = cfg.seed + 7919 * rank
     inp = W.make_inputs(cfg, device="cuda", seed=seed)
     kv_bytes = inp.kv_scale_bytes()
@@ -339,7 +346,7 @@ def main():
     stream = torch.cuda.current_stream()
 
     def step():
-        M.decode_inputs(inp, out=out, lse=lse, stream=stream)
+        M.decode_inputs(inp, out=out, lse=lse, stream=stream, fold_scales=fold)
 
     for _ in range(max(3, args.warmup)):
         flush.zero_()
@@ -405,7 +412,7 @@ def main():
             if dslut is not None:
                 dslut.copy_(hslut, non_blocking=True)
             M.decode(dq, inp.blocks, inp.scales, dl, dlut, dslut, T, inp.max_cache_length, inp.layer_idx,
-                     inp.softmax_scale, out=out, lse=lse, stream=stream)
+                     inp.softmax_scale, out=out, lse=lse, stream=stream, fold_scales=fold)
             hout.copy_(out, non_blocking=True)
             hlse.copy_(lse, non_blocking=True)
 
@@ -440,7 +447,7 @@ def main():
     tflops_k = flops / (kern_ms * 1e-3) / 1e12
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        cpu = cpu_oracle_baseline(inp, args.cpu_seconds)
+        cpu = cpu_oracle_baseline(inp, args.cpu_seconds, fold=fold)
     if rank == 0:
         line = {
             "metric": METRIC, "value": gbs, "unit": "GB/s", "n_gpus": world, "steps": K, "warmup": args.warmup,

@@ -111,6 +111,34 @@ mla_status_t mla_decode_paged_fp8(
     const mla_paged_shape_t* shape, void* out, float* lse, cudaStream_t stream);
 
 /*
+ * mla_decode_paged_fp8_scale_folded -- the decode with the per-token scale folded out of the
+ * keys and values (no counterpart on the reference pages; it rearranges their arithmetic).
+ *
+ * The key and value elements are the e4m3 values themselves, converted to bf16 exactly (every
+ * e4m3 value is a bf16 value), and the scale s_t multiplies column t of the scores and column t
+ * of the softmax weights:
+ *     x[t] = softmax_scale * s_t * <q[b,i,h,:], e4m3(code_t)>,
+ *     out[b,i,h,:] = (sum_t bf16_rn(exp(x[t] - m) * s_t) e4m3(code_t)[0:512]) / sum_t exp(x[t] - m).
+ * In exact arithmetic this is attention over the unrounded products e4m3 * s_t, so it is closer to
+ * that than mla_decode_paged_fp8 is; it differs from mla_decode_paged_fp8 by the fp32 and bf16
+ * roundings that entry point applies to each dequantised element (well inside the decode's
+ * tolerance, but not bit for bit).  The converter does no scale arithmetic, which is what makes it
+ * faster.
+ *
+ * Arguments, ownership, workspace and errors as for mla_decode_paged_fp8, with these limits:
+ * head_dim_granularity must be 1 (else MLA_ERR_UNSUPPORTED); codes 0x7F / 0xFF (e4m3 NaN) are not
+ * propagated as NaN (the cache the KV-store step writes holds none).
+ * The kernel uses the full 227 KB of shared memory of a CTA; mla_get_device_status reports
+ * MLA_ERR_UNSUPPORTED if the runtime placed dynamic shared memory so that the kernel's layout
+ * did not fit (it then writes nothing).
+ */
+mla_status_t mla_decode_paged_fp8_scale_folded(
+    const void* q, const void* blocks, const float* scales,
+    const uint32_t* cache_lengths, const uint32_t* lookup_table, const uint32_t* scales_lookup_table,
+    uint32_t max_prompt_length, uint32_t max_cache_length, uint32_t layer_idx, float softmax_scale,
+    const mla_paged_shape_t* shape, void* out, float* lse, cudaStream_t stream);
+
+/*
  * mla_decode_paged_fp8_noalloc -- the same decode, for callers that cannot allocate device memory
  * (for instance while a CUDA graph is being captured, under an allocator that owns the whole
  * device, or in a service that forbids allocation once it is running).  The reference pages have

@@ -67,6 +67,23 @@ constexpr uint32_t SRED = SP0 + 2 * SP_STRIDE;   // row-max exchange [2][128] f3
 constexpr uint32_t SBAR = SRED + 1536;
 constexpr uint32_t SMEM_USED = SBAR + 256;
 constexpr uint32_t SMEM_ALLOC = SMEM_USED + 1024;   // slack for aligning the base
+// Scale-folding mode only: the per-token scales of the last four tiles ([4][64] f32), handed from
+// the converter to the softmax warps.  It sits after SMEM_USED, inside the alignment slack, with
+// the allocation raised to the 227 KB limit; the kernel checks that the base needed at most
+// SMEM_FOLD_MAX_PAD bytes of alignment (it needs none when the runtime places dynamic shared
+// memory on a 1 KB boundary) and reports STATUS_LAYOUT otherwise.
+constexpr uint32_t SSC = SMEM_USED;
+constexpr uint32_t SSC_STRIDE = 64 * 4;
+constexpr uint32_t SMEM_ALLOC_FOLD = 232448;
+constexpr uint32_t SMEM_FOLD_MAX_PAD = SMEM_ALLOC_FOLD - SSC - 4 * SSC_STRIDE;
+static_assert(SMEM_ALLOC_FOLD >= SSC + 4 * SSC_STRIDE, "fold scale array does not fit");
+
+// How the per-token scale enters the computation.
+enum ScaleMode : int {
+  SCALE_TOKEN = 0,   // K, V = bf16_rn(f32_rn(e4m3 * s_t)), one scale per token
+  SCALE_BLOCK = 1,   // the same with g scales per token, each over 576 / g contiguous dims
+  SCALE_FOLD = 2     // K, V = exact e4m3 values; s_t scales score column t and weight column t
+};
 
 enum Bar : uint32_t {
   B_K_FULL = 0,    // [2] CTA 0: 16 warp arrivals (8 converter warps of each CTA): K half converted
@@ -83,11 +100,12 @@ enum Bar : uint32_t {
   B_RED = 17,      // [2] softmax warps of this CTA: row-max exchange of a tile (4 warp arrivals)
   B_REDL = 19,     // softmax warps of this CTA: row-sum exchange at a unit's end (4 warp arrivals)
   B_EXIT = 20,     // both CTAs: the peer has finished (1 remote arrival)
-  NUM_BARS = 21
+  B_SC_FULL = 21,  // [4] scale-folding mode: 8 converter-warp arrivals, a tile's scales are in SSC
+  NUM_BARS = 25
 };
-static_assert(8 * NUM_BARS <= 192, "barrier block overlaps the scalars after it");
-constexpr uint32_t S_TMEM_BASE = SBAR + 192;
-constexpr uint32_t S_ABORT = SBAR + 196;
+static_assert(8 * NUM_BARS <= 240, "barrier block overlaps the scalars after it");
+constexpr uint32_t S_TMEM_BASE = SBAR + 240;
+constexpr uint32_t S_ABORT = SBAR + 244;
 
 // TMEM columns (pair layout)
 constexpr uint32_t T_O = 0;                      // P.V halves: cols 0..127 (dims 0..255), 128..255 (256..511)
@@ -99,6 +117,7 @@ constexpr uint32_t IDESC_PV = ptx::idesc_bf16_f32(128, 256, false, true);
 
 constexpr unsigned STATUS_BOUNDS = 1u;
 constexpr unsigned STATUS_TIMEOUT = 2u;
+constexpr unsigned STATUS_LAYOUT = 4u;   // the shared-memory base was not aligned as the fold mode needs
 constexpr uint64_t WAIT_LIMIT_NS = 2000000000ull;   // 2 s per wait
 
 // Optional per-stage timestamps (build with -DMLA_TRACE): cluster 0 writes %clock64 values to
@@ -277,6 +296,26 @@ __device__ __forceinline__ void dequant16(uint4 raw, float s, uint32_t (&w)[8]) 
   }
 }
 
+// Scale-folding mode: 16 e4m3 bytes -> 16 bf16 values, exactly (no scale).  e4m3 -> f16 is exact
+// (every e4m3 value is a normal f16 or zero, f16 exponent field 6..23 for nonzero values, low 3
+// mantissa bits zero).  Shifting the f16 magnitude bits right by 3 lines its exponent and top 7
+// mantissa bits up with the bf16 fields, which reads as the same value times 2^-112 (a normal bf16
+// for nonzero values, zero for zero); the sign bit is put back in place and one packed bf16
+// multiply by 2^112 (exact: a power of two, result exponent field 118..135) restores the value.
+__device__ __forceinline__ uint32_t f16x2_to_bf16x2_e4m3(uint32_t h) {
+  const uint32_t mag = (h >> 3) & 0x0FFF0FFFu;
+  return ptx::mul_bf16x2(mag | (h & 0x80008000u), 0x77807780u);   // 0x7780 = bf16 2^112
+}
+
+__device__ __forceinline__ void exact16(uint4 raw, uint32_t (&w)[8]) {
+  const uint32_t in[4] = {raw.x, raw.y, raw.z, raw.w};
+#pragma unroll
+  for (int k = 0; k < 4; ++k) {
+    w[2 * k] = f16x2_to_bf16x2_e4m3(ptx::e4m3x2_to_f16x2(static_cast<uint16_t>(in[k] & 0xFFFFu)));
+    w[2 * k + 1] = f16x2_to_bf16x2_e4m3(ptx::e4m3x2_to_f16x2(static_cast<uint16_t>(in[k] >> 16)));
+  }
+}
+
 // Byte offset of 16-byte unit `u` (0..7) of row `r` in a K-major SWIZZLE_128B atom column whose
 // 8-row groups are 1024 B apart.
 __device__ __forceinline__ uint32_t sw128_off(int r, int u) {
@@ -372,14 +411,15 @@ __device__ __forceinline__ TilePtrs lut_finish(const DecodeParams& p, const LutV
   return T;
 }
 
-// A tile's bytes are fetched in parts: register slots [S0, S1) of the own key (slot 0 brings the
-// scale), and the other key's chunks (with its scale).  The converter issues the next tile's slots
-// 0-2 before converting the current tile's own key and the rest after it, which keeps fewer
-// registers live at once (measured: the decode runs ~20% faster than with one fetch up front).
+// A tile's bytes are fetched in parts: register slots [S0, S1) of the own key, and the other key's
+// chunks.  With one scale per token, slot 0 also brings both keys' scales (so that they arrive
+// early); with block scales each chunk brings its own.  The converter reloads each part right
+// after it has converted that part of the current tile (see converter_role).
 template <int S0, int S1, bool BS>
 __device__ __forceinline__ void fetch_own_part(const DecodeParams& p, const TilePtrs& T, int c, int t, RawTile& R) {
   const int q = conv_q(t);
   R.own_ok = T.own_ok;
+  if (!BS && S0 == 0 && T.oth_ok) R.sp[0] = __ldg(p.scales + T.ps);
   if (T.own_ok) {
     const uint8_t* ov = p.blocks + static_cast<size_t>(T.ov) * HEAD_DIM;
     if (!BS && S0 == 0) R.so[0] = __ldg(p.scales + T.os);
@@ -400,7 +440,6 @@ __device__ __forceinline__ void fetch_oth(const DecodeParams& p, const TilePtrs&
   R.oth_ok = T.oth_ok;
   if (T.oth_ok) {
     const uint8_t* pv = p.blocks + static_cast<size_t>(T.pv) * HEAD_DIM;
-    if (!BS) R.sp[0] = __ldg(p.scales + T.ps);
 #pragma unroll
     for (int k = 0; k < 2; ++k) {
       const int jc = q + 8 * k;                              // chunk index within D_c (0..15)
@@ -464,21 +503,26 @@ __device__ __forceinline__ void store_tile(int c, int t, const RawTile& R, uint3
 }
 
 // The decode's converter writes the two operands of a tile at different times: the K half as soon
-// as its buffer is free (store_k), the V operand once P.V two tiles back has finished (store_v).
-// store_k keeps the two chunks of the own key that also belong to the V operand (slots 3 and 4:
-// V chunks q and q + 8) so that store_v need not convert them again; they come last so that they
-// occupy registers only once the other chunks are done.
-template <bool BS>
-__device__ __forceinline__ void store_k(int c, int t, const RawTile& R, uint32_t sk, uint32_t (&keep0)[8],
-                                        uint32_t (&keep1)[8]) {
+// as its buffer is free (store_k_part), the V operand once P.V two tiles back has finished
+// (store_v).  store_k_part converts own-key slots [S0, S1); it keeps the two chunks that also
+// belong to the V operand (slots 3 and 4: V chunks q and q + 8) so that store_v need not convert
+// them again.  The tile's flags and per-token scales come as arguments because the registers of
+// R are being refilled with the next tile while this one is converted.
+template <int S0, int S1, bool BS, bool FOLD>
+__device__ __forceinline__ void store_k_part(int c, int t, const RawTile& R, bool own_ok, float s_own, uint32_t sk,
+                                             uint32_t (&keep0)[8], uint32_t (&keep1)[8]) {
   const int row = conv_row(t), q = conv_q(t);
 #pragma unroll
-  for (int sl = 0; sl < 5; ++sl) {
+  for (int sl = S0; sl < S1; ++sl) {
     const int qq = q + 8 * own_k(sl, c);
     if (qq >= 36) continue;
     uint32_t w[8];
-    if (R.own_ok) {
-      dequant16(R.own[sl], R.so[BS ? sl : 0], w);
+    if (own_ok) {
+      if (FOLD) {
+        exact16(R.own[sl], w);
+      } else {
+        dequant16(R.own[sl], BS ? R.so[sl] : s_own, w);
+      }
     } else {
 #pragma unroll
       for (int x = 0; x < 8; ++x) w[x] = 0u;
@@ -495,9 +539,9 @@ __device__ __forceinline__ void store_k(int c, int t, const RawTile& R, uint32_t
   }
 }
 
-template <bool BS>
-__device__ __forceinline__ void store_v(int c, int t, const RawTile& R, const uint32_t (&keep0)[8],
-                                        const uint32_t (&keep1)[8], uint32_t sv) {
+template <bool BS, bool FOLD>
+__device__ __forceinline__ void store_v(int c, int t, const RawTile& R, bool oth_ok, float s_oth,
+                                        const uint32_t (&keep0)[8], const uint32_t (&keep1)[8], uint32_t sv) {
   const int row = conv_row(t), q = conv_q(t);
   const int vrow_own = HALF_BN * c + row;
   const int vrow_oth = HALF_BN * (1 - c) + row;
@@ -507,8 +551,12 @@ __device__ __forceinline__ void store_v(int c, int t, const RawTile& R, const ui
   for (int k = 0; k < 2; ++k) {
     const int jc = q + 8 * k;
     uint32_t w[8];
-    if (R.oth_ok) {
-      dequant16(R.oth[k], R.sp[BS ? k : 0], w);
+    if (oth_ok) {
+      if (FOLD) {
+        exact16(R.oth[k], w);
+      } else {
+        dequant16(R.oth[k], BS ? R.sp[k] : s_oth, w);
+      }
     } else {
 #pragma unroll
       for (int x = 0; x < 8; ++x) w[x] = 0u;
@@ -584,14 +632,19 @@ struct TileCursor {
 
 // =============================================================================================
 // converter role (warps 0-7); the same code in both CTAs of the pair (c = rank).
-// Software pipeline over the tile sequence: while tile g is converted, the FP8 bytes of tile g+1 are
-// in flight and the page-table entries of tile g+2 are being read.  Buffers alternate by tile
-// parity; the K half of tile g waits for Q.K^T(g-2) (S_FULL), the V operand for P.V(g-2).
-// Returns early (with the abort flag set by the failing wait) when a wait gives up.
+// Software pipeline over the tile sequence with one set of tile registers R: each part of R (own-key
+// slots 0-2, own-key slots 3-4, other-key chunks) is refilled with tile g+1's bytes right after tile
+// g's copy of that part has been converted, so every load has a whole tile period to arrive and no
+// register is copied between tiles.  The page-table entries of tile g+2 are read meanwhile.
+// Buffers alternate by tile parity; the K half of tile g waits for Q.K^T(g-2) (S_FULL), the V
+// operand for P.V(g-2).  Returns early (with the abort flag set by the failing wait) when a wait
+// gives up.
 // =============================================================================================
-template <bool BS>
+template <int MODE>
 __device__ __forceinline__ void converter_role(const DecodeParams& p, int k, uint32_t base, int lane,
                                                volatile uint32_t* abort, uint32_t peer_abort, uint32_t c) {
+  constexpr bool BS = MODE == SCALE_BLOCK;
+  constexpr bool FOLD = MODE == SCALE_FOLD;
   const int C = static_cast<int>(c);
   const int t = threadIdx.x;
 #define BAR(i) (base + SBAR + 8u * (i))
@@ -603,12 +656,12 @@ __device__ __forceinline__ void converter_role(const DecodeParams& p, int k, uin
   if (!cur.valid) return;
   TileInfo n1 = ts.take(p);
   TileInfo n2 = ts.take(p);
-  RawTile ra, rb;
+  RawTile R;
   bool bad = false;
   {
     const TilePtrs t0 = lut_finish(p, lut_issue(p, C, t, item_b(p, cur.item), cur.nvis, cur.j), bad);
     if (bad) raise_status(p.status, STATUS_BOUNDS);
-    fetch<BS>(p, t0, C, t, ra);
+    fetch<BS>(p, t0, C, t, R);
   }
   TilePtrs t1{};
   if (n1.valid) {
@@ -616,58 +669,63 @@ __device__ __forceinline__ void converter_role(const DecodeParams& p, int k, uin
     if (bad) raise_status(p.status, STATUS_BOUNDS);
   }
   uint32_t g = 0;
-  // One tile: convert RCUR while RNXT (the next tile) is being fetched.
-#define MLA_CONV_STEP(RCUR, RNXT)                                                                        \
-  {                                                                                                      \
-    const uint32_t kb = g & 1, free_par = ((g >> 1) & 1) ^ 1;                                           \
-    MLA_WAIT_RET(BAR(B_S_FULL + kb), free_par);                                                          \
-    if (t == 0) MLA_TRACE_EV(g, 1);                                                                      \
-    if (t == 224) MLA_TRACE_EV(g, 26);                                                                   \
-    if (n1.valid) fetch_own_part<0, 3, BS>(p, t1, C, t, RNXT);                                                          \
-    if (t == 0) MLA_TRACE_EV(g, 16);                                                                     \
-    uint32_t keep0[8], keep1[8];                                                                         \
-    store_k<BS>(C, t, RCUR, base + SK0 + kb * SK_STRIDE, keep0, keep1);                                      \
-    if (n1.valid) {                                                                                     \
-      fetch_own_part<3, 5, BS>(p, t1, C, t, RNXT);                                                           \
-      fetch_oth<BS>(p, t1, C, t, RNXT);                                                                      \
-    }                                                          \
-    LutVals v2{};                                                                                        \
-    if (n2.valid) v2 = lut_issue(p, C, t, item_b(p, n2.item), n2.nvis, n2.j);                         \
-    if (t == 0) MLA_TRACE_EV(g, 4);                                                                      \
-    if (t == 224) MLA_TRACE_EV(g, 27);                                                                   \
-    ptx::fence_proxy_async_smem();                                                                       \
-    __syncwarp();                                                                                        \
-    if (lane == 0) ptx::mbar_arrive_cluster(k_full0 + 8u * kb);                                          \
-    if (t == 0) MLA_TRACE_EV(g, 5);                                                                      \
-    if (t == 224) MLA_TRACE_EV(g, 28);                                                                   \
-    MLA_WAIT_RET(BAR(B_PV_DONE + kb), free_par);                                                         \
-    if (t == 0) MLA_TRACE_EV(g, 6);                                                                      \
-    if (t == 224) MLA_TRACE_EV(g, 29);                                                                   \
-    store_v<BS>(C, t, RCUR, keep0, keep1, base + SV0 + kb * SV_STRIDE);                                      \
-    ptx::fence_proxy_async_smem();                                                                       \
-    __syncwarp();                                                                                        \
-    if (lane == 0) ptx::mbar_arrive_cluster(v_full0 + 8u * kb);                                          \
-    if (t == 0) MLA_TRACE_EV(g, 2);                                                                      \
-    if (t == 224) MLA_TRACE_EV(g, 30);                                                                   \
-    if (n2.valid) {                                                                                      \
-      t1 = lut_finish(p, v2, bad);                                                                       \
-      if (bad) raise_status(p.status, STATUS_BOUNDS);                                                    \
-    }                                                                                                    \
-    if (t == 0) MLA_TRACE_EV(g, 7);                                                                      \
-    if (t == 224) MLA_TRACE_EV(g, 31);                                                                   \
-    ++g;                                                                                                 \
-  }
-  // Rolled loop (one copy of the step keeps the hot code small): the next tile's bytes move from
-  // rb to ra at the end of a step, when they have normally arrived.
+  // Rolled loop (one copy of the step keeps the hot code small).
   while (true) {
-    MLA_CONV_STEP(ra, rb)
+    const uint32_t kb = g & 1, free_par = ((g >> 1) & 1) ^ 1;
+    MLA_WAIT_RET(BAR(B_S_FULL + kb), free_par);
+    if (t == 0) MLA_TRACE_EV(g, 1);
+    if (t == 224) MLA_TRACE_EV(g, 26);
+    // tile g's flags and per-token scales (R is refilled with tile g+1 below)
+    const bool own_ok = R.own_ok, oth_ok = R.oth_ok;
+    const float s_own = R.so[0], s_oth = R.sp[0];
+    if (FOLD) {
+      // the tile's 64 per-token scales for the softmax (0 for keys not read)
+      if (conv_q(t) == 0) {
+        const uint32_t sa = base + SSC + (g & 3) * SSC_STRIDE + 4 * conv_row(t);
+        ptx::st_shared_f32(sa + 4 * HALF_BN * C, own_ok ? s_own : 0.f);
+        ptx::st_shared_f32(sa + 4 * HALF_BN * (1 - C), oth_ok ? s_oth : 0.f);
+      }
+      __syncwarp();
+      if (lane == 0) ptx::mbar_arrive(BAR(B_SC_FULL + (g & 3)));
+    }
+    uint32_t keep0[8], keep1[8];
+    const uint32_t sk = base + SK0 + kb * SK_STRIDE;
+    store_k_part<0, 3, BS, FOLD>(C, t, R, own_ok, s_own, sk, keep0, keep1);
+    if (n1.valid) fetch_own_part<0, 3, BS>(p, t1, C, t, R);
+    if (t == 0) MLA_TRACE_EV(g, 16);
+    store_k_part<3, 5, BS, FOLD>(C, t, R, own_ok, s_own, sk, keep0, keep1);
+    if (n1.valid) fetch_own_part<3, 5, BS>(p, t1, C, t, R);
+    LutVals v2{};
+    if (n2.valid) v2 = lut_issue(p, C, t, item_b(p, n2.item), n2.nvis, n2.j);
+    if (t == 0) MLA_TRACE_EV(g, 4);
+    if (t == 224) MLA_TRACE_EV(g, 27);
+    ptx::fence_proxy_async_smem();
+    __syncwarp();
+    if (lane == 0) ptx::mbar_arrive_cluster(k_full0 + 8u * kb);
+    if (t == 0) MLA_TRACE_EV(g, 5);
+    if (t == 224) MLA_TRACE_EV(g, 28);
+    MLA_WAIT_RET(BAR(B_PV_DONE + kb), free_par);
+    if (t == 0) MLA_TRACE_EV(g, 6);
+    if (t == 224) MLA_TRACE_EV(g, 29);
+    store_v<BS, FOLD>(C, t, R, oth_ok, s_oth, keep0, keep1, base + SV0 + kb * SV_STRIDE);
+    ptx::fence_proxy_async_smem();
+    __syncwarp();
+    if (lane == 0) ptx::mbar_arrive_cluster(v_full0 + 8u * kb);
+    if (t == 0) MLA_TRACE_EV(g, 2);
+    if (t == 224) MLA_TRACE_EV(g, 30);
+    if (n1.valid) fetch_oth<BS>(p, t1, C, t, R);
+    if (n2.valid) {
+      t1 = lut_finish(p, v2, bad);
+      if (bad) raise_status(p.status, STATUS_BOUNDS);
+    }
+    if (t == 0) MLA_TRACE_EV(g, 7);
+    if (t == 224) MLA_TRACE_EV(g, 31);
+    ++g;
     if (!n1.valid) break;
-    ra = rb;
     cur = n1;
     n1 = n2;
     n2 = ts.take(p);
   }
-#undef MLA_CONV_STEP
 #undef MLA_WAIT_RET
 #undef BAR
 }
@@ -675,13 +733,19 @@ __device__ __forceinline__ void converter_role(const DecodeParams& p, int k, uin
 // =============================================================================================
 // decode kernel
 // =============================================================================================
-// BS: block scales (head_dim_granularity > 1) instead of one scale per token.
-template <bool BS>
+// MODE: a ScaleMode (per-token scales, block scales, or per-token scales folded into S and P).
+template <int MODE>
 __global__ void __launch_bounds__(NUM_THREADS, 1) mla_decode_kernel(const __grid_constant__ DecodeParams p) {
+  constexpr bool FOLD = MODE == SCALE_FOLD;
   if (threadIdx.x == 0) MLA_MARK_MIN(1);
   ptx::griddep_launch_dependents();   // the combine kernel may start launching (it waits for this grid)
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  if (FOLD && static_cast<uint32_t>(smem - smem_raw) > SMEM_FOLD_MAX_PAD) {
+    // every CTA of the launch sees the same base, so all of them leave here together
+    if (threadIdx.x == 0) raise_status(p.status, STATUS_LAYOUT);
+    return;
+  }
   const uint32_t base = ptx::smem_u32(smem);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const uint32_t c = ptx::cluster_ctarank();
@@ -709,6 +773,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) mla_decode_kernel(const __grid
     ptx::mbar_init(BAR(B_DRAIN), 2);
     ptx::mbar_init(BAR(B_REDL), 4);
     ptx::mbar_init(BAR(B_EXIT), 1);
+    for (uint32_t i = 0; i < 4; ++i) ptx::mbar_init(BAR(B_SC_FULL + i), CONV_WARPS);
     *abort = 0u;
     ptx::fence_mbar_init();
   }
@@ -732,7 +797,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) mla_decode_kernel(const __grid
 
   if (warp < CONV_WARPS) {
     // ------------------------------------------------------------------ converter
-    converter_role<BS>(p, k, base, lane, abort, peer_abort, c);
+    converter_role<MODE>(p, k, base, lane, abort, peer_abort, c);
   } else if (warp < SM_WARP0 + 4) {
     // ------------------------------------------------------------------ softmax / epilogue
     const int t = threadIdx.x - 32 * SM_WARP0;
@@ -751,6 +816,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) mla_decode_kernel(const __grid
       for (int j = u.tb; j < u.te; ++j, ++g) {
         const uint32_t sb = g & 1;
         MLA_WAIT_WARP(BAR(B_S_FULL + sb), (g >> 1) & 1);
+        if (FOLD) MLA_WAIT_WARP(BAR(B_SC_FULL + (g & 3)), (g >> 2) & 1);
         if (t == 0) MLA_TRACE_EV(g, 8);
         ptx::tc_fence_after();
         float x[32];
@@ -768,10 +834,28 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) mla_decode_kernel(const __grid
         if (t == 0) MLA_TRACE_EV(g, 9);
         const int nv = min(BN, u.nvis - j * BN) - HALF_BN * hh;   // valid keys in this lane's half
         float mt = -INFINITY;
+        // scale-folding mode: the scales of this lane's 32 keys (written before K_FULL of this
+        // tile; buffer g & 3 is rewritten only after this warp has finished tile g)
+        const uint32_t sc_addr = base + SSC + (g & 3) * SSC_STRIDE + 4 * HALF_BN * hh;
+        if (FOLD) {
 #pragma unroll
-        for (int q = 0; q < 32; ++q) {
-          x[q] = (q < nv) ? x[q] * p.scale_log2 : -INFINITY;
-          mt = fmaxf(mt, x[q]);
+          for (int v = 0; v < 8; ++v) {
+            const uint4 s4 = ptx::ld_shared_v4(sc_addr + 16 * v);
+            const float sc[4] = {__uint_as_float(s4.x), __uint_as_float(s4.y), __uint_as_float(s4.z),
+                                 __uint_as_float(s4.w)};
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+              const int q = 4 * v + e;
+              x[q] = (q < nv) ? x[q] * (p.scale_log2 * sc[e]) : -INFINITY;
+              mt = fmaxf(mt, x[q]);
+            }
+          }
+        } else {
+#pragma unroll
+          for (int q = 0; q < 32; ++q) {
+            x[q] = (q < nv) ? x[q] * p.scale_log2 : -INFINITY;
+            mt = fmaxf(mt, x[q]);
+          }
         }
         // the other half of this head row lives in lane t ^ 64 (another warp of this warpgroup)
         red_max[sb * 128 + t] = mt;
@@ -790,12 +874,28 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) mla_decode_kernel(const __grid
         }
         float lsum = 0.f;
         uint32_t pw[16];
+        if (FOLD) {
+          // l sums the weights; the P operand carries weight * s_t
 #pragma unroll
-        for (int q = 0; q < 16; ++q) {
-          const float p0 = ptx::ex2_approx(x[2 * q] - m_ref);
-          const float p1 = ptx::ex2_approx(x[2 * q + 1] - m_ref);
-          lsum += p0 + p1;
-          pw[q] = ptx::pack_bf16x2(p0, p1);
+          for (int v = 0; v < 8; ++v) {
+            const uint4 s4 = ptx::ld_shared_v4(sc_addr + 16 * v);
+            const float p0 = ptx::ex2_approx(x[4 * v] - m_ref);
+            const float p1 = ptx::ex2_approx(x[4 * v + 1] - m_ref);
+            const float p2 = ptx::ex2_approx(x[4 * v + 2] - m_ref);
+            const float p3 = ptx::ex2_approx(x[4 * v + 3] - m_ref);
+            lsum += p0 + p1;                // the per-token mode's summation order
+            lsum += p2 + p3;
+            pw[2 * v] = ptx::pack_bf16x2(p0 * __uint_as_float(s4.x), p1 * __uint_as_float(s4.y));
+            pw[2 * v + 1] = ptx::pack_bf16x2(p2 * __uint_as_float(s4.z), p3 * __uint_as_float(s4.w));
+          }
+        } else {
+#pragma unroll
+          for (int q = 0; q < 16; ++q) {
+            const float p0 = ptx::ex2_approx(x[2 * q] - m_ref);
+            const float p1 = ptx::ex2_approx(x[2 * q + 1] - m_ref);
+            lsum += p0 + p1;
+            pw[q] = ptx::pack_bf16x2(p0, p1);
+          }
         }
         l += lsum;
         if (t == 0) MLA_TRACE_EV(g, 11);

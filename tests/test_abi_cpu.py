@@ -66,6 +66,23 @@ def test_host_validation_rejects_null_and_misaligned(lib):
     assert _call(lib, _shape(), T=0) == 1
 
 
+def test_scale_folded_host_validation(lib):
+    """The scale-folding entry shares the decode's checks and takes only one scale per token; all of
+    these fail on the host before anything is launched."""
+    def fold(shape, **kw):
+        a = dict(q=FAKE, blocks=FAKE, scales=FAKE, lens=FAKE, lut=FAKE, T=1, maxc=64, layer=0, out=FAKE)
+        a.update(kw)
+        return lib.mla_decode_paged_fp8_scale_folded(a["q"], a["blocks"], a["scales"], a["lens"], a["lut"], None,
+                                                     a["T"], a["maxc"], a["layer"], 0.07,
+                                                     ctypes.byref(shape) if shape is not None else None,
+                                                     a["out"], None, None)
+    assert fold(None) == 1
+    assert fold(_shape(), blocks=None) == 1
+    assert fold(_shape(head_dim=512)) == 2
+    assert fold(_shape(head_dim_granularity=9)) == 2
+    assert "one scale per token" in lib.mla_last_error_string().decode()
+
+
 def _store(lib, shape, latent=FAKE, lens=FAKE, lut=FAKE, slut=None, T=1, layer=0, blocks=FAKE, scales=FAKE):
     return lib.mla_kv_store_fp8(latent, lens, lut, slut, T, layer,
                                 ctypes.byref(shape) if shape is not None else None, blocks, scales, None)
