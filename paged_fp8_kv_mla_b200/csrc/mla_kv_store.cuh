@@ -12,8 +12,8 @@
 //
 // Eight lanes per token (a warp stores four tokens): lane k of a token's group reads 16-byte chunks
 // k, k + 8, ..., k + 64 of the 1152-byte bf16 row (each step of the group reads 128 contiguous
-// bytes), the group reduces |x| with shuffles, and each lane writes the 8 code bytes of each of its
-// nine chunks.  HBM-bound: 1152 B read and 580 B written per token.
+// bytes), the group reduces max |x| with shuffles, and each lane writes the 8 code bytes of each of
+// its nine chunks.  HBM-bound: 1152 B read and 580 B written per token.
 #pragma once
 #include <cstdint>
 #include "mla_kernels.cuh"
@@ -45,47 +45,49 @@ __device__ __forceinline__ uint32_t e4m3x2_rn_sat(float lo, float hi) {
 __device__ __forceinline__ float bf16_lo(uint32_t w) { return __uint_as_float(w << 16); }
 __device__ __forceinline__ float bf16_hi(uint32_t w) { return __uint_as_float(w & 0xFFFF0000u); }
 
-// The quotient x / s is only needed to e4m3 precision.  With r = RN(1 / s), y = RN(x * r) is
-// within 2.5 fp32 ulps of RN(x / s) (two roundings of relative size 2^-24 each, plus the half ulp
-// of RN(x / s)), so both round to the same e4m3 code unless they straddle a rounding midpoint of
-// e4m3: a value whose low 20 mantissa bits are 0x80000 in the normal range (e4m3 keeps 3 of the
-// 23 bits), or any value in the subnormal range |y| < 2^-6 (steps of 2^-9).  needs_exact flags y
-// within 4 ulps of a midpoint or in that range; only those values take the IEEE division.
-__device__ __forceinline__ bool needs_exact(float y) {
-  const uint32_t u = __float_as_uint(y);
-  return ((u & 0xFFFFFu) - 0x7FFFCu) <= 8u || (fabsf(y) < 0.015625f && y != 0.f);
-}
+// The quotient RN(x / s) by one correction of the reciprocal product (P. Markstein, "Computation of
+// elementary functions on the IBM RISC System/6000 processor", IBM J. Res. Dev. 34(1), 1990):
+// with r = RN(1 / s) and y0 = RN(x * r), the remainder x - y0 * s is computed by one fma and
+// y = RN(y0 + (x - y0 * s) * r) by another.  Checked in exact arithmetic before use: for bf16 x
+// with |x| >= 2^-100 and fp32 s, y equals the IEEE quotient bit for bit (27 M cases); smaller |x|
+// (where the remainder can fall into the subnormal range) only reach e4m3 code 0, and for every
+// s >= 2^-90 the e4m3 code of y equals the code of RN(x / s) (30 M cases, zeros of both signs
+// included).  The remainder is formed as -(y0 * s - x) so that a zero keeps its sign.  Tokens whose
+// scale is below 2^-90 take the IEEE division.
+constexpr float KVS_FAST_MIN_SCALE = 8.077935669463161e-28f;   // 2^-90
 
-// 8 bf16 (one 16-byte chunk) / s -> 8 e4m3 codes; r = RN(1 / s).
+// 8 bf16 (one 16-byte chunk) / s -> 8 e4m3 codes; r = RN(1 / s), s >= 2^-90.
 __device__ __forceinline__ uint2 quant8(uint4 v, float s, float r) {
   const uint32_t in[4] = {v.x, v.y, v.z, v.w};
-  float y[8];
-  bool slow = false;
-#pragma unroll
-  for (int k = 0; k < 4; ++k) {
-    y[2 * k] = bf16_lo(in[k]) * r;
-    y[2 * k + 1] = bf16_hi(in[k]) * r;
-  }
-#pragma unroll
-  for (int j = 0; j < 8; ++j) slow |= needs_exact(y[j]);
-  if (slow) {
-#pragma unroll
-    for (int j = 0; j < 8; ++j) {
-      const float x = (j & 1) ? bf16_hi(in[j >> 1]) : bf16_lo(in[j >> 1]);
-      if (needs_exact(y[j])) y[j] = __fdiv_rn(x, s);
-    }
-  }
+  const float2 ss = make_float2(s, s), rr = make_float2(r, r);
   uint32_t c[4];
 #pragma unroll
-  for (int k = 0; k < 4; ++k) c[k] = e4m3x2_rn_sat(y[2 * k], y[2 * k + 1]);
+  for (int k = 0; k < 4; ++k) {
+    const float2 x = make_float2(bf16_lo(in[k]), bf16_hi(in[k]));
+    const float2 y0 = __fmul2_rn(x, rr);
+    const float2 t = __ffma2_rn(y0, ss, make_float2(-x.x, -x.y));          // y0 * s - x
+    const float2 y = __ffma2_rn(make_float2(-t.x, -t.y), rr, y0);          // y0 + (x - y0 * s) * r
+    c[k] = e4m3x2_rn_sat(y.x, y.y);
+  }
   return make_uint2(c[0] | (c[1] << 16), c[2] | (c[3] << 16));
 }
 
-__device__ __forceinline__ float absmax8(uint4 v, float m) {
+// The same with the IEEE division (tokens with a scale below 2^-90).
+__device__ __forceinline__ uint2 quant8_div(uint4 v, float s) {
   const uint32_t in[4] = {v.x, v.y, v.z, v.w};
+  uint32_t c[4];
 #pragma unroll
-  for (int k = 0; k < 4; ++k) m = fmaxf(m, fmaxf(fabsf(bf16_lo(in[k])), fabsf(bf16_hi(in[k]))));
-  return m;
+  for (int k = 0; k < 4; ++k) c[k] = e4m3x2_rn_sat(__fdiv_rn(bf16_lo(in[k]), s), __fdiv_rn(bf16_hi(in[k]), s));
+  return make_uint2(c[0] | (c[1] << 16), c[2] | (c[3] << 16));
+}
+
+// max |x| over a chunk as bf16 bit patterns: for non-NaN values the magnitude bits order like the
+// magnitudes, so a per-halfword unsigned max of (bits & 0x7FFF) is the bf16 of max |x|.
+__device__ __forceinline__ uint32_t absmax8_bits(uint4 v, uint32_t m2) {
+  m2 = __vmaxu2(m2, v.x & 0x7FFF7FFFu);
+  m2 = __vmaxu2(m2, v.y & 0x7FFF7FFFu);
+  m2 = __vmaxu2(m2, v.z & 0x7FFF7FFFu);
+  return __vmaxu2(m2, v.w & 0x7FFF7FFFu);
 }
 
 constexpr int KVS_LANES = 8;                       // lanes per token
@@ -116,23 +118,29 @@ __global__ void __launch_bounds__(32 * KVS_WARPS) mla_kv_store_kernel(const __gr
     if (!ok && k == 0) atomicOr(p.status, 1u);
   }
   uint4 v[KVS_CHUNKS];
-  float m = 0.f;
+  uint32_t m2 = 0;
   if (ok) {
     const uint4* src = reinterpret_cast<const uint4*>(p.latent + static_cast<size_t>(tok) * 576);
 #pragma unroll
     for (int j = 0; j < KVS_CHUNKS; ++j) v[j] = src[k + KVS_LANES * j];
 #pragma unroll
-    for (int j = 0; j < KVS_CHUNKS; ++j) m = absmax8(v[j], m);
+    for (int j = 0; j < KVS_CHUNKS; ++j) m2 = absmax8_bits(v[j], m2);
   }
-  // reduce over the token's 8 lanes (all 32 lanes take part; dead tokens carry m = 0)
+  // reduce over the token's 8 lanes (all 32 lanes take part; dead tokens carry 0)
 #pragma unroll
-  for (int o = KVS_LANES / 2; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+  for (int o = KVS_LANES / 2; o > 0; o >>= 1) m2 = __vmaxu2(m2, __shfl_xor_sync(0xffffffffu, m2, o));
   if (!ok) return;
+  const float m = __uint_as_float(max(m2 & 0xFFFFu, m2 >> 16) << 16);
   const float s = m > 0.f ? __fdiv_rn(m, 448.f) : 1.f;
-  const float r = __frcp_rn(s);
   uint2* dst = reinterpret_cast<uint2*>(p.blocks + row * 576);
+  if (s >= KVS_FAST_MIN_SCALE) {
+    const float r = __frcp_rn(s);
 #pragma unroll
-  for (int j = 0; j < KVS_CHUNKS; ++j) dst[k + KVS_LANES * j] = quant8(v[j], s, r);
+    for (int j = 0; j < KVS_CHUNKS; ++j) dst[k + KVS_LANES * j] = quant8(v[j], s, r);
+  } else {
+#pragma unroll
+    for (int j = 0; j < KVS_CHUNKS; ++j) dst[k + KVS_LANES * j] = quant8_div(v[j], s);
+  }
   if (k == 0) p.scales[srow] = s;
 }
 

@@ -122,6 +122,32 @@ def test_store_special_rows():
     _check_bitexact(blocks, scales, ref_b, ref_s)
 
 
+def test_store_rows_around_the_division_switch_and_signed_zeros():
+    """Per-token scales just above and below 2^-90 (the kernel's switch between the corrected
+    reciprocal product and the IEEE division), rows of negative zeros, and zeros of both signs
+    inside a normal row: all bit-exact against the oracle."""
+    inp = _custom(B=1, T=8, P=16, lengths=(3,))
+    blocks, scales = _poison_new_rows(inp)
+    g = torch.Generator().manual_seed(5)
+    x = torch.randn((1, 8, 576), generator=g)
+    edge = 448.0 * 2.0 ** -90
+    for i, f in enumerate((1.02, 1.0, 0.98, 0.5)):
+        row = x[0, i] / x[0, i].abs().max() * (edge * f)
+        x[0, i] = row
+    x[0, 4] = -0.0
+    x[0, 5, ::3] = -0.0
+    x[0, 5, 1::3] = 0.0
+    x[0, 6] = torch.randn(576, generator=g) * 2.0 ** -100
+    x[0, 6, 0] = 1.0                                          # tiny values beside a normal maximum
+    x[0, 7] = torch.randn(576, generator=g) * 1e30
+    lat = x.to(torch.bfloat16).cuda()
+    ref_b, ref_s = _oracle_store(inp, lat, blocks, scales)
+    M.kv_store(lat, inp.cache_lengths, inp.lookup_table, inp.scales_lookup_table, inp.layer_idx, blocks, scales)
+    torch.cuda.synchronize()
+    assert M.device_status() == 0
+    _check_bitexact(blocks, scales, ref_b, ref_s)
+
+
 def test_store_rows_where_reciprocal_and_division_differ():
     """Rows on which x * RN(1/s) and RN(x / s) round to different e4m3 codes (found by a seeded
     search): the kernel's fast path must fall back to the division exactly there."""
