@@ -557,7 +557,7 @@ mla_status_t mla_debug_marks(unsigned long long* out8, int reset) {
   MLA_CUDA(cudaDeviceSynchronize());
   MLA_CUDA(cudaMemcpyFromSymbol(out8, mla::g_trace_marks, 8 * sizeof(unsigned long long)));
   if (reset) {
-    const unsigned long long init[8] = {0ull, ~0ull, 0ull, ~0ull, 0ull, 0ull, 0ull, 0ull};
+    const unsigned long long init[8] = {0ull, ~0ull, 0ull, ~0ull, 0ull, ~0ull, 0ull, 0ull};
     MLA_CUDA(cudaMemcpyToSymbol(mla::g_trace_marks, init, sizeof(init)));
   }
   return MLA_OK;

@@ -218,7 +218,8 @@ __device__ __forceinline__ void raise_status(unsigned int* status, unsigned bits
 // trace[2 * TRACE_TILES * TRACE_EVENTS + 4 * blockIdx.x + {0, 1, 2}].
 #ifdef MLA_TRACE
 // Trace builds: %globaltimer marks of one decode call: [0] plan end, [1] first decode CTA entry,
-// [2] last decode CTA exit, [3] first combine CTA entry, [4] last combine CTA exit.
+// [2] last decode CTA exit, [3] first combine CTA past its grid-dependency wait, [4] last combine
+// warp done, [5] first combine CTA entry.
 __device__ unsigned long long g_trace_marks[8];
 #define MLA_MARK_MIN(i) atomicMin(&g_trace_marks[i], static_cast<unsigned long long>(ptx::globaltimer()))
 #define MLA_MARK_MAX(i) atomicMax(&g_trace_marks[i], static_cast<unsigned long long>(ptx::globaltimer()))
@@ -1240,6 +1241,7 @@ constexpr int COMBINE_HEADS = 8;
 
 __global__ void __launch_bounds__(32 * COMBINE_HEADS)
 mla_combine_kernel(const __grid_constant__ DecodeParams p) {
+  if (threadIdx.x == 0) MLA_MARK_MIN(5);
   ptx::griddep_wait();   // the decode kernel's partials are complete and visible
   if (threadIdx.x == 0) MLA_MARK_MIN(3);
   const int per_item = MROWS / COMBINE_HEADS;
@@ -1256,27 +1258,30 @@ mla_combine_kernel(const __grid_constant__ DecodeParams p) {
   const int g = it - bi * p.G, b = static_cast<int>(p.divT.div(bi)), i = bi - b * p.T;
   const int head = g * MROWS + h;
   if (head >= p.H) return;
-  float mx = -INFINITY;
-  for (int kk = k0; kk <= k1; ++kk) {
-    const int slot = 2 * kk + (max(s, kk * tpc) == kk * tpc ? 0 : 1);
-    mx = fmaxf(mx, p.part_lse[slot * MROWS + h]);
-  }
+  // one pass over the pieces, merging with a running maximum (each piece's LSE and data are loaded
+  // together, so the pieces' loads overlap)
+  float mx = -INFINITY, tot = 0.f;
   float4 acc[4];
 #pragma unroll
   for (int j = 0; j < 4; ++j) acc[j] = make_float4(0.f, 0.f, 0.f, 0.f);
-  float tot = 0.f;
+#pragma unroll 2
   for (int kk = k0; kk <= k1; ++kk) {
     const int slot = 2 * kk + (max(s, kk * tpc) == kk * tpc ? 0 : 1);
-    const float wgt = __expf(p.part_lse[slot * MROWS + h] - mx);
-    tot += wgt;
+    const float l = p.part_lse[slot * MROWS + h];
     const float4* src = reinterpret_cast<const float4*>(p.part_o + (static_cast<size_t>(slot) * MROWS + h) * V_DIM);
+    float4 v[4];
+#pragma unroll
+    for (int j = 0; j < 4; ++j) v[j] = src[j * 32 + lane];
+    const float mn = fmaxf(mx, l);
+    const float a = __expf(mx - mn), wgt = __expf(l - mn);   // a = 0 for the first piece
+    mx = mn;
+    tot = tot * a + wgt;
 #pragma unroll
     for (int j = 0; j < 4; ++j) {
-      const float4 v = src[j * 32 + lane];
-      acc[j].x += wgt * v.x;
-      acc[j].y += wgt * v.y;
-      acc[j].z += wgt * v.z;
-      acc[j].w += wgt * v.w;
+      acc[j].x = acc[j].x * a + wgt * v[j].x;
+      acc[j].y = acc[j].y * a + wgt * v[j].y;
+      acc[j].z = acc[j].z * a + wgt * v[j].z;
+      acc[j].w = acc[j].w * a + wgt * v[j].w;
     }
   }
   const float inv = 1.f / tot;
@@ -1289,6 +1294,7 @@ mla_combine_kernel(const __grid_constant__ DecodeParams p) {
     reinterpret_cast<uint2*>(dst)[j * 32 + lane] = o;
   }
   if (lane == 0 && p.lse) p.lse[(static_cast<size_t>(b) * p.T + i) * p.H + head] = mx + __logf(tot);
+  if (lane == 0) MLA_MARK_MAX(4);
 }
 
 // =============================================================================================
