@@ -211,6 +211,26 @@ mla_status_t mla_kv_store_fp8(
     const mla_paged_shape_t* shape, void* blocks, float* scales, cudaStream_t stream);
 
 /*
+ * mla_merge_lse_parts_bf16 -- the merge step of context parallelism (no counterpart on the
+ * reference pages): when every rank decodes a contiguous, page-aligned range of each request's
+ * keys (mla_decode_paged_fp8 on a page table that lists only those pages), the ranks' results are
+ * exchanged and merged here.  For each of `rows` rows (request, query token, head) and parts
+ * r = 0 .. num_parts - 1:
+ *     lse[row] = ln sum_r e^{lses[r][row]},   out[row] = sum_r e^{lses[r][row] - lse[row]} outs[r][row]
+ * which is the softmax attention over the union of the parts' keys.  A part with lse = -inf (no keys)
+ * is skipped; a row with no non-empty part gets out = 0 and lse = -inf.
+ *
+ *   outs   bf16 [num_parts, rows, 512], device, 16-byte aligned (each part's decode `out`)
+ *   lses   fp32 [num_parts, rows], device (each part's decode `lse`, natural log)
+ *   out    bf16 [rows, 512], device, 16-byte aligned, fully overwritten; may not alias outs
+ *   lse    fp32 [rows] or NULL
+ * Asynchronous on `stream`; rows = 0 is a no-op.  Errors: MLA_ERR_INVALID_ARG (NULL or misaligned
+ * pointers, num_parts < 1), MLA_ERR_CUDA.
+ */
+mla_status_t mla_merge_lse_parts_bf16(const void* outs, const float* lses, int32_t num_parts, int64_t rows,
+                                      void* out, float* lse, cudaStream_t stream);
+
+/*
  * mla_set_num_clusters -- test and tuning hook: fix the number of 2-CTA clusters
  * the decode splits the keys over (0 restores the default, one per resident
  * cluster slot of the device).  Process-wide.  Smaller values make fewer, longer

@@ -23,7 +23,7 @@ STATUS_NAMES = {0: "MLA_OK", 1: "MLA_ERR_INVALID_ARG", 2: "MLA_ERR_UNSUPPORTED",
 EXPORTED = ["mla_decode_paged_fp8", "mla_gather_dequant_bf16", "mla_set_num_clusters",
             "mla_get_num_clusters", "mla_last_error_string", "mla_get_device_status",
             "mla_release_workspace", "mla_version", "mla_set_timing_events", "mla_decode_paged_fp8_noalloc",
-            "mla_kv_store_fp8", "mla_decode_paged_fp8_scale_folded"]
+            "mla_kv_store_fp8", "mla_decode_paged_fp8_scale_folded", "mla_merge_lse_parts_bf16"]
 
 
 class MlaError(RuntimeError):
@@ -53,6 +53,8 @@ def load(path: str = LIB_PATH) -> ctypes.CDLL:
     lib.mla_decode_paged_fp8.argtypes = [vp, vp, vp, vp, vp, vp, u32, u32, u32, f32,
                                          ctypes.POINTER(PagedShape), vp, vp, vp]
     lib.mla_decode_paged_fp8.restype = ctypes.c_int
+    lib.mla_merge_lse_parts_bf16.argtypes = [vp, vp, ctypes.c_int32, ctypes.c_int64, vp, vp, vp]
+    lib.mla_merge_lse_parts_bf16.restype = ctypes.c_int
     lib.mla_decode_paged_fp8_scale_folded.argtypes = lib.mla_decode_paged_fp8.argtypes
     lib.mla_decode_paged_fp8_scale_folded.restype = ctypes.c_int
     lib.mla_decode_paged_fp8_noalloc.argtypes = [vp, vp, vp, vp, vp, vp, u32, u32, u32, f32,
@@ -164,6 +166,25 @@ def decode_noalloc(q, blocks, scales, cache_lengths, lookup_table, scales_lookup
                                           _ptr(lookup_table), _ptr(scales_lookup_table), int(max_prompt_length),
                                           int(max_cache_length), int(layer_idx), float(softmax_scale),
                                           ctypes.byref(shp), _ptr(out), _ptr(lse), _stream(stream))
+    _check(st)
+    return out, lse
+
+
+def merge_parts(outs, lses, out=None, lse=None, stream=None):
+    """mla_merge_lse_parts_bf16: outs bf16 [R, ..., 512] and lses fp32 [R, ...] (the parts' decode
+    results over disjoint key ranges) -> (out bf16 [..., 512], lse fp32 [...])."""
+    lib = load()
+    _contig(outs, lses)
+    R = outs.shape[0]
+    rows = lses[0].numel()
+    if outs.shape[:-1] != lses.shape or outs.shape[-1] != 512:
+        raise ValueError("outs must be [R, ..., 512] and lses [R, ...] with the same leading dims")
+    if out is None:
+        out = torch.empty(outs.shape[1:], dtype=torch.bfloat16, device=outs.device)
+    if lse is None:
+        lse = torch.empty(lses.shape[1:], dtype=torch.float32, device=lses.device)
+    _contig(out, lse)
+    st = lib.mla_merge_lse_parts_bf16(_ptr(outs), _ptr(lses), int(R), int(rows), _ptr(out), _ptr(lse), _stream(stream))
     _check(st)
     return out, lse
 

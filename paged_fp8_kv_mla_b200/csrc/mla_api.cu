@@ -12,6 +12,7 @@
 
 #include "mla_kernels.cuh"
 #include "mla_kv_store.cuh"
+#include "mla_merge.cuh"
 #include "mla_paged_fp8.h"
 
 namespace {
@@ -624,6 +625,25 @@ mla_status_t mla_decode_paged_fp8_noalloc(const void* q, const void* blocks, con
   p.scale_log2 = softmax_scale * 1.4426950408889634f;
 
   return launch_path(p, NC, cache_lengths, max_cache_length, stream, false);
+}
+
+mla_status_t mla_merge_lse_parts_bf16(const void* outs, const float* lses, int32_t num_parts, int64_t rows,
+                                      void* out, float* lse, cudaStream_t stream) {
+  if (num_parts < 1 || rows < 0) return fail(MLA_ERR_INVALID_ARG, "num_parts must be >= 1 and rows >= 0");
+  if (rows == 0) return MLA_OK;
+  if (!outs || !lses || !out) return fail(MLA_ERR_INVALID_ARG, "outs, lses and out must be non-NULL");
+  if (!aligned16(outs) || !aligned16(out)) return fail(MLA_ERR_INVALID_ARG, "outs and out must be 16-byte aligned");
+  if (rows > (1ll << 40) / num_parts) return fail(MLA_ERR_UNSUPPORTED, "too many rows");
+  int dev = 0;
+  MLA_CUDA(cudaGetDevice(&dev));
+  int sms = 0;
+  MLA_CUDA(cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev));
+  long long blocks = (rows + mla::MERGE_WARPS - 1) / mla::MERGE_WARPS;
+  if (blocks > 8ll * sms) blocks = 8ll * sms;
+  mla::mla_merge_parts_kernel<<<static_cast<unsigned>(blocks), 32 * mla::MERGE_WARPS, 0, stream>>>(
+      static_cast<const uint16_t*>(outs), lses, num_parts, static_cast<long long>(rows), static_cast<uint16_t*>(out), lse);
+  MLA_CUDA(cudaGetLastError());
+  return MLA_OK;
 }
 
 mla_status_t mla_get_device_status(cudaStream_t stream) {

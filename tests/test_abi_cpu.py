@@ -83,6 +83,15 @@ def test_scale_folded_host_validation(lib):
     assert "one scale per token" in lib.mla_last_error_string().decode()
 
 
+def test_merge_host_validation(lib):
+    """Argument checks of the LSE merge; none of these launches anything (rows = 0 is a no-op)."""
+    f = lib.mla_merge_lse_parts_bf16
+    assert f(FAKE, FAKE, 2, 0, FAKE, None, None) == 0
+    assert f(FAKE, FAKE, 0, 10, FAKE, None, None) == 1
+    assert f(None, FAKE, 2, 10, FAKE, None, None) == 1
+    assert f(FAKE, FAKE, 2, 10, ctypes.c_void_p(0x10004), None, None) == 1
+
+
 def _store(lib, shape, latent=FAKE, lens=FAKE, lut=FAKE, slut=None, T=1, layer=0, blocks=FAKE, scales=FAKE):
     return lib.mla_kv_store_fp8(latent, lens, lut, slut, T, layer,
                                 ctypes.byref(shape) if shape is not None else None, blocks, scales, None)
