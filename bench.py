@@ -134,6 +134,20 @@ class ClockSampler:
         return {"sm_mhz": sm[len(sm) // 2], "sm_max_mhz": mx, "reasons": reasons, "samples": len(rows)}
 
 
+def rank_seed(base_seed: int, rank: int) -> int:
+    """Each replica decodes its own batch (weak scaling): rank r draws its inputs from seed base + 7919 r."""
+    return base_seed + 7919 * rank
+
+
+def max_over_ranks(dist, values, device):
+    """Element-wise maximum of per-rank timings (ms) across the process group (one all_reduce)."""
+    if dist is None:
+        return [float(v) for v in values]
+    t = torch.tensor([float(v) for v in values], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return [float(x) for x in t.tolist()]
+
+
 def cpu_oracle_baseline(inp, budget_s, rank_requests=None, fold=False):
     """The float64 oracle, as it stands, on whole requests of the same workload until ~budget_s."""
     import numpy as np
@@ -334,7 +348,7 @@ def main():
     if fold:
         from dataclasses import replace
         cfg = replace(cfg, name=f"{cfg.name}_scale_folded")
-    seed = cfg.seed + 7919 * rank
+    seed = rank_seed(cfg.seed, rank)
     inp = W.make_inputs(cfg, device="cuda", seed=seed)
     kv_bytes = inp.kv_scale_bytes()
     flops = inp.flops()
@@ -431,16 +445,12 @@ def main():
         torch.cuda.synchronize()
         e2e_ms = sum(a.elapsed_time(b) for a, b in eev) / Ke
         if dist:
-            t = torch.tensor([e2e_ms], device="cuda")
-            dist.all_reduce(t, op=dist.ReduceOp.MAX)
-            e2e_ms = float(t.item())
+            e2e_ms = max_over_ranks(dist, [e2e_ms], "cuda")[0]
         e2e = {"value": kv_bytes * world / (e2e_ms * 1e-3) / 1e9, "unit": "GB/s", "h2d_bytes_per_step": h2d,
                "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms}
 
     if dist:
-        t = torch.tensor([step_ms, kern_ms], device="cuda")
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        step_ms, kern_ms = float(t[0].item()), float(t[1].item())
+        step_ms, kern_ms = max_over_ranks(dist, [step_ms, kern_ms], "cuda")
 
     peaks = load_peaks()
     gbs = kv_bytes * world / (step_ms * 1e-3) / 1e9
