@@ -181,8 +181,8 @@ mla_status_t mla_gather_dequant_bf16(
 /*
  * mla_kv_store_fp8 -- the KV-store step that produces the cache the decode reads: quantise the
  * step's new tokens' latent to e4m3 with one fp32 scale per token and scatter each row into its
- * page.  The quantiser is the pages' data recipe (per-token scale amax / 448, e4m3 round to
- * nearest with saturation); the placement is the page-table layout of
+ * page.  The quantiser is the per-token FP8 recipe that also generates the test workloads
+ * (scale amax / 448, e4m3 round to nearest with saturation); the placement is the page-table layout of
  * generic_get_paged_cache_with_scales.
  *
  * For new token i of request b, at position t = cache_lengths[b] + i (the step's tokens follow

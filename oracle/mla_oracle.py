@@ -27,9 +27,9 @@ What it computes, step by step, in the order the pages lay out the data:
    new tokens are already in the cache); query i of request b sees keys
    t <= cache_lengths[b] + i (causal among the new tokens).
 
-4. The KV-store step that produces this path's input (the data-generation
-   recipe of the pages' config 0: per-token scale f32(amax) / 448, e4m3 codes
-   with round-to-nearest and saturation).  For new token i of request b, at
+4. The KV-store step that produces this path's input (the per-token FP8
+   recipe that also generates the test workloads: scale f32(amax) / 448, e4m3
+   codes with round-to-nearest and saturation).  For new token i of request b, at
    position t = cache_lengths[b] + i (reading R1), with x the 576 bf16 values:
    scale = f32(max_d |x_d|) / 448 rounded to fp32 (1.0 for an all-zero row),
    code_d = e4m3_rn_sat(f32_rn(x_d / scale)), written to blocks[blk, 0,

@@ -23,7 +23,9 @@
 //   warps 0-7   converter: FP8 -> bf16 dequant of the tile's keys into the UMMA K-major
 //               SWIZZLE_128B layout, K half first (its buffer frees as soon as Q.K^T of the tile two
 //               back has finished), then the V operand (its buffer frees after P.V two back); the
-//               FP8 bytes of tile g+1 are loaded into registers while tile g is converted
+//               FP8 bytes of tile g+1 are loaded into registers while tile g is converted (in the
+//               scale-folding mode the converted values are the exact e4m3 values and the tile's
+//               per-token scales go to the softmax warps through a small shared array)
 //   warps 8-11  softmax: online softmax of the CTA's 64 heads (two lanes per head row), P -> SMEM,
 //               lazy O rescale, epilogue
 //   warp 12     Q.K^T issuer (CTA 0 of the pair; one elected lane issues) and TMEM owner (pair

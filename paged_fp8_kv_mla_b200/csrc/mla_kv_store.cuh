@@ -7,8 +7,9 @@
 //                                                  e4m3 with saturation to +-448),
 // written to blocks[blk, 0, layer, t % P, 0, :] with blk = lookup_table[b][t / P], and the scale to
 // scales[sblk, 0, layer, t % P, 0, 0] with sblk from scales_lookup_table when given, else blk
-// (the layout of generic_get_paged_cache_with_scales; the quantiser is the pages' data recipe:
-// per-token scale amax / 448, e4m3 round-to-nearest with saturation).
+// (the layout of generic_get_paged_cache_with_scales; the quantiser is the usual per-token FP8
+// recipe, also used to generate the test workloads: scale amax / 448, e4m3 round-to-nearest with
+// saturation).
 //
 // Eight lanes per token (a warp stores four tokens): lane k of a token's group reads 16-byte chunks
 // k, k + 8, ..., k + 64 of the 1152-byte bf16 row (each step of the group reads 128 contiguous

@@ -53,7 +53,7 @@ class DecodeConfig:
     pool_kind: str = "permuted"      # "permuted" (pool = pool_factor * pages needed) | "exact"
     pool_factor: float = 1.0
     pool_extra: int = 0
-    num_blocks: Optional[int] = None  # fixed pool size (config 0)
+    num_blocks: Optional[int] = None  # fixed pool size (the tiny two-request workload)
     separate_scales: bool = False     # scales paged through their own id space
     scales_pool_extra: int = 0
     outlier_rate: float = 0.0

@@ -5,7 +5,8 @@ mla_decode_paged_fp8_noalloc exists for callers that may not allocate device mem
 after start-up).  It keeps its split plan and partial results in a fixed array built into the
 library instead of the lazily allocated workspace, so this test calls it twice in a row with
 different problems (the second call finds the first call's leftovers in the array) and compares each
-result with mla_decode_paged_fp8 on the same inputs, at the tolerances the parity tests use.
+result with mla_decode_paged_fp8 on the same inputs, at the tolerances the parity tests use.  A
+second test captures the call in a CUDA graph and replays it with new inputs.
 
 The file name sorts last so that a run stopping at the first failure has run every other test
 first; the test also passes on its own in a fresh process.
@@ -61,3 +62,34 @@ def test_noalloc_matches_regular_entry_two_calls_in_a_row(first, second):
         torch.cuda.synchronize()
         assert M.device_status() == 0
         _close(out, lse, out_ref, lse_ref)
+
+
+def test_noalloc_captured_in_a_cuda_graph_replays_with_new_inputs():
+    """Capture the no-allocation decode once, then change q and the cache lengths in place (same
+    shapes, lengths within the captured max_cache_length, same page tables and pool) and replay:
+    the replay must equal the regular entry on the new inputs bit for bit (same kernels, same split)."""
+    inp = W.make_inputs(W.CONFIGS[1], device="cuda")
+    q = inp.q.clone()
+    lens = inp.cache_lengths.clone()
+    out = torch.empty((inp.cfg.batch, 1, inp.cfg.num_q_heads, 512), dtype=torch.bfloat16, device="cuda")
+    lse = torch.empty((inp.cfg.batch, 1, inp.cfg.num_q_heads), dtype=torch.float32, device="cuda")
+    args = (inp.blocks, inp.scales, lens, inp.lookup_table, inp.scales_lookup_table, 1, inp.max_cache_length,
+            inp.layer_idx, inp.softmax_scale, out, lse)
+    _lib.decode_noalloc(q, *args)                      # first call outside capture (sets up the scratch)
+    torch.cuda.synchronize()
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph):
+        _lib.decode_noalloc(q, *args)
+    g = torch.Generator(device="cuda")
+    g.manual_seed(99)
+    for step in range(2):
+        q.copy_(torch.randn(q.shape, generator=g, device="cuda").to(torch.bfloat16))
+        lens.copy_((inp.cache_lengths.to(torch.int64) - 37 * (step + 1)).clamp_min(0).to(torch.int32))
+        graph.replay()
+        torch.cuda.synchronize()
+        assert M.device_status() == 0
+        ref_out, ref_lse = M.decode(q, inp.blocks, inp.scales, lens, inp.lookup_table, inp.scales_lookup_table, 1,
+                                    inp.max_cache_length, inp.layer_idx, inp.softmax_scale)
+        torch.cuda.synchronize()
+        assert torch.equal(out, ref_out) and torch.equal(lse, ref_lse)
+    del graph
