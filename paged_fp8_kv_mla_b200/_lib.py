@@ -112,6 +112,62 @@ def _contig(*ts):
             raise ValueError("all tensors must be contiguous")
 
 
+_U32 = (torch.int32,) + ((torch.uint32,) if hasattr(torch, "uint32") else ())
+_CODES = (torch.uint8,) + ((torch.float8_e4m3fn,) if hasattr(torch, "float8_e4m3fn") else ())
+
+
+def _expect(name, t, dtypes, ndim=None, last=None, optional=False):
+    """The C ABI takes untyped pointers, so the binding checks what it passes: dtype, rank, last dim
+    and contiguity (the device is checked last, by _same_device)."""
+    if t is None:
+        if optional:
+            return
+        raise ValueError(f"{name} is required")
+    if not isinstance(t, torch.Tensor):
+        raise TypeError(f"{name} must be a torch.Tensor")
+    if t.dtype not in dtypes:
+        raise ValueError(f"{name} must have dtype {' or '.join(str(d) for d in dtypes)} (got {t.dtype})")
+    if ndim is not None and t.dim() != ndim:
+        raise ValueError(f"{name} must be {ndim}-D (got shape {tuple(t.shape)})")
+    if last is not None and t.shape[-1] != last:
+        raise ValueError(f"{name} must have last dim {last} (got shape {tuple(t.shape)})")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+
+
+def _same_device(*ts):
+    devs = {t.device for t in ts if t is not None}
+    if any(d.type != "cuda" for d in devs):
+        raise ValueError("all tensors must be CUDA tensors")
+    if len(devs) > 1:
+        raise ValueError(f"all tensors must be on one CUDA device (got {sorted(str(d) for d in devs)})")
+
+
+def _check_cache(blocks, scales, cache_lengths, lookup_table, scales_lookup_table, batch):
+    _expect("blocks", blocks, _CODES, ndim=6)
+    _expect("scales", scales, (torch.float32,), ndim=6)
+    _expect("cache_lengths", cache_lengths, _U32, ndim=1)
+    _expect("lookup_table", lookup_table, _U32, ndim=2)
+    _expect("scales_lookup_table", scales_lookup_table, _U32, ndim=2, optional=True)
+    if cache_lengths.shape[0] != batch or lookup_table.shape[0] != batch:
+        raise ValueError(f"cache_lengths and lookup_table must have {batch} rows (one per request)")
+    if scales_lookup_table is not None and tuple(scales_lookup_table.shape) != tuple(lookup_table.shape):
+        raise ValueError("scales_lookup_table must have the shape of lookup_table")
+
+
+def _check_decode(q, blocks, scales, cache_lengths, lookup_table, scales_lookup_table, out, lse):
+    _expect("q", q, (torch.bfloat16,), ndim=4, last=576)
+    B, T, H, _ = q.shape
+    _check_cache(blocks, scales, cache_lengths, lookup_table, scales_lookup_table, B)
+    _expect("out", out, (torch.bfloat16,), ndim=4, last=512, optional=True)
+    _expect("lse", lse, (torch.float32,), ndim=3, optional=True)
+    if out is not None and tuple(out.shape) != (B, T, H, 512):
+        raise ValueError(f"out must be {(B, T, H, 512)} (got {tuple(out.shape)})")
+    if lse is not None and tuple(lse.shape) != (B, T, H):
+        raise ValueError(f"lse must be {(B, T, H)} (got {tuple(lse.shape)})")
+    _same_device(q, blocks, scales, cache_lengths, lookup_table, scales_lookup_table, out, lse)
+
+
 def decode(q, blocks, scales, cache_lengths, lookup_table, scales_lookup_table, max_prompt_length: int,
            max_cache_length: int, layer_idx: int, softmax_scale: float, out=None, lse=None, stream=None,
            want_lse: bool = True, fold_scales: bool = False):
@@ -122,9 +178,9 @@ def decode(q, blocks, scales, cache_lengths, lookup_table, scales_lookup_table, 
     fold_scales=True calls mla_decode_paged_fp8_scale_folded instead (g = 1 only).
     Returns (out bf16 [B, T, H, 512], lse fp32 [B, T, H] or None).
     """
+    _check_decode(q, blocks, scales, cache_lengths, lookup_table, scales_lookup_table, out, lse)
     lib = load()
     B, T, H, D = q.shape
-    _contig(q, blocks, scales, cache_lengths, lookup_table, scales_lookup_table)
     if out is None:
         out = torch.empty((B, T, H, 512), dtype=torch.bfloat16, device=q.device)
     if lse is None and want_lse:
@@ -142,9 +198,11 @@ def kv_store(latent, cache_lengths, lookup_table, scales_lookup_table, layer_idx
              stream=None):
     """mla_kv_store_fp8 on torch tensors: quantise latent bf16 [B, T, 576] and write it in place into
     blocks / scales at positions cache_lengths[b] + i (page tables as for decode)."""
-    lib = load()
+    _expect("latent", latent, (torch.bfloat16,), ndim=3, last=576)
     B, T, D = latent.shape
-    _contig(latent, blocks, scales, cache_lengths, lookup_table, scales_lookup_table)
+    _check_cache(blocks, scales, cache_lengths, lookup_table, scales_lookup_table, B)
+    _same_device(latent, blocks, scales, cache_lengths, lookup_table, scales_lookup_table)
+    lib = load()
     shp = paged_shape(B, 0, blocks, scales, lookup_table)
     st = lib.mla_kv_store_fp8(_ptr(latent), _ptr(cache_lengths), _ptr(lookup_table), _ptr(scales_lookup_table),
                               int(T), int(layer_idx), ctypes.byref(shp), _ptr(blocks), _ptr(scales), _stream(stream))
@@ -158,9 +216,11 @@ def decode_noalloc(q, blocks, scales, cache_lengths, lookup_table, scales_lookup
 
     `out` and `lse` must be preallocated by the caller.
     """
+    if out is None or lse is None:
+        raise ValueError("decode_noalloc needs preallocated out and lse")
+    _check_decode(q, blocks, scales, cache_lengths, lookup_table, scales_lookup_table, out, lse)
     lib = load()
     B, T, H, D = q.shape
-    _contig(q, blocks, scales, cache_lengths, lookup_table, scales_lookup_table, out, lse)
     shp = paged_shape(B, H, blocks, scales, lookup_table)
     st = lib.mla_decode_paged_fp8_noalloc(_ptr(q), _ptr(blocks), _ptr(scales), _ptr(cache_lengths),
                                           _ptr(lookup_table), _ptr(scales_lookup_table), int(max_prompt_length),
@@ -173,12 +233,16 @@ def decode_noalloc(q, blocks, scales, cache_lengths, lookup_table, scales_lookup
 def merge_parts(outs, lses, out=None, lse=None, stream=None):
     """mla_merge_lse_parts_bf16: outs bf16 [R, ..., 512] and lses fp32 [R, ...] (the parts' decode
     results over disjoint key ranges) -> (out bf16 [..., 512], lse fp32 [...])."""
+    _expect("outs", outs, (torch.bfloat16,), last=512)
+    _expect("lses", lses, (torch.float32,))
+    if outs.dim() < 2 or outs.shape[:-1] != lses.shape:
+        raise ValueError("outs must be [R, ..., 512] and lses [R, ...] with the same leading dims")
+    _expect("out", out, (torch.bfloat16,), optional=True)
+    _expect("lse", lse, (torch.float32,), optional=True)
+    _same_device(outs, lses, out, lse)
     lib = load()
-    _contig(outs, lses)
     R = outs.shape[0]
     rows = lses[0].numel()
-    if outs.shape[:-1] != lses.shape or outs.shape[-1] != 512:
-        raise ValueError("outs must be [R, ..., 512] and lses [R, ...] with the same leading dims")
     if out is None:
         out = torch.empty(outs.shape[1:], dtype=torch.bfloat16, device=outs.device)
     if lse is None:
@@ -199,10 +263,14 @@ def gather_dequant(blocks, scales, cache_lengths, lookup_table, scales_lookup_ta
                    max_prompt_length: int, max_cache_length: int, layer_idx: int, max_keys: Optional[int] = None,
                    out_k=None, stream=None):
     """mla_gather_dequant_bf16: bf16 [B, max_keys, 576] of every stored key (rows past n_b untouched)."""
-    lib = load()
-    _contig(blocks, scales, cache_lengths, lookup_table, scales_lookup_table)
+    _check_cache(blocks, scales, cache_lengths, lookup_table, scales_lookup_table, batch)
     if max_keys is None:
         max_keys = max_cache_length + max_prompt_length
+    _expect("out_k", out_k, (torch.bfloat16,), ndim=3, last=576, optional=True)
+    if out_k is not None and tuple(out_k.shape) != (batch, max_keys, 576):
+        raise ValueError(f"out_k must be {(batch, max_keys, 576)} (got {tuple(out_k.shape)})")
+    _same_device(blocks, scales, cache_lengths, lookup_table, scales_lookup_table, out_k)
+    lib = load()
     if out_k is None:
         out_k = torch.zeros((batch, max_keys, 576), dtype=torch.bfloat16, device=blocks.device)
     shp = paged_shape(batch, 1, blocks, scales, lookup_table)
