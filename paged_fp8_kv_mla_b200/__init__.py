@@ -7,5 +7,5 @@ parallelism (`context_parallel`).
 """
 from ._lib import (  # noqa: F401
     MlaError, decode, decode_inputs, gather_dequant, kv_store, set_num_clusters, get_num_clusters, device_status,
-    release_workspace, version, set_timing_events, load, LIB_PATH, EXPORTED, merge_parts,
+    release_workspace, version, set_timing_events, load, LIB_PATH, EXPORTED, merge_parts, decode_noalloc,
 )
