@@ -64,10 +64,16 @@ def load_peaks():
 
 
 def kernel_source_sha():
+    """Hash of the CUDA sources' code (comments and whitespace removed), so that a recorded ncu
+    capture stays valid across comment edits and becomes invalid with any code change."""
+    import re
     h = hashlib.sha256()
-    for f in ("ptx.cuh", "mla_kernels.cuh", "mla_api.cu", "mla_kv_store.cuh"):
-        with open(os.path.join(ROOT, "paged_fp8_kv_mla_b200", "csrc", f), "rb") as fh:
-            h.update(fh.read())
+    for f in ("ptx.cuh", "mla_kernels.cuh", "mla_api.cu", "mla_kv_store.cuh", "mla_merge.cuh"):
+        with open(os.path.join(ROOT, "paged_fp8_kv_mla_b200", "csrc", f)) as fh:
+            src = fh.read()
+        src = re.sub(r"/\*.*?\*/", " ", src, flags=re.S)
+        src = re.sub(r"//[^\n]*", " ", src)
+        h.update(" ".join(src.split()).encode())
     return h.hexdigest()[:16]
 
 
