@@ -60,9 +60,10 @@ typedef enum {
 
 /* Shapes of the paged cache (the 6-D tensors of "generic_get_paged_cache_with_scales")
  * and of q.  Implemented subset: head_dim == 576, v_dim == 512, num_kv_heads == 1,
- * head_dim_granularity == 1 (one fp32 scale per token), page_size a multiple of 16,
- * kv_dim >= 1 (index 0, the latent cache, is read), any num_q_heads >= 1 (processed
- * in groups of 128). */
+ * head_dim_granularity g in {1, 2, 3, 4, 6, 9, 12, 18, 36} (g fp32 scales per token, scale j
+ * covering dims [j * 576 / g, (j + 1) * 576 / g); the KV-store step and the scale-folding decode
+ * take g = 1 only), page_size a multiple of 16, kv_dim >= 1 (index 0, the latent cache, is read),
+ * any num_q_heads >= 1 (processed in groups of 128). */
 typedef struct {
   int32_t batch;                /* B */
   int32_t num_q_heads;          /* H */
@@ -75,7 +76,7 @@ typedef struct {
   int32_t num_kv_heads;         /* num_heads of blocks / scales: 1 */
   int32_t num_scale_blocks;     /* leading dim of scales (may differ from num_blocks
                                    when scales_lookup_table != NULL) */
-  int32_t head_dim_granularity; /* last dim of scales: 1 */
+  int32_t head_dim_granularity; /* last dim of scales: g (1 = one scale per token) */
   int32_t max_pages;            /* second dim of lookup_table (and scales_lookup_table) */
 } mla_paged_shape_t;
 
@@ -84,7 +85,8 @@ typedef struct {
  *
  *   q                    bf16 [batch, max_prompt_length, num_q_heads, 576], 16-byte aligned
  *   blocks               e4m3 [num_blocks, kv_dim, num_layers, page_size, 1, 576], 16-byte aligned
- *   scales               fp32 [num_scale_blocks, kv_dim, num_layers, page_size, 1, 1], 16-byte aligned
+ *   scales               fp32 [num_scale_blocks, kv_dim, num_layers, page_size, 1, g], 16-byte aligned;
+ *                        with g > 1, dim d of a key uses its scale d / (576 / g)
  *   cache_lengths        uint32 [batch]: tokens cached before this step
  *   lookup_table         uint32 [batch, max_pages]: logical page -> block id
  *   scales_lookup_table  NULL, or uint32 [batch, max_pages]: logical page -> scale block id
