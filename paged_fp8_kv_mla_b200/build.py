@@ -1,6 +1,6 @@
 """Build the C-ABI shared library libmla_paged_fp8.so in place (nvcc, sm_100a only).
 
-    python -m paged_fp8_kv_mla_b200.build [--debug] [--verbose-ptxas]
+    python -m paged_fp8_kv_mla_b200.build [--debug] [--verbose-ptxas] [--trace]
 
 No GPU is needed: nvcc cross-compiles for sm_100a.  The library links the CUDA
 runtime statically and reaches the driver's tensor-map encoder through
@@ -23,6 +23,9 @@ def _deps():
     return sorted(os.path.join(d, f) for f in os.listdir(d) if f.endswith((".cu", ".cuh"))) + \
         [os.path.join(ROOT, "include", "mla_paged_fp8.h")]
 LIB = os.path.join(PKG, "libmla_paged_fp8.so")
+# Diagnostic variant with the decode kernel's per-stage %clock64 stamps compiled in (read by
+# paged_fp8_kv_mla_b200.trace); never the library the product path loads.
+TRACE_LIB = os.path.join(PKG, "libmla_paged_fp8_trace.so")
 
 
 def nvcc_path() -> str:
@@ -39,7 +42,10 @@ def needs_build(out: str = LIB) -> bool:
     return any(os.path.getmtime(d) > t for d in _deps() + [__file__])
 
 
-def build(debug: bool = False, verbose_ptxas: bool = False, force: bool = False, out: str = LIB) -> str:
+def build(debug: bool = False, verbose_ptxas: bool = False, force: bool = False, out: str = LIB,
+          trace: bool = False) -> str:
+    if trace and out == LIB:
+        out = TRACE_LIB
     if not force and not needs_build(out):
         return out
     cmd = [
@@ -50,6 +56,8 @@ def build(debug: bool = False, verbose_ptxas: bool = False, force: bool = False,
     ] + SRC
     if debug:
         cmd += ["-DMLA_DEBUG=1"]
+    if trace:
+        cmd += ["-DMLA_TRACE"]
     if verbose_ptxas:
         cmd += ["-Xptxas", "-v"]
     r = subprocess.run(cmd, capture_output=True, text=True)
@@ -66,5 +74,6 @@ if __name__ == "__main__":
     ap = argparse.ArgumentParser()
     ap.add_argument("--debug", action="store_true")
     ap.add_argument("--verbose-ptxas", action="store_true")
+    ap.add_argument("--trace", action="store_true", help="build the diagnostic trace variant")
     a = ap.parse_args()
-    print(build(debug=a.debug, verbose_ptxas=a.verbose_ptxas, force=True))
+    print(build(debug=a.debug, verbose_ptxas=a.verbose_ptxas, force=True, trace=a.trace))

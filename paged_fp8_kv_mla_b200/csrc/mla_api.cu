@@ -553,7 +553,8 @@ mla_status_t mla_debug_set_trace(unsigned long long* buf) {
 }
 
 // Trace builds only: copies the %globaltimer marks of the last decode call (plan end, first decode
-// CTA entry, last decode CTA exit, first combine CTA entry) to out8 and, if reset, re-arms them.
+// CTA entry, last decode CTA exit, first combine CTA past its wait, last combine warp done, first
+// combine CTA entry) to out8 and, if reset, re-arms them.
 mla_status_t mla_debug_marks(unsigned long long* out8, int reset) {
   MLA_CUDA(cudaDeviceSynchronize());
   MLA_CUDA(cudaMemcpyFromSymbol(out8, mla::g_trace_marks, 8 * sizeof(unsigned long long)));
