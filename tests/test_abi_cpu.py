@@ -92,6 +92,20 @@ def test_merge_host_validation(lib):
     assert f(FAKE, FAKE, 2, 10, ctypes.c_void_p(0x10004), None, None) == 1
 
 
+def test_empty_batch_is_a_no_op_on_every_entry(lib):
+    """batch = 0 (or no new tokens) returns MLA_OK after the host checks, before any CUDA call."""
+    shp = _shape(batch=0)
+    assert _call(lib, shp) == 0
+    assert lib.mla_decode_paged_fp8_scale_folded(FAKE, FAKE, FAKE, FAKE, FAKE, None, 1, 64, 0, 0.07,
+                                                 ctypes.byref(shp), FAKE, None, None) == 0
+    assert lib.mla_decode_paged_fp8_noalloc(FAKE, FAKE, FAKE, FAKE, FAKE, None, 1, 64, 0, 0.07,
+                                            ctypes.byref(shp), FAKE, None, None) == 0
+    assert lib.mla_gather_dequant_bf16(FAKE, FAKE, FAKE, FAKE, None, 1, 64, 0, ctypes.byref(shp), FAKE, 65,
+                                       None) == 0
+    assert _store(lib, _shape(batch=0)) == 0
+    assert _store(lib, _shape(), T=0) == 0
+
+
 def _store(lib, shape, latent=FAKE, lens=FAKE, lut=FAKE, slut=None, T=1, layer=0, blocks=FAKE, scales=FAKE):
     return lib.mla_kv_store_fp8(latent, lens, lut, slut, T, layer,
                                 ctypes.byref(shape) if shape is not None else None, blocks, scales, None)
