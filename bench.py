@@ -154,6 +154,15 @@ def max_over_ranks(dist, values, device):
     return [float(x) for x in t.tolist()]
 
 
+def sum_over_ranks(dist, values, device):
+    """Element-wise sum across the process group (the work all replicas did: their batches differ)."""
+    if dist is None:
+        return [float(v) for v in values]
+    t = torch.tensor([float(v) for v in values], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.SUM)
+    return [float(x) for x in t.tolist()]
+
+
 def cpu_oracle_baseline(inp, budget_s, rank_requests=None, fold=False):
     """The float64 oracle, as it stands, on whole requests of the same workload until ~budget_s."""
     import numpy as np
@@ -358,6 +367,8 @@ def main():
     inp = W.make_inputs(cfg, device="cuda", seed=seed)
     kv_bytes = inp.kv_scale_bytes()
     flops = inp.flops()
+    # the bytes every replica reads in one step (each draws its own batch of lengths)
+    kv_bytes_all = sum_over_ranks(dist, [kv_bytes], "cuda")[0]
     B, T = cfg.batch, cfg.q_len
     out = torch.empty((B, T, cfg.num_q_heads, 512), dtype=torch.bfloat16, device="cuda")
     lse = torch.empty((B, T, cfg.num_q_heads), dtype=torch.float32, device="cuda")
@@ -452,14 +463,14 @@ def main():
         e2e_ms = sum(a.elapsed_time(b) for a, b in eev) / Ke
         if dist:
             e2e_ms = max_over_ranks(dist, [e2e_ms], "cuda")[0]
-        e2e = {"value": kv_bytes * world / (e2e_ms * 1e-3) / 1e9, "unit": "GB/s", "h2d_bytes_per_step": h2d,
+        e2e = {"value": kv_bytes_all / (e2e_ms * 1e-3) / 1e9, "unit": "GB/s", "h2d_bytes_per_step": h2d,
                "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms}
 
     if dist:
         step_ms, kern_ms = max_over_ranks(dist, [step_ms, kern_ms], "cuda")
 
     peaks = load_peaks()
-    gbs = kv_bytes * world / (step_ms * 1e-3) / 1e9
+    gbs = kv_bytes_all / (step_ms * 1e-3) / 1e9
     tflops_k = flops / (kern_ms * 1e-3) / 1e12
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
@@ -473,7 +484,8 @@ def main():
             "hbm_frac": gbs / world / peaks["hbm_gbs"],
             "config": {"workload": cfg.name, "config_index": args.config, "batch": B, "q_len": T,
                        "num_q_heads": cfg.num_q_heads, "page_size": cfg.page_size,
-                       "kv_scale_bytes_per_step": kv_bytes, "flops_per_step": flops,
+                       "kv_scale_bytes_per_step": kv_bytes, "kv_scale_bytes_per_step_all_gpus": kv_bytes_all,
+                       "flops_per_step": flops,
                        "l2": "flushed before every timed step (write of %d MB)" % (flush.numel() >> 20),
                        "parallelism": f"replicas x{world}"},
             "roofline": {"kernel": "mla_decode_kernel", "bound": "tensor", "achieved": tflops_k,
