@@ -5,7 +5,6 @@ import os
 import re
 
 import pytest
-import torch
 
 import paged_fp8_kv_mla_b200 as M
 from paged_fp8_kv_mla_b200 import _lib, build

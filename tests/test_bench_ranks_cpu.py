@@ -3,8 +3,6 @@ inputs (different seeds, same shapes), the reported time is the maximum over ran
 the sum of every rank's bytes."""
 import os
 
-import pytest
-import torch
 import torch.distributed as dist
 import torch.multiprocessing as mp
 

@@ -13,7 +13,7 @@ import torch
 import paged_fp8_kv_mla_b200 as M
 from oracle import mla_oracle as O
 from paged_fp8_kv_mla_b200 import workloads as W
-from tests.oracle_io import oracle_decode, to_numpy
+from tests.oracle_io import oracle_decode
 
 pytestmark = pytest.mark.gpu
 

@@ -6,8 +6,6 @@ bf16 tiles must be bit-exact.  Page permutation and scale id space must not
 change the GPU result at all (the reduction order depends only on logical token
 order and lengths).
 """
-import math
-
 import numpy as np
 import pytest
 import torch
