@@ -151,7 +151,11 @@ mla_status_t mla_decode_paged_fp8_scale_folded(
  * the library: about 42.5 MB on every GPU that loads the library, held until the process exits.
  * It never calls cudaMalloc or cudaFree.  Limits: batch * max_prompt_length *
  * ceil(num_q_heads / 128) <= 65536 (else MLA_ERR_UNSUPPORTED, with the reason in
- * mla_last_error_string), and the keys are split over at most 80 two-CTA clusters.
+ * mla_last_error_string), and the keys are split over at most 80 two-CTA clusters: when the
+ * cluster count in force (the device's resident count, 74 on a B200, or the one set with
+ * mla_set_num_clusters) is larger, the call returns MLA_ERR_UNSUPPORTED instead of changing the
+ * split, so a successful call always splits the keys exactly as mla_decode_paged_fp8 does and
+ * returns bit-identical results.
  * The first call on a device looks up the array's device address and sets kernel attributes; make
  * that first call before any stream capture.  All calls share the array: calls whose GPU work
  * overlaps (for example on two streams) race and corrupt each other's results, so serialise them.
@@ -248,6 +252,24 @@ mla_status_t mla_set_num_clusters(int32_t num_clusters);
  * the caller.
  */
 mla_status_t mla_set_timing_events(cudaEvent_t before, cudaEvent_t after);
+
+/*
+ * mla_set_wait_limit_ns -- bound of every wait inside the decode kernel (the roles of a CTA pair
+ * hand tiles to each other through mbarriers).  A wait that runs out makes every role of the pair
+ * stop, drain its own copies and MMAs and return; the call's results are then undefined and the
+ * next mla_get_device_status returns MLA_ERR_TIMEOUT.  Default 2 s; accepted range [1 ms, 60 s]
+ * (else MLA_ERR_INVALID_ARG).  Process-wide; applies to calls made after it.
+ */
+mla_status_t mla_set_wait_limit_ns(uint64_t ns);
+
+/*
+ * mla_debug_withhold_arrival_once -- test hook for the timeout path: in the next decode call (of
+ * any entry point) the Q loader of CTA 1 of the first cluster withholds its arrival on the first
+ * unit's Q-ready barrier, so the Q.K^T issuer's wait runs out after the wait limit.  The call
+ * returns normally, its results are undefined, and mla_get_device_status then reports
+ * MLA_ERR_TIMEOUT; the device stays usable.  No reference page has a counterpart.
+ */
+mla_status_t mla_debug_withhold_arrival_once(void);
 
 /* Number of clusters the next decode on the current device will use. */
 int32_t mla_get_num_clusters(void);

@@ -6,6 +6,6 @@ build step (`build`), the seeded workload generators (`workloads`) and the host 
 parallelism (`context_parallel`).
 """
 from ._lib import (  # noqa: F401
-    MlaError, decode, decode_inputs, gather_dequant, kv_store, set_num_clusters, get_num_clusters, device_status,
+    MlaError, decode, decode_inputs, gather_dequant, kv_store, set_num_clusters, get_num_clusters, set_wait_limit_ns, withhold_arrival_once, device_status,
     release_workspace, version, set_timing_events, load, LIB_PATH, EXPORTED, merge_parts, decode_noalloc,
 )

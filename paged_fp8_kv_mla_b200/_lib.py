@@ -23,7 +23,8 @@ STATUS_NAMES = {0: "MLA_OK", 1: "MLA_ERR_INVALID_ARG", 2: "MLA_ERR_UNSUPPORTED",
 EXPORTED = ["mla_decode_paged_fp8", "mla_gather_dequant_bf16", "mla_set_num_clusters",
             "mla_get_num_clusters", "mla_last_error_string", "mla_get_device_status",
             "mla_release_workspace", "mla_version", "mla_set_timing_events", "mla_decode_paged_fp8_noalloc",
-            "mla_kv_store_fp8", "mla_decode_paged_fp8_scale_folded", "mla_merge_lse_parts_bf16"]
+            "mla_kv_store_fp8", "mla_decode_paged_fp8_scale_folded", "mla_merge_lse_parts_bf16",
+            "mla_set_wait_limit_ns", "mla_debug_withhold_arrival_once"]
 
 
 class MlaError(RuntimeError):
@@ -75,6 +76,10 @@ def load(path: str = LIB_PATH) -> ctypes.CDLL:
     lib.mla_get_device_status.restype = ctypes.c_int
     lib.mla_release_workspace.argtypes = []
     lib.mla_release_workspace.restype = ctypes.c_int
+    lib.mla_set_wait_limit_ns.argtypes = [ctypes.c_uint64]
+    lib.mla_set_wait_limit_ns.restype = ctypes.c_int
+    lib.mla_debug_withhold_arrival_once.argtypes = []
+    lib.mla_debug_withhold_arrival_once.restype = ctypes.c_int
     lib.mla_set_timing_events.argtypes = [vp, vp]
     lib.mla_set_timing_events.restype = ctypes.c_int
     lib.mla_version.argtypes = []
@@ -283,6 +288,16 @@ def gather_dequant(blocks, scales, cache_lengths, lookup_table, scales_lookup_ta
 
 def set_num_clusters(n: int):
     _check(load().mla_set_num_clusters(int(n)))
+
+
+def set_wait_limit_ns(ns: int):
+    """Bound of every wait inside the decode kernel (default 2 s)."""
+    _check(load().mla_set_wait_limit_ns(int(ns)))
+
+
+def withhold_arrival_once():
+    """Test hook: the next decode call withholds one barrier arrival, so a bounded wait runs out."""
+    _check(load().mla_debug_withhold_arrival_once())
 
 
 def get_num_clusters() -> int:

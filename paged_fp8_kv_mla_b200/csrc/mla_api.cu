@@ -52,6 +52,8 @@ Workspace g_ws[kMaxDevices];
 int g_default_nc[kMaxDevices];         // resident 2-CTA cluster slots, 0 = not queried yet
 bool g_attr_set[kMaxDevices];
 int g_forced_nc = 0;
+unsigned long long g_wait_limit_ns = mla::DEFAULT_WAIT_LIMIT_NS;
+int g_inject_once = mla::INJECT_NONE;   // test hook, consumed by the next decode call
 
 size_t align_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
 
@@ -254,6 +256,14 @@ unsigned int* status_ptr() {
   return p;
 }
 
+// Wait bound of the decode kernel's mbarrier waits, and the one-shot test hook.
+void set_wait_params(mla::DecodeParams* p) {
+  std::lock_guard<std::mutex> lk(g_mu);
+  p->wait_limit_ns = g_wait_limit_ns;
+  p->inject = g_inject_once;
+  g_inject_once = mla::INJECT_NONE;
+}
+
 // The three launches of one decode call on `stream`: plan -> decode -> combine.  The decode and
 // combine kernels are launched as programmatic dependents of the kernel before them, so their
 // launch and (for the decode kernel) prologue overlap the previous kernel; each waits for its
@@ -362,6 +372,20 @@ mla_status_t mla_set_num_clusters(int32_t num_clusters) {
   return MLA_OK;
 }
 
+mla_status_t mla_set_wait_limit_ns(uint64_t ns) {
+  if (ns < 1000000ull || ns > 60000000000ull)
+    return fail(MLA_ERR_INVALID_ARG, "wait limit %llu ns outside [1 ms, 60 s]", static_cast<unsigned long long>(ns));
+  std::lock_guard<std::mutex> lk(g_mu);
+  g_wait_limit_ns = ns;
+  return MLA_OK;
+}
+
+mla_status_t mla_debug_withhold_arrival_once(void) {
+  std::lock_guard<std::mutex> lk(g_mu);
+  g_inject_once = mla::INJECT_SKIP_Q_ARRIVAL;
+  return MLA_OK;
+}
+
 mla_status_t mla_set_timing_events(cudaEvent_t before, cudaEvent_t after) {
   if ((before == nullptr) != (after == nullptr)) return fail(MLA_ERR_INVALID_ARG, "pass both events or neither");
   g_ev_before = before;
@@ -429,6 +453,7 @@ mla_status_t decode_alloc(const void* q, const void* blocks, const float* scales
   p.status = status_ptr();
   if (!p.status) return fail(MLA_ERR_CUDA, "status word address unavailable");
   p.scale_log2 = softmax_scale * 1.4426950408889634f;
+  set_wait_params(&p);
 #ifdef MLA_TRACE
   p.trace = g_trace;
 #endif
@@ -481,6 +506,7 @@ mla_status_t mla_gather_dequant_bf16(const void* blocks, const float* scales, co
   p.slut = scales_lookup_table;
   p.status = status_ptr();
   if (!p.status) return fail(MLA_ERR_CUDA, "status word address unavailable");
+  p.wait_limit_ns = g_wait_limit_ns;
   const int tiles = static_cast<int>((static_cast<uint64_t>(max_keys) + mla::BN - 1) / mla::BN);
   const int64_t gx = static_cast<int64_t>(p.B) * tiles;
   if (gx > 0x7FFFFFFF) return fail(MLA_ERR_UNSUPPORTED, "grid too large");
@@ -600,7 +626,10 @@ mla_status_t mla_decode_paged_fp8_noalloc(const void* q, const void* blocks, con
   int NC = 0;
   st = device_setup(dev, &NC);
   if (st != MLA_OK) return st;
-  if (NC > kNoAllocMaxClusters) NC = kNoAllocMaxClusters;
+  if (NC > kNoAllocMaxClusters)
+    return fail(MLA_ERR_UNSUPPORTED,
+                "the no-allocation decode splits the keys over at most %d clusters, this call would use %d "
+                "(lower it with mla_set_num_clusters)", kNoAllocMaxClusters, NC);
   p.NC = NC;
 
   void* ws = nullptr;
@@ -624,6 +653,7 @@ mla_status_t mla_decode_paged_fp8_noalloc(const void* q, const void* blocks, con
   p.status = status_ptr();
   if (!p.status) return fail(MLA_ERR_CUDA, "status word address unavailable");
   p.scale_log2 = softmax_scale * 1.4426950408889634f;
+  set_wait_params(&p);
 
   return launch_path(p, NC, cache_lengths, max_cache_length, stream, false);
 }

@@ -17,21 +17,27 @@
 //           D_c = [128c, 128c+128) u [256+128c, 256+128c+128).  Its own 32 keys' D_c dims come from
 //           the same conversion as its K half; it dequantises the other CTA's 32 keys' D_c dims
 //           itself (256 of their 576 bytes), so no converted data crosses between SMs.
-// Every KV byte is read from HBM once (the second CTA's partial reads hit L2).
+// Every KV byte is read from HBM once (the other CTA's partial reads hit L2).
 //
-// Warp roles per CTA (480 threads):
-//   warps 0-7   converter: FP8 -> bf16 dequant of the tile's keys into the UMMA K-major
-//               SWIZZLE_128B layout, K half first (its buffer frees as soon as Q.K^T of the tile two
-//               back has finished), then the V operand (its buffer frees after P.V two back); the
-//               FP8 bytes of tile g+1 are loaded into registers while tile g is converted (in the
-//               scale-folding mode the converted values are the exact e4m3 values and the tile's
-//               per-token scales go to the softmax warps through a small shared array)
-//   warps 8-11  softmax: online softmax of the CTA's 64 heads (two lanes per head row), P -> SMEM,
+// The FP8 pages reach shared memory through a two-stage ring ("KVLoad2CvtProducer", which stages
+// FP8 tiles in shared memory for converter warps behind a producer): per tile, CTA c's producer
+// bulk-copies its own 32 keys' rows (one contiguous 18 KB run per page) and their per-token
+// scales into a stage, with a full / empty mbarrier pair per stage.
+//
+// Warp roles per CTA (640 threads):
+//   warps 0-11  converter, three groups of four warps (one warp of each group per scheduler).  Group
+//               q dequantises atom columns 3q..3q+2 (192 dims) of the CTA's own 32 keys from the
+//               ring into the K half buffer (single buffered: written once Q.K^T of the previous
+//               tile has finished), then its share of the V operand (double buffered) once P.V two
+//               tiles back has finished.  The other CTA's keys' D_c bytes are loaded from global
+//               memory (they are in L2: the other CTA's producer brought them) one tile ahead.
+//   warps 12-15 softmax: online softmax of the CTA's 64 heads (two lanes per head row), P -> SMEM,
 //               lazy O rescale, epilogue
-//   warp 12     Q.K^T issuer (CTA 0 of the pair; one elected lane issues) and TMEM owner (pair
+//   warp 16     Q.K^T issuer (CTA 0 of the pair; one elected lane issues) and TMEM owner (pair
 //               allocation in both CTAs)
-//   warp 13     P.V issuer (CTA 0)
-//   warp 14     Q loader: one TMA tile load of the CTA's 64 heads x 576 dims per unit
+//   warp 17     P.V issuer (CTA 0)
+//   warp 18     Q loader: one TMA tile load of the CTA's 64 heads x 576 dims per unit
+//   warp 19     FP8 producer: page-table lookup and bulk copies of the ring (one elected lane)
 #pragma once
 #include <cuda_bf16.h>
 #include <cstdint>
@@ -45,33 +51,41 @@ constexpr int HEAD_DIM = 576;
 constexpr int V_DIM = 512;
 constexpr int MROWS = 128;      // query heads per item (pair MMA M)
 constexpr int HPC = 64;         // query heads per CTA
-constexpr int NUM_THREADS = 480;
-constexpr int CONV_THREADS = 256;
-constexpr int CONV_WARPS = CONV_THREADS / 32;
-constexpr int SM_WARP0 = 8;     // first softmax warp (warps 8..11 reach TMEM lane quadrants 0..3)
-constexpr int QK_WARP = 12;     // Q.K^T issuer (CTA 0), TMEM owner (both CTAs)
-constexpr int PV_WARP = 13;     // P.V issuer (CTA 0)
-constexpr int Q_WARP = 14;      // Q tile loader
+constexpr int CONV_WARPS = 12;
+constexpr int CONV_THREADS = 32 * CONV_WARPS;
+constexpr int CONV_GROUP = 128;  // threads per converter group (three groups, 3 atom columns each)
+constexpr int SM_WARP0 = 12;    // first softmax warp (warps 12..15 reach TMEM lane quadrants 0..3)
+constexpr int QK_WARP = 16;     // Q.K^T issuer (CTA 0), TMEM owner (both CTAs)
+constexpr int PV_WARP = 17;     // P.V issuer (CTA 0)
+constexpr int Q_WARP = 18;      // Q tile loader
+constexpr int LOAD_WARP = 19;   // FP8 producer
+constexpr int NUM_THREADS = 640;
+static_assert(SM_WARP0 % 4 == 0, "softmax warps must start a warpgroup (TMEM lane quadrants)");
 
-// ---- shared memory map (offsets from a 1024-byte aligned base); all operands K-major SWIZZLE_128B,
-//      one "atom column" = 64 bf16 dims x rows at 128 B, 8-row groups 1024 B apart
+// ---- shared memory map (offsets from a 1024-byte aligned base); all bf16 operands K-major
+//      SWIZZLE_128B, one "atom column" = 64 bf16 dims x rows at 128 B, 8-row groups 1024 B apart
 constexpr uint32_t SQ = 0;                       // Q: 9 atom columns x (64 rows x 128 B)
 constexpr uint32_t SQ_ATOM = 8192;
-constexpr uint32_t SK0 = 9 * SQ_ATOM;            // K half (2 buffers): 9 atom columns x (32 rows x 128 B)
+constexpr uint32_t SK = 9 * SQ_ATOM;             // K half (one buffer): 9 atom columns x (32 rows x 128 B)
 constexpr uint32_t SK_ATOM = 4096;
-constexpr uint32_t SK_STRIDE = 9 * SK_ATOM;
-constexpr uint32_t SV0 = SK0 + 2 * SK_STRIDE;    // V operand (2 buffers): 4 atom columns x (64 rows x 128 B)
+constexpr uint32_t SK_BYTES = 9 * SK_ATOM;
+constexpr uint32_t SV0 = SK + SK_BYTES;          // V operand (2 buffers): 4 atom columns x (64 rows x 128 B)
 constexpr uint32_t SV_ATOM = 8192;
 constexpr uint32_t SV_STRIDE = 4 * SV_ATOM;
 constexpr uint32_t SP0 = SV0 + 2 * SV_STRIDE;    // P (2 buffers): 64 rows x 128 B
 constexpr uint32_t SP_STRIDE = 8192;
-constexpr uint32_t SRED = SP0 + 2 * SP_STRIDE;   // row-max exchange [2][128] f32, row-sum exchange [128] f32
+constexpr uint32_t SRING = SP0 + 2 * SP_STRIDE;  // FP8 ring (2 stages): 32 rows x 576 B, then 32 fp32 scales
+constexpr uint32_t RING_ROWS = HALF_BN * HEAD_DIM;
+constexpr uint32_t RING_STAGE = RING_ROWS + HALF_BN * 4;
+constexpr uint32_t SRED = SRING + 2 * RING_STAGE;   // row-max exchange [2][128] f32, row-sum exchange [128] f32
 constexpr uint32_t SBAR = SRED + 1536;
 constexpr uint32_t SMEM_USED = SBAR + 256;
 constexpr uint32_t SMEM_ALLOC = SMEM_USED + 1024;   // slack for aligning the base
+static_assert(SMEM_ALLOC <= 232448, "shared memory map exceeds 227 KB");
+static_assert(RING_STAGE % 16 == 0 && SRING % 16 == 0, "bulk copies need 16-byte aligned stages");
 // Scale-folding mode only: the per-token scales of the last four tiles ([4][64] f32), handed from
 // the converter to the softmax warps.  It sits after SMEM_USED, inside the alignment slack, with
-// the allocation raised to the 227 KB limit; the kernel checks that the base needed at most
+// the allocation at the 227 KB limit; the kernel checks that the base needed at most
 // SMEM_FOLD_MAX_PAD bytes of alignment (it needs none when the runtime places dynamic shared
 // memory on a 1 KB boundary) and reports STATUS_LAYOUT otherwise.
 constexpr uint32_t SSC = SMEM_USED;
@@ -88,24 +102,27 @@ enum ScaleMode : int {
 };
 
 enum Bar : uint32_t {
-  B_K_FULL = 0,    // [2] CTA 0: 16 warp arrivals (8 converter warps of each CTA): K half converted
-  B_V_FULL = 2,    // [2] CTA 0: 16 warp arrivals: V operand converted
-  B_PV_DONE = 4,   // [2] both CTAs: pair commit after P.V of a tile (its V and P buffers are free)
-  B_S_FULL = 6,    // [2] both CTAs: pair commit after Q.K^T of a tile (its K buffer is free)
-  B_S_FREE = 8,    // [2] CTA 0: 8 warp arrivals (4 softmax warps of each CTA hold S in registers)
-  B_P_FULL = 10,   // [2] CTA 0: 8 warp arrivals
-  B_Q_FULL = 12,   // CTA 0: 2 arrivals (the Q loader of each CTA)
-  B_Q_FREE = 13,   // both CTAs: pair commit after the last Q.K^T of a unit
-  B_Q_LOCAL = 14,  // both CTAs: transaction barrier of this CTA's Q tile load
-  B_O_FREE = 15,   // CTA 0: 8 warp arrivals after each CTA's epilogue
-  B_DRAIN = 16,    // CTA 0: one commit from each issuer at exit
-  B_RED = 17,      // [2] softmax warps of this CTA: row-max exchange of a tile (4 warp arrivals)
-  B_REDL = 19,     // softmax warps of this CTA: row-sum exchange at a unit's end (4 warp arrivals)
-  B_EXIT = 20,     // both CTAs: the peer has finished (1 remote arrival)
-  B_SC_FULL = 21,  // [4] scale-folding mode: 8 converter-warp arrivals, a tile's scales are in SSC
-  NUM_BARS = 25
+  B_K_FULL = 0,       // CTA 0: 24 warp arrivals (12 converter warps of each CTA): K half converted
+  B_V_FULL = 1,       // [2] CTA 0: 24 warp arrivals: V operand converted
+  B_PV_DONE = 3,      // [2] both CTAs: pair commit after P.V of a tile (its V and P buffers are free)
+  B_S_FULL = 5,       // [2] both CTAs: pair commit after Q.K^T of a tile (S ready, K buffer free)
+  B_S_FREE = 7,       // [2] CTA 0: 8 warp arrivals (4 softmax warps of each CTA hold S in registers)
+  B_P_FULL = 9,       // [2] CTA 0: 8 warp arrivals
+  B_Q_FULL = 11,      // CTA 0: 2 arrivals (the Q loader of each CTA)
+  B_Q_FREE = 12,      // both CTAs: pair commit after the last Q.K^T of a unit
+  B_Q_LOCAL = 13,     // both CTAs: transaction barrier of this CTA's Q tile load
+  B_O_FREE = 14,      // CTA 0: 8 warp arrivals after each CTA's epilogue
+  B_DRAIN = 15,       // CTA 0: one commit from each issuer at exit
+  B_RED = 16,         // [2] softmax warps of this CTA: row-max exchange of a tile (4 warp arrivals)
+  B_REDL = 18,        // softmax warps of this CTA: row-sum exchange at a unit's end (4 warp arrivals)
+  B_EXIT = 19,        // both CTAs: the peer has finished (1 remote arrival)
+  B_SC_FULL = 20,     // [4] scale-folding mode: 12 converter-warp arrivals, a tile's scales are in SSC
+  B_RING_FULL = 24,   // [2] this CTA: the producer's expect_tx arrival + the stage's bulk-copy bytes
+  B_RING_EMPTY = 26,  // [2] this CTA: 12 converter-warp arrivals, the stage has been read
+  NUM_BARS = 28
 };
-static_assert(8 * NUM_BARS <= 240, "barrier block overlaps the scalars after it");
+static_assert(8 * NUM_BARS <= 232, "barrier block overlaps the scalars after it");
+constexpr uint32_t S_MASK = SBAR + 232;      // [2] u32: rows of each ring stage that were copied
 constexpr uint32_t S_TMEM_BASE = SBAR + 240;
 constexpr uint32_t S_ABORT = SBAR + 244;
 
@@ -120,7 +137,12 @@ constexpr uint32_t IDESC_PV = ptx::idesc_bf16_f32(128, 256, false, true);
 constexpr unsigned STATUS_BOUNDS = 1u;
 constexpr unsigned STATUS_TIMEOUT = 2u;
 constexpr unsigned STATUS_LAYOUT = 4u;   // the shared-memory base was not aligned as the fold mode needs
-constexpr uint64_t WAIT_LIMIT_NS = 2000000000ull;   // 2 s per wait
+constexpr uint64_t DEFAULT_WAIT_LIMIT_NS = 2000000000ull;   // 2 s per wait unless the caller sets another
+
+// Test hook (DecodeParams::inject): the Q loader of CTA 1 of cluster 0 withholds its arrival on the
+// first unit's Q_FULL barrier, so the Q.K^T issuer's bounded wait runs out.
+constexpr int INJECT_NONE = 0;
+constexpr int INJECT_SKIP_Q_ARRIVAL = 1;
 
 // Optional per-stage timestamps (build with -DMLA_TRACE): cluster 0 writes %clock64 values to
 // trace[(cta * TRACE_TILES + tile) * TRACE_EVENTS + event] for its first TRACE_TILES tiles.
@@ -146,7 +168,7 @@ struct DecodeParams {
   unsigned long long* trace;       // null unless tracing
   const uint16_t* q;               // bf16 bits [B, T, H, 576]
   const uint8_t* blocks;           // e4m3 [NB, KVD, NL, P, 1, 576]
-  const float* scales;             // fp32 [NSB, KVD, NL, P, 1, 1]
+  const float* scales;             // fp32 [NSB, KVD, NL, P, 1, SG]
   const int32_t* item_start;       // [items + 1] tile prefix
   const int32_t* item_nvis;        // [items] visible keys (clamped)
   const int32_t* cluster_first;    // [NC] first item of each cluster range
@@ -158,6 +180,8 @@ struct DecodeParams {
   float* part_o;                   // [2 NC][128][512]
   float* part_lse;                 // [2 NC][128]
   unsigned int* status;
+  unsigned long long wait_limit_ns;   // bound of every mbarrier wait in the decode kernel
+  int inject;                      // INJECT_NONE, or a test hook that withholds one arrival
   int B, T, H, G, P, KVD, NL, layer, NB, NSB, max_pages, items, NC;
   FastDiv divP, divG, divT;        // by the page size, the head-group count and the query length
   int SG;                          // scales per token (head_dim_granularity): 1, or g with 576 / g % 16 == 0
@@ -240,10 +264,10 @@ __device__ unsigned long long g_trace_marks[8];
 #endif
 
 // Bounded wait on an mbarrier phase (CTA-scope acquire; barriers arrived on by this CTA's threads,
-// by the peer CTA's threads through remote arrives, or by tcgen05 commits).  Returns false when the
-// wait gives up or another role already gave up; the first to give up marks the CTA, its peer and
-// the status word.  The loop is kept small (it is inlined at every wait) and the give-up path is
-// out of line.
+// by the peer CTA's threads through remote arrives, by tcgen05 commits or by bulk-copy bytes).
+// Returns false when the wait gives up or another role already gave up; the first to give up
+// marks the CTA, its peer and the status word.  The loop is kept small (it is inlined at every
+// wait) and the give-up path is out of line.
 __device__ __noinline__ bool wait_gave_up(volatile uint32_t* abort, unsigned int* status, uint32_t peer_abort) {
   if (!*abort) {
     *abort = 1u;
@@ -254,29 +278,36 @@ __device__ __noinline__ bool wait_gave_up(volatile uint32_t* abort, unsigned int
 }
 
 __device__ __forceinline__ bool wait_bar(uint32_t addr, uint32_t parity, volatile uint32_t* abort,
-                                         unsigned int* status, uint32_t peer_abort) {
+                                         unsigned int* status, uint32_t peer_abort, uint64_t limit) {
   if (ptx::mbar_try_wait(addr, parity)) return true;
   const uint64_t t0 = ptx::globaltimer();
   while (!ptx::mbar_try_wait_sleep(addr, parity, 20000u)) {
     if (*abort) return false;
-    if (ptx::globaltimer() - t0 > WAIT_LIMIT_NS) return wait_gave_up(abort, status, peer_abort);
+    if (ptx::globaltimer() - t0 > limit) return wait_gave_up(abort, status, peer_abort);
   }
   return true;
 }
 
-// The same bound, polling instead of suspending in try_wait: the MMA issuers use it because a
-// suspended thread resumes hundreds of cycles after the phase completes, and the issuers sit on
-// the critical path of every tile.
+// The same bound, polling instead of suspending in try_wait: the MMA issuers and the converter's
+// K-buffer wait use it because a suspended thread resumes hundreds of cycles after the phase
+// completes, and those waits sit on the critical path of every tile.
 __device__ __forceinline__ bool poll_bar(uint32_t addr, uint32_t parity, volatile uint32_t* abort,
-                                         unsigned int* status, uint32_t peer_abort) {
+                                         unsigned int* status, uint32_t peer_abort, uint64_t limit) {
   if (ptx::mbar_test_wait(addr, parity)) return true;
   const uint64_t t0 = ptx::globaltimer();
   while (!ptx::mbar_test_wait(addr, parity)) {
     __nanosleep(32);
     if (*abort) return false;
-    if (ptx::globaltimer() - t0 > WAIT_LIMIT_NS) return wait_gave_up(abort, status, peer_abort);
+    if (ptx::globaltimer() - t0 > limit) return wait_gave_up(abort, status, peer_abort);
   }
   return true;
+}
+
+// Time-bounded wait that ignores the abort flag: for the completion of this CTA's own bulk copies
+// and TMA loads before it exits (they land whatever the other roles did).
+__device__ __forceinline__ void drain_bar(uint32_t addr, uint32_t parity, uint64_t limit) {
+  const uint64_t t0 = ptx::globaltimer();
+  while (!ptx::mbar_try_wait(addr, parity) && ptx::globaltimer() - t0 < limit) {}
 }
 
 // ---------------------------------------------------------------------------------------------
@@ -319,268 +350,66 @@ __device__ __forceinline__ void exact16(uint4 raw, uint32_t (&w)[8]) {
   }
 }
 
+template <bool FOLD>
+__device__ __forceinline__ void convert16(bool ok, uint4 raw, float s, uint32_t (&w)[8]) {
+  if (ok) {
+    if (FOLD) {
+      exact16(raw, w);
+    } else {
+      dequant16(raw, s, w);
+    }
+  } else {
+#pragma unroll
+    for (int x = 0; x < 8; ++x) w[x] = 0u;
+  }
+}
+
 // Byte offset of 16-byte unit `u` (0..7) of row `r` in a K-major SWIZZLE_128B atom column whose
 // 8-row groups are 1024 B apart.
 __device__ __forceinline__ uint32_t sw128_off(int r, int u) {
   return (r >> 3) * 1024 + (r & 7) * 128 + ((u ^ (r & 7)) << 4);
 }
 
-__device__ __forceinline__ void st_chunk(uint32_t atom_base, int row, int u0, const uint32_t (&w)[8]) {
-  ptx::st_shared_v4(atom_base + sw128_off(row, u0), w[0], w[1], w[2], w[3]);
-  ptx::st_shared_v4(atom_base + sw128_off(row, u0 + 1), w[4], w[5], w[6], w[7]);
+// One 16-dim chunk (32 bytes of bf16) at chunk position cq (0..3) of an atom column's row.
+__device__ __forceinline__ void st_chunk(uint32_t atom_base, int row, int cq, const uint32_t (&w)[8]) {
+  ptx::st_shared_v4(atom_base + sw128_off(row, 2 * cq), w[0], w[1], w[2], w[3]);
+  ptx::st_shared_v4(atom_base + sw128_off(row, 2 * cq + 1), w[4], w[5], w[6], w[7]);
 }
 
-// Converter thread t (of 256) owns key row conv_row(t) (0..31) of both key halves and the 16-byte
-// chunks conv_q(t) + 8k of it.  Each group of 8 consecutive threads (one phase of a 16-byte shared
-// store) covers chunk slots 0..3 of two adjacent rows, so that its 8 stores land on 8 different
-// 16-byte positions of the 128-byte swizzle row (even rows on even positions, odd rows on odd
-// ones); each warp still reads 4 whole rows (coalesced).
-__device__ __forceinline__ int conv_row(int t) { return ((t >> 4) << 1) | ((t >> 2) & 1); }
-__device__ __forceinline__ int conv_q(int t) { return (t & 3) | (((t >> 3) & 1) << 2); }
+// Converter thread layout.  Thread t (0..383) is in group q = t / 128; thread tau = t % 128 of a
+// group owns key row conv_row(tau) (0..31) and chunk position conv_cq(tau) (0..3) of each 64-dim
+// atom column the group handles.  The 8 threads of one 16-byte shared-memory phase cover the 4
+// chunk positions of two adjacent rows, so their stores land on 8 different 16-byte positions of
+// the 128-byte swizzle row (even rows on even positions, odd rows on odd ones), and their 16-byte
+// reads of the FP8 ring (576-byte rows: adjacent rows start 16 banks apart) hit 8 distinct bank
+// quads.
+__device__ __forceinline__ int conv_row(int tau) { return ((tau >> 3) << 1) | ((tau >> 2) & 1); }
+__device__ __forceinline__ int conv_cq(int tau) { return tau & 3; }
 
-// The FP8 bytes of one tile that one converter thread converts: of row conv_row(t) and chunks
-// conv_q(t) + 8k,
-//   own key   32c + row    : the 36 chunks of its 576-byte row (576 dims) -> K half buffer; its D_c
-//                            chunks also -> V buffer
-//   other key 32(1-c) + row: the 16 chunks of D_c -> V buffer
-// Register slot s (0..4) of RawTile::own holds chunk conv_q(t) + 8 * own_k(s, c) of the own key:
-// slot 0 the chunk past dim 512 (k = 4; only threads with conv_q(t) < 4 have one), slots 1 and 2 the
-// two chunks outside D_c, slots 3 and 4 the two inside D_c (k = c and 2 + c).  With this order the
-// converter finds the V chunks in fixed registers whichever CTA of the pair it runs in, so both CTAs
-// run the same code.
-__device__ __forceinline__ int own_k(int s, int c) {
-  return s == 0 ? 4 : s == 1 ? 1 - c : s == 2 ? 3 - c : s == 3 ? c : 2 + c;
-}
+// V atom column va (0..3) of CTA c's V operand holds the 64 dims of absolute atom column
+// v_atom(va, c) (D_c = atom columns 2c, 2c+1, 4+2c, 5+2c); a K atom column a belongs to D_c when
+// it is one of these, at V atom column k_to_v(a, c).
+__device__ __forceinline__ int v_atom(int va, int c) { return va < 2 ? 2 * c + va : 4 + 2 * c + (va - 2); }
+__device__ __forceinline__ bool k_in_dc(int a, int c) { return a < 8 && ((a >> 1) == c || (a >> 1) == 2 + c); }
+__device__ __forceinline__ int k_to_v(int a, int c) { return ((a >> 1) == c) ? (a & 1) : 2 + (a & 1); }
 
-// With per-token scales (BS = false) only so[0] and sp[0] are used; with block scales (BS = true,
-// head_dim_granularity g > 1) each register slot carries the scale of its chunk's block, scale
-// index = chunk / (36 / g).
-struct RawTile {
-  uint4 own[5];
-  uint4 oth[2];
-  float so[5], sp[2];
-  bool own_ok, oth_ok;
-};
-
-// Three phases so that the page-table reads and the data reads of later tiles overlap the
-// conversion of the current one:
-//   lut_issue : read the page-table entries of thread t's two keys of tile j (request b)
-//   lut_finish: turn them into row pointers (ids past the pool are flagged; that key reads as zero)
-//   fetch     : issue the 16-byte loads of those rows and their scales
-struct LutVals {
-  uint32_t ob, osb, pb, psb;       // value / scale block ids of the own and other key
-  uint32_t oslot, pslot;           // slots of the two keys within their pages
-  uint32_t flags;                  // LV_OWN_IN | LV_OTH_IN (key visible, page inside the table) | LV_BAD
-};
-constexpr uint32_t LV_OWN_IN = 1u, LV_OTH_IN = 2u, LV_BAD = 4u;
-
-struct TilePtrs {                 // row indices into blocks / scales (both < 2^32, checked on the host)
-  uint32_t ov, os, pv, ps;
-  bool own_ok, oth_ok;
-};
-
-__device__ __forceinline__ LutVals lut_issue(const DecodeParams& p, int c, int t, int b, int nvis, int j) {
-  const int row = conv_row(t);
-  LutVals V;
-  const int otok = j * BN + HALF_BN * c + row;
-  const int ptok = j * BN + HALF_BN * (1 - c) + row;
-  const uint32_t* lrow = p.lut + static_cast<size_t>(b) * p.max_pages;
-  const uint32_t* srow = p.slut ? p.slut + static_cast<size_t>(b) * p.max_pages : lrow;
-  const int opage = static_cast<int>(p.divP.div(otok)), ppage = static_cast<int>(p.divP.div(ptok));
-  V.oslot = static_cast<uint32_t>(otok - opage * p.P);
-  V.pslot = static_cast<uint32_t>(ptok - ppage * p.P);
-  uint32_t f = 0;
-  if (otok < nvis) f |= (opage < p.max_pages) ? LV_OWN_IN : LV_BAD;
-  if (ptok < nvis) f |= (ppage < p.max_pages) ? LV_OTH_IN : LV_BAD;
-  V.flags = f;
-  V.ob = V.osb = V.pb = V.psb = 0;
-  if (f & LV_OWN_IN) { V.ob = __ldg(lrow + opage); V.osb = __ldg(srow + opage); }
-  if (f & LV_OTH_IN) { V.pb = __ldg(lrow + ppage); V.psb = __ldg(srow + ppage); }
-  return V;
-}
-
-__device__ __forceinline__ TilePtrs lut_finish(const DecodeParams& p, const LutVals& V, bool& bad) {
-  TilePtrs T;
-  const bool own_in = (V.flags & LV_OWN_IN) != 0, oth_in = (V.flags & LV_OTH_IN) != 0;
-  T.own_ok = own_in && V.ob < static_cast<uint32_t>(p.NB) && V.osb < static_cast<uint32_t>(p.NSB);
-  T.oth_ok = oth_in && V.pb < static_cast<uint32_t>(p.NB) && V.psb < static_cast<uint32_t>(p.NSB);
-  bad = (V.flags & LV_BAD) != 0 || (own_in && !T.own_ok) || (oth_in && !T.oth_ok);
-  const uint32_t per_blk = static_cast<uint32_t>(p.KVD * p.NL * p.P);
-  const uint32_t lay = static_cast<uint32_t>(p.layer * p.P);
-  T.ov = V.ob * per_blk + lay + V.oslot;
-  T.os = V.osb * per_blk + lay + V.oslot;
-  T.pv = V.pb * per_blk + lay + V.pslot;
-  T.ps = V.psb * per_blk + lay + V.pslot;
-  return T;
-}
-
-// A tile's bytes are fetched in parts: register slots [S0, S1) of the own key, and the other key's
-// chunks.  With one scale per token, slot 0 also brings both keys' scales (so that they arrive
-// early); with block scales each chunk brings its own.  The converter reloads each part right
-// after it has converted that part of the current tile (see converter_role).
-template <int S0, int S1, bool BS>
-__device__ __forceinline__ void fetch_own_part(const DecodeParams& p, const TilePtrs& T, int c, int t, RawTile& R) {
-  const int q = conv_q(t);
-  R.own_ok = T.own_ok;
-  if (!BS && S0 == 0 && T.oth_ok) R.sp[0] = __ldg(p.scales + T.ps);
-  if (T.own_ok) {
-    const uint8_t* ov = p.blocks + static_cast<size_t>(T.ov) * HEAD_DIM;
-    if (!BS && S0 == 0) R.so[0] = __ldg(p.scales + T.os);
-#pragma unroll
-    for (int sl = S0; sl < S1; ++sl) {
-      const int qq = q + 8 * own_k(sl, c);
-      if (qq < 36) {
-        R.own[sl] = ptx::ldg_stream_v4(ov + 16 * qq);
-        if (BS) R.so[sl] = __ldg(p.scales + static_cast<size_t>(T.os) * p.SG + p.divCPB.div(qq));
-      }
-    }
-  }
-}
-
-template <bool BS>
-__device__ __forceinline__ void fetch_oth(const DecodeParams& p, const TilePtrs& T, int c, int t, RawTile& R) {
-  const int q = conv_q(t);
-  R.oth_ok = T.oth_ok;
-  if (T.oth_ok) {
-    const uint8_t* pv = p.blocks + static_cast<size_t>(T.pv) * HEAD_DIM;
-#pragma unroll
-    for (int k = 0; k < 2; ++k) {
-      const int jc = q + 8 * k;                              // chunk index within D_c (0..15)
-      const int qq = jc < 8 ? 8 * c + jc : 16 + 8 * c + (jc - 8);
-      R.oth[k] = ptx::ldg_stream_v4(pv + 16 * qq);
-      if (BS) R.sp[k] = __ldg(p.scales + static_cast<size_t>(T.ps) * p.SG + p.divCPB.div(qq));
-    }
-  }
-}
-
-template <bool BS>
-__device__ __forceinline__ void fetch(const DecodeParams& p, const TilePtrs& T, int c, int t, RawTile& R) {
-  fetch_own_part<0, 5, BS>(p, T, c, t, R);
-  fetch_oth<BS>(p, T, c, t, R);
-}
-
-// All three phases at once (for callers with nothing to overlap).  Returns false on a bad page id.
-template <bool BS>
-__device__ __forceinline__ bool load_tile(const DecodeParams& p, int c, int t, int b, int nvis, int j, RawTile& R) {
-  bool bad;
-  const TilePtrs T = lut_finish(p, lut_issue(p, c, t, b, nvis, j), bad);
-  fetch<BS>(p, T, c, t, R);
-  return !bad;
-}
-
-// Dequantises thread t's part of a loaded tile into the K half buffer `sk` and the V buffer `sv`.
-template <bool BS>
-__device__ __forceinline__ void store_tile(int c, int t, const RawTile& R, uint32_t sk, uint32_t sv) {
-  const int row = conv_row(t), q = conv_q(t);
-  const int vrow_own = HALF_BN * c + row;
-  const int vrow_oth = HALF_BN * (1 - c) + row;
-#pragma unroll
-  for (int sl = 0; sl < 5; ++sl) {
-    const int qq = q + 8 * own_k(sl, c);                     // chunk of the 576-byte row
-    if (qq >= 36) continue;
-    uint32_t w[8];
-    if (R.own_ok) {
-      dequant16(R.own[sl], R.so[BS ? sl : 0], w);
-    } else {
-#pragma unroll
-      for (int x = 0; x < 8; ++x) w[x] = 0u;
-    }
-    st_chunk(sk + (qq >> 2) * SK_ATOM, row, (qq & 3) * 2, w);
-    if (sl >= 3) {                                           // D_c chunk: V chunk q (slot 3) or q + 8 (slot 4)
-      const int jc = q + (sl == 4 ? 8 : 0);
-      st_chunk(sv + (jc >> 2) * SV_ATOM, vrow_own, (jc & 3) * 2, w);
-    }
-  }
-#pragma unroll
-  for (int k = 0; k < 2; ++k) {
-    const int jc = q + 8 * k;
-    uint32_t w[8];
-    if (R.oth_ok) {
-      dequant16(R.oth[k], R.sp[BS ? k : 0], w);
-    } else {
-#pragma unroll
-      for (int x = 0; x < 8; ++x) w[x] = 0u;
-    }
-    st_chunk(sv + (jc >> 2) * SV_ATOM, vrow_oth, (jc & 3) * 2, w);
-  }
-}
-
-// The decode's converter writes the two operands of a tile at different times: the K half as soon
-// as its buffer is free (store_k_part), the V operand once P.V two tiles back has finished
-// (store_v).  store_k_part converts own-key slots [S0, S1); it keeps the two chunks that also
-// belong to the V operand (slots 3 and 4: V chunks q and q + 8) so that store_v need not convert
-// them again.  The tile's flags and per-token scales come as arguments because the registers of
-// R are being refilled with the next tile while this one is converted.
-template <int S0, int S1, bool BS, bool FOLD>
-__device__ __forceinline__ void store_k_part(int c, int t, const RawTile& R, bool own_ok, float s_own, uint32_t sk,
-                                             uint32_t (&keep0)[8], uint32_t (&keep1)[8]) {
-  const int row = conv_row(t), q = conv_q(t);
-#pragma unroll
-  for (int sl = S0; sl < S1; ++sl) {
-    const int qq = q + 8 * own_k(sl, c);
-    if (qq >= 36) continue;
-    uint32_t w[8];
-    if (own_ok) {
-      if (FOLD) {
-        exact16(R.own[sl], w);
-      } else {
-        dequant16(R.own[sl], BS ? R.so[sl] : s_own, w);
-      }
-    } else {
-#pragma unroll
-      for (int x = 0; x < 8; ++x) w[x] = 0u;
-    }
-    st_chunk(sk + (qq >> 2) * SK_ATOM, row, (qq & 3) * 2, w);
-    if (sl == 3) {
-#pragma unroll
-      for (int x = 0; x < 8; ++x) keep0[x] = w[x];
-    }
-    if (sl == 4) {
-#pragma unroll
-      for (int x = 0; x < 8; ++x) keep1[x] = w[x];
-    }
-  }
-}
-
-template <bool BS, bool FOLD>
-__device__ __forceinline__ void store_v(int c, int t, const RawTile& R, bool oth_ok, float s_oth,
-                                        const uint32_t (&keep0)[8], const uint32_t (&keep1)[8], uint32_t sv) {
-  const int row = conv_row(t), q = conv_q(t);
-  const int vrow_own = HALF_BN * c + row;
-  const int vrow_oth = HALF_BN * (1 - c) + row;
-  st_chunk(sv + (q >> 2) * SV_ATOM, vrow_own, (q & 3) * 2, keep0);
-  st_chunk(sv + ((q + 8) >> 2) * SV_ATOM, vrow_own, (q & 3) * 2, keep1);
-#pragma unroll
-  for (int k = 0; k < 2; ++k) {
-    const int jc = q + 8 * k;
-    uint32_t w[8];
-    if (oth_ok) {
-      if (FOLD) {
-        exact16(R.oth[k], w);
-      } else {
-        dequant16(R.oth[k], BS ? R.sp[k] : s_oth, w);
-      }
-    } else {
-#pragma unroll
-      for (int x = 0; x < 8; ++x) w[x] = 0u;
-    }
-    st_chunk(sv + (jc >> 2) * SV_ATOM, vrow_oth, (jc & 3) * 2, w);
-  }
-}
+// The group that also converts V atom column 3 of the other CTA's keys (balances the work: that
+// group owns no or only one of the CTA's own D_c atom columns).
+__device__ __forceinline__ int extra_group(int c) { return c == 0 ? 2 : 0; }
 
 // Request index of an item (items are ordered (b, i, g)).
 __device__ __forceinline__ int item_b(const DecodeParams& p, int item) {
   return static_cast<int>(p.divT.div(p.divG.div(item)));
 }
 
-// What the converter needs to know about one tile (request, query token and head group follow
-// from the item index).
+// What the converter and the producer need to know about one tile (request, query token and head
+// group follow from the item index).
 struct TileInfo {
   int item, nvis, j;
   bool first, valid;
 };
 
-// Produces the tile sequence of a cluster one TileInfo at a time (a lighter TileCursor).
+// Produces the tile sequence of a cluster one TileInfo at a time.
 struct TileStream {
   UnitWalker wk;
   int item, nvis, j, te;
@@ -633,15 +462,155 @@ struct TileCursor {
   }
 };
 
+// Page-table lookup of one key: value row and scale row (indices into blocks / scales as
+// [rows][576] and [rows][SG]; both < 2^32, checked on the host).  Returns false (and sets `bad`)
+// for a page past the table or an id past its pool; the key then reads as zero.
+__device__ __forceinline__ bool key_rows(const DecodeParams& p, int b, int tok, uint32_t& vrow, uint32_t& srow,
+                                         bool& bad) {
+  const uint32_t page = p.divP.div(static_cast<uint32_t>(tok));
+  const uint32_t slot = static_cast<uint32_t>(tok) - page * static_cast<uint32_t>(p.P);
+  if (page >= static_cast<uint32_t>(p.max_pages)) {
+    bad = true;
+    return false;
+  }
+  const size_t e = static_cast<size_t>(b) * p.max_pages + page;
+  const uint32_t blk = __ldg(p.lut + e);
+  const uint32_t sblk = p.slut ? __ldg(p.slut + e) : blk;
+  if (blk >= static_cast<uint32_t>(p.NB) || sblk >= static_cast<uint32_t>(p.NSB)) {
+    bad = true;
+    return false;
+  }
+  const uint32_t per_blk = static_cast<uint32_t>(p.KVD * p.NL * p.P);
+  const uint32_t lay = static_cast<uint32_t>(p.layer * p.P);
+  vrow = blk * per_blk + lay + slot;
+  srow = sblk * per_blk + lay + slot;
+  return true;
+}
+
+// ---------------------------------------------------------------------------------------------
+// Producer side of one ring stage: the page runs of the `n` keys starting at token tok0 of request
+// b (at most two runs: page sizes are multiples of 16 and a half tile is 32 keys), each one bulk
+// copy of its rows into stage rows [r0, r0 + len) and, with per-token scales (SC), one bulk copy of
+// their scales (rounded up to whole 16-byte units, which stays inside the page).  Writes the mask of
+// copied rows to `mask_addr`, then arrives on `full` with the byte count and issues the copies.
+// ---------------------------------------------------------------------------------------------
+template <bool SC>
+__device__ __forceinline__ void issue_half_tile(const DecodeParams& p, uint32_t stage, uint32_t full,
+                                                uint32_t mask_addr, int b, int tok0, int n) {
+  bool bad = false;
+  uint32_t mask = 0, tx = 0;
+  // first run: from tok0 to the end of its page (or of the half tile)
+  const int len0 = min(n, p.P - static_cast<int>(p.divP.mod(static_cast<uint32_t>(tok0))));
+  uint32_t v0 = 0, s0 = 0, v1 = 0, s1 = 0;
+  const bool ok0 = n > 0 && key_rows(p, b, tok0, v0, s0, bad);
+  // second run: the rest, which starts on a page boundary and is at most 16 <= P keys long
+  const int len1 = n - max(len0, 0);
+  const bool ok1 = len1 > 0 && key_rows(p, b, tok0 + len0, v1, s1, bad);
+  if (ok0) {
+    mask |= (len0 >= 32 ? 0xFFFFFFFFu : ((1u << len0) - 1u));
+    tx += static_cast<uint32_t>(len0) * HEAD_DIM + (SC ? ((static_cast<uint32_t>(len0) + 3u) & ~3u) * 4u : 0u);
+  }
+  if (ok1) {
+    mask |= ((1u << len1) - 1u) << len0;
+    tx += static_cast<uint32_t>(len1) * HEAD_DIM + (SC ? ((static_cast<uint32_t>(len1) + 3u) & ~3u) * 4u : 0u);
+  }
+  if (bad) raise_status(p.status, STATUS_BOUNDS);
+  ptx::st_shared_u32(mask_addr, mask);
+  ptx::mbar_arrive_expect_tx(full, tx);
+  if (ok0) {
+    ptx::bulk_load(stage, p.blocks + static_cast<size_t>(v0) * HEAD_DIM, static_cast<uint32_t>(len0) * HEAD_DIM, full);
+    if (SC) ptx::bulk_load(stage + RING_ROWS, p.scales + s0, ((static_cast<uint32_t>(len0) + 3u) & ~3u) * 4u, full);
+  }
+  if (ok1) {
+    const uint32_t r1 = static_cast<uint32_t>(len0);
+    ptx::bulk_load(stage + r1 * HEAD_DIM, p.blocks + static_cast<size_t>(v1) * HEAD_DIM,
+                   static_cast<uint32_t>(len1) * HEAD_DIM, full);
+    if (SC) ptx::bulk_load(stage + RING_ROWS + 4u * r1, p.scales + s1, ((static_cast<uint32_t>(len1) + 3u) & ~3u) * 4u, full);
+  }
+}
+
+// Values a converter thread loads one tile ahead from global memory: the other CTA's key's D_c
+// chunks (V atom column = its group, and V atom column 3 for the extra group) with their scales,
+// and in the block-scale mode the scales of its own key's three K chunks.
+struct Ahead {
+  uint4 oth[2];
+  float s_oth[2];
+  float s_own[3];
+  bool oth_ok, own_ok;
+};
+
+template <bool BS>
+__device__ __forceinline__ bool load_ahead(const DecodeParams& p, const TileInfo& ti, int c, int grp, int r, int cq,
+                                           bool extra, Ahead& A) {
+  bool bad = false;
+  const int b = item_b(p, ti.item);
+  const int tok = ti.j * BN + HALF_BN * (1 - c) + r;
+  uint32_t vrow = 0, srow = 0;
+  A.oth_ok = tok < ti.nvis && key_rows(p, b, tok, vrow, srow, bad);
+  if (A.oth_ok) {
+    const uint8_t* row = p.blocks + static_cast<size_t>(vrow) * HEAD_DIM;
+    const int q0 = 4 * v_atom(grp, c) + cq;
+    A.oth[0] = ptx::ldg_stream_v4(row + 16 * q0);
+    if (BS) A.s_oth[0] = __ldg(p.scales + static_cast<size_t>(srow) * p.SG + p.divCPB.div(q0));
+    else A.s_oth[0] = __ldg(p.scales + srow);
+    if (extra) {
+      const int q1 = 4 * v_atom(3, c) + cq;
+      A.oth[1] = ptx::ldg_stream_v4(row + 16 * q1);
+      A.s_oth[1] = BS ? __ldg(p.scales + static_cast<size_t>(srow) * p.SG + p.divCPB.div(q1)) : A.s_oth[0];
+    }
+  }
+  if (BS) {
+    const int otok = ti.j * BN + HALF_BN * c + r;
+    uint32_t ov = 0, os = 0;
+    A.own_ok = otok < ti.nvis && key_rows(p, b, otok, ov, os, bad);
+    if (A.own_ok) {
+#pragma unroll
+      for (int m = 0; m < 3; ++m)
+        A.s_own[m] = __ldg(p.scales + static_cast<size_t>(os) * p.SG + p.divCPB.div(4 * (3 * grp + m) + cq));
+    }
+  } else {
+    A.own_ok = true;
+  }
+  return !bad;
+}
+
+// K-half part of one tile for a converter thread: its three chunks of the own key's row, read from
+// a ring stage (raw) and dequantised into the K half buffer at `sk`.
+template <bool BS, bool FOLD>
+__device__ __forceinline__ void convert_k(int grp, int r, int cq, bool ok, const uint4 (&raw)[3], float s_tok,
+                                          const float (&s_blk)[3], uint32_t sk, int c, uint32_t (&keep0)[8],
+                                          uint32_t (&keep1)[8], int& va0, int& va1) {
+  int nd = 0;
+  va0 = va1 = -1;
+#pragma unroll
+  for (int m = 0; m < 3; ++m) {
+    const int a = 3 * grp + m;
+    uint32_t w[8];
+    convert16<FOLD>(ok, raw[m], BS ? s_blk[m] : s_tok, w);
+    st_chunk(sk + a * SK_ATOM, r, cq, w);
+    if (k_in_dc(a, c)) {
+      if (nd == 0) {
+#pragma unroll
+        for (int x = 0; x < 8; ++x) keep0[x] = w[x];
+        va0 = k_to_v(a, c);
+      } else {
+#pragma unroll
+        for (int x = 0; x < 8; ++x) keep1[x] = w[x];
+        va1 = k_to_v(a, c);
+      }
+      ++nd;
+    }
+  }
+}
+
 // =============================================================================================
-// converter role (warps 0-7); the same code in both CTAs of the pair (c = rank).
-// Software pipeline over the tile sequence with one set of tile registers R: each part of R (own-key
-// slots 0-2, own-key slots 3-4, other-key chunks) is refilled with tile g+1's bytes right after tile
-// g's copy of that part has been converted, so every load has a whole tile period to arrive and no
-// register is copied between tiles.  The page-table entries of tile g+2 are read meanwhile.
-// Buffers alternate by tile parity; the K half of tile g waits for Q.K^T(g-2) (S_FULL), the V
-// operand for P.V(g-2).  Returns early (with the abort flag set by the failing wait) when a wait
-// gives up.
+// converter role (warps 0-11); the same code in both CTAs of the pair (c = rank).
+// Per tile g: read the thread's three FP8 chunks and the own key's scale from ring stage g % 2 and
+// release the stage; once Q.K^T(g-1) has finished (the K half buffer is free) dequantise them into
+// it; once P.V(g-2) has finished (V buffer g % 2 is free) write the V operand: the kept own-key
+// D_c chunks and the other key's D_c chunks (loaded from global memory during tile g-1).  Then
+// load the other key's chunks of tile g+1.  Returns early (with the abort flag set by the failing
+// wait) when a wait gives up.
 // =============================================================================================
 template <int MODE>
 __device__ __forceinline__ void converter_role(const DecodeParams& p, int k, uint32_t base, int lane,
@@ -650,86 +619,116 @@ __device__ __forceinline__ void converter_role(const DecodeParams& p, int k, uin
   constexpr bool FOLD = MODE == SCALE_FOLD;
   const int C = static_cast<int>(c);
   const int t = threadIdx.x;
+  const int grp = t / CONV_GROUP, tau = t % CONV_GROUP;
+  const int r = conv_row(tau), cq = conv_cq(tau);
+  const bool extra = grp == extra_group(C);
+  const uint64_t lim = p.wait_limit_ns;
 #define BAR(i) (base + SBAR + 8u * (i))
 #define MLA_WAIT_RET(b_, parity)                                                               \
-  if (!__all_sync(0xffffffffu, wait_bar((b_), (parity), abort, p.status, peer_abort))) return;
+  if (!__all_sync(0xffffffffu, wait_bar((b_), (parity), abort, p.status, peer_abort, lim))) return;
+#define MLA_POLL_RET(b_, parity)                                                               \
+  if (!__all_sync(0xffffffffu, poll_bar((b_), (parity), abort, p.status, peer_abort, lim))) return;
   const uint32_t k_full0 = ptx::mapa(BAR(B_K_FULL), 0), v_full0 = ptx::mapa(BAR(B_V_FULL), 0);
   TileStream ts(p, k);
   TileInfo cur = ts.take(p);
   if (!cur.valid) return;
-  TileInfo n1 = ts.take(p);
-  TileInfo n2 = ts.take(p);
-  RawTile R;
-  bool bad = false;
-  {
-    const TilePtrs t0 = lut_finish(p, lut_issue(p, C, t, item_b(p, cur.item), cur.nvis, cur.j), bad);
-    if (bad) raise_status(p.status, STATUS_BOUNDS);
-    fetch<BS>(p, t0, C, t, R);
-  }
-  TilePtrs t1{};
-  if (n1.valid) {
-    t1 = lut_finish(p, lut_issue(p, C, t, item_b(p, n1.item), n1.nvis, n1.j), bad);
-    if (bad) raise_status(p.status, STATUS_BOUNDS);
-  }
+  TileInfo nxt = ts.take(p);
+  Ahead A;
+  if (!load_ahead<BS>(p, cur, C, grp, r, cq, extra, A)) raise_status(p.status, STATUS_BOUNDS);
   uint32_t g = 0;
   // Rolled loop (one copy of the step keeps the hot code small).
   while (true) {
-    const uint32_t kb = g & 1, free_par = ((g >> 1) & 1) ^ 1;
-    MLA_WAIT_RET(BAR(B_S_FULL + kb), free_par);
+    const uint32_t st = g & 1;
+    MLA_WAIT_RET(BAR(B_RING_FULL + st), (g >> 1) & 1);
     if (t == 0) MLA_TRACE_EV(g, 1);
-    if (t == 224) MLA_TRACE_EV(g, 26);
-    // tile g's flags and per-token scales (R is refilled with tile g+1 below)
-    const bool own_ok = R.own_ok, oth_ok = R.oth_ok;
-    const float s_own = R.so[0], s_oth = R.sp[0];
+    const uint32_t stage = base + SRING + st * RING_STAGE;
+    const bool own_ok = ((ptx::ld_shared_u32(base + S_MASK + 4 * st) >> r) & 1u) != 0 && A.own_ok;
+    uint4 raw[3];
+#pragma unroll
+    for (int m = 0; m < 3; ++m) raw[m] = ptx::ld_shared_v4(stage + r * HEAD_DIM + 16 * (4 * (3 * grp + m) + cq));
+    const float s_own = BS ? 0.f : ptx::ld_shared_f32(stage + RING_ROWS + 4 * r);
+    __syncwarp();
+    if (lane == 0) ptx::mbar_arrive(BAR(B_RING_EMPTY + st));    // the reads above are ordered before it
+    // K half buffer: free once Q.K^T of the previous tile has finished
+    if (g > 0) MLA_POLL_RET(BAR(B_S_FULL + ((g - 1) & 1)), ((g - 1) >> 1) & 1);
+    if (t == 0) MLA_TRACE_EV(g, 16);
     if (FOLD) {
-      // the tile's 64 per-token scales for the softmax (0 for keys not read)
-      if (conv_q(t) == 0) {
-        const uint32_t sa = base + SSC + (g & 3) * SSC_STRIDE + 4 * conv_row(t);
+      // the tile's 64 per-token scales for the softmax (0 for keys not read); the softmax of tile
+      // g - 4 has read this buffer (it finished before S_FREE(g - 3), which Q.K^T(g - 1) waited for)
+      if (grp == 0 && cq == 0) {
+        const uint32_t sa = base + SSC + (g & 3) * SSC_STRIDE + 4 * r;
         ptx::st_shared_f32(sa + 4 * HALF_BN * C, own_ok ? s_own : 0.f);
-        ptx::st_shared_f32(sa + 4 * HALF_BN * (1 - C), oth_ok ? s_oth : 0.f);
+        ptx::st_shared_f32(sa + 4 * HALF_BN * (1 - C), A.oth_ok ? A.s_oth[0] : 0.f);
       }
       __syncwarp();
       if (lane == 0) ptx::mbar_arrive(BAR(B_SC_FULL + (g & 3)));
     }
     uint32_t keep0[8], keep1[8];
-    const uint32_t sk = base + SK0 + kb * SK_STRIDE;
-    store_k_part<0, 3, BS, FOLD>(C, t, R, own_ok, s_own, sk, keep0, keep1);
-    if (n1.valid) fetch_own_part<0, 3, BS>(p, t1, C, t, R);
-    if (t == 0) MLA_TRACE_EV(g, 16);
-    store_k_part<3, 5, BS, FOLD>(C, t, R, own_ok, s_own, sk, keep0, keep1);
-    if (n1.valid) fetch_own_part<3, 5, BS>(p, t1, C, t, R);
-    LutVals v2{};
-    if (n2.valid) v2 = lut_issue(p, C, t, item_b(p, n2.item), n2.nvis, n2.j);
-    if (t == 0) MLA_TRACE_EV(g, 4);
-    if (t == 224) MLA_TRACE_EV(g, 27);
+    int va0, va1;
+    convert_k<BS, FOLD>(grp, r, cq, own_ok, raw, s_own, A.s_own, base + SK, C, keep0, keep1, va0, va1);
     ptx::fence_proxy_async_smem();
     __syncwarp();
-    if (lane == 0) ptx::mbar_arrive_cluster(k_full0 + 8u * kb);
+    if (lane == 0) ptx::mbar_arrive_cluster(k_full0);
     if (t == 0) MLA_TRACE_EV(g, 5);
-    if (t == 224) MLA_TRACE_EV(g, 28);
-    MLA_WAIT_RET(BAR(B_PV_DONE + kb), free_par);
+    // V operand buffer g % 2: free once P.V(g - 2) has finished
+    MLA_WAIT_RET(BAR(B_PV_DONE + st), ((g >> 1) & 1) ^ 1);
     if (t == 0) MLA_TRACE_EV(g, 6);
-    if (t == 224) MLA_TRACE_EV(g, 29);
-    store_v<BS, FOLD>(C, t, R, oth_ok, s_oth, keep0, keep1, base + SV0 + kb * SV_STRIDE);
+    {
+      const uint32_t sv = base + SV0 + st * SV_STRIDE;
+      const int vrow_own = HALF_BN * C + r, vrow_oth = HALF_BN * (1 - C) + r;
+      if (va0 >= 0) st_chunk(sv + va0 * SV_ATOM, vrow_own, cq, keep0);
+      if (va1 >= 0) st_chunk(sv + va1 * SV_ATOM, vrow_own, cq, keep1);
+      uint32_t w[8];
+      convert16<FOLD>(A.oth_ok, A.oth[0], A.s_oth[0], w);
+      st_chunk(sv + grp * SV_ATOM, vrow_oth, cq, w);
+      if (extra) {
+        convert16<FOLD>(A.oth_ok, A.oth[1], A.s_oth[1], w);
+        st_chunk(sv + 3 * SV_ATOM, vrow_oth, cq, w);
+      }
+    }
     ptx::fence_proxy_async_smem();
     __syncwarp();
-    if (lane == 0) ptx::mbar_arrive_cluster(v_full0 + 8u * kb);
+    if (lane == 0) ptx::mbar_arrive_cluster(v_full0 + 8u * st);
     if (t == 0) MLA_TRACE_EV(g, 2);
-    if (t == 224) MLA_TRACE_EV(g, 30);
-    if (n1.valid) fetch_oth<BS>(p, t1, C, t, R);
-    if (n2.valid) {
-      t1 = lut_finish(p, v2, bad);
-      if (bad) raise_status(p.status, STATUS_BOUNDS);
-    }
-    if (t == 0) MLA_TRACE_EV(g, 7);
-    if (t == 224) MLA_TRACE_EV(g, 31);
     ++g;
-    if (!n1.valid) break;
-    cur = n1;
-    n1 = n2;
-    n2 = ts.take(p);
+    if (!nxt.valid) break;
+    if (!load_ahead<BS>(p, nxt, C, grp, r, cq, extra, A)) raise_status(p.status, STATUS_BOUNDS);
+    if (t == 0) MLA_TRACE_EV(g - 1, 7);
+    cur = nxt;
+    nxt = ts.take(p);
   }
+#undef MLA_POLL_RET
 #undef MLA_WAIT_RET
+#undef BAR
+}
+
+// =============================================================================================
+// producer role (lane 0 of warp 19): walks the cluster's tiles and fills ring stage g % 2 with the
+// own keys' rows (and per-token scales) of tile g once the converters have released the stage.
+// Before returning it waits (bounded, whatever the other roles did) for the copies of the last
+// two stages it armed, so that no bulk copy into this CTA's shared memory is in flight at exit.
+// =============================================================================================
+template <int MODE>
+__device__ __forceinline__ void producer_role(const DecodeParams& p, int k, uint32_t base, volatile uint32_t* abort,
+                                              uint32_t peer_abort, uint32_t c) {
+  constexpr bool SC = MODE != SCALE_BLOCK;
+#define BAR(i) (base + SBAR + 8u * (i))
+  TileStream ts(p, k);
+  uint32_t g = 0;
+  while (true) {
+    const TileInfo ti = ts.take(p);
+    if (!ti.valid) break;
+    const uint32_t st = g & 1;
+    if (!wait_bar(BAR(B_RING_EMPTY + st), ((g >> 1) & 1) ^ 1, abort, p.status, peer_abort, p.wait_limit_ns)) break;
+    if (g < 64 && k == 0) MLA_TRACE_EV(g, 24);
+    const int tok0 = ti.j * BN + HALF_BN * static_cast<int>(c);
+    const int n = max(0, min(HALF_BN, ti.nvis - tok0));
+    issue_half_tile<SC>(p, base + SRING + st * RING_STAGE, BAR(B_RING_FULL + st), base + S_MASK + 4 * st,
+                        item_b(p, ti.item), tok0, n);
+    ++g;
+  }
+  for (uint32_t gd = (g >= 2 ? g - 2 : 0); gd < g; ++gd)
+    drain_bar(BAR(B_RING_FULL + (gd & 1)), (gd >> 1) & 1, p.wait_limit_ns);
 #undef BAR
 }
 
@@ -756,18 +755,21 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) mla_decode_kernel(const __grid
   const int k = static_cast<int>(ptx::cluster_id_x());
   volatile uint32_t* abort = reinterpret_cast<volatile uint32_t*>(smem + S_ABORT);
   const uint32_t peer_abort = ptx::mapa(base + S_ABORT, peer);
+  const uint64_t lim = p.wait_limit_ns;
 #define BAR(i) (base + SBAR + 8u * (i))
   MLA_TRACE_CTA(0);
 
   if (threadIdx.x == 0) {
+    ptx::mbar_init(BAR(B_K_FULL), 2 * CONV_WARPS);
     for (uint32_t i = 0; i < 2; ++i) {
-      ptx::mbar_init(BAR(B_K_FULL + i), 2 * CONV_WARPS);
       ptx::mbar_init(BAR(B_V_FULL + i), 2 * CONV_WARPS);
       ptx::mbar_init(BAR(B_PV_DONE + i), 1);
       ptx::mbar_init(BAR(B_S_FULL + i), 1);
       ptx::mbar_init(BAR(B_S_FREE + i), 8);
       ptx::mbar_init(BAR(B_P_FULL + i), 8);
       ptx::mbar_init(BAR(B_RED + i), 4);
+      ptx::mbar_init(BAR(B_RING_FULL + i), 1);
+      ptx::mbar_init(BAR(B_RING_EMPTY + i), CONV_WARPS);
     }
     ptx::mbar_init(BAR(B_Q_FULL), 2);
     ptx::mbar_init(BAR(B_Q_FREE), 1);
@@ -794,9 +796,9 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) mla_decode_kernel(const __grid
 // Whole-warp roles bail out together so that the warp-collective instructions after a wait never
 // run on a partial warp.
 #define MLA_WAIT_WARP(b_, parity)                                                              \
-  if (!__all_sync(0xffffffffu, wait_bar((b_), (parity), abort, p.status, peer_abort))) goto role_done;
+  if (!__all_sync(0xffffffffu, wait_bar((b_), (parity), abort, p.status, peer_abort, lim))) goto role_done;
 #define MLA_POLL_WARP(b_, parity)                                                              \
-  if (!__all_sync(0xffffffffu, poll_bar((b_), (parity), abort, p.status, peer_abort))) goto role_done;
+  if (!__all_sync(0xffffffffu, poll_bar((b_), (parity), abort, p.status, peer_abort, lim))) goto role_done;
 
   if (warp < CONV_WARPS) {
     // ------------------------------------------------------------------ converter
@@ -1016,7 +1018,9 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) mla_decode_kernel(const __grid
   } else if (warp == Q_WARP) {
     // ------------------------------------------------------------------ Q loader (both CTAs)
     // Per unit: wait until the last Q.K^T of the previous unit has finished, then one TMA load per
-    // 64-dim atom column of the CTA's 64 heads (heads past H read as zero).
+    // 64-dim atom column of the CTA's 64 heads (heads past H read as zero).  The load's own
+    // barrier is always waited for (time-bounded, whatever the other roles did), so no TMA write
+    // into this CTA's shared memory is in flight when it exits.
     if (lane == 0) {
       const uint32_t q_full = ptx::mapa(BAR(B_Q_FULL), 0);
       ptx::prefetch_tmap(&p.tmap_q);
@@ -1024,21 +1028,24 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) mla_decode_kernel(const __grid
       Unit u;
       uint32_t uu = 0;
       while (wk.next(p, u)) {
-        if (!wait_bar(BAR(B_Q_FREE), (uu & 1) ^ 1, abort, p.status, peer_abort)) break;
-        if (uu < 2 && c == 0) MLA_TRACE_EV(uu, 24);
+        if (!wait_bar(BAR(B_Q_FREE), (uu & 1) ^ 1, abort, p.status, peer_abort, lim)) break;
         ptx::mbar_arrive_expect_tx(BAR(B_Q_LOCAL), 9 * SQ_ATOM);
 #pragma unroll 1
         for (int a = 0; a < 9; ++a)
           ptx::tma_load_3d(base + SQ + a * SQ_ATOM, &p.tmap_q, 64 * a, u.g * MROWS + HPC * static_cast<int>(c),
                            u.b * p.T + u.i, BAR(B_Q_LOCAL));
-        if (!wait_bar(BAR(B_Q_LOCAL), uu & 1, abort, p.status, peer_abort)) break;
-        if (uu < 2 && c == 0) MLA_TRACE_EV(uu, 25);
-        ptx::mbar_arrive_cluster(q_full);
+        drain_bar(BAR(B_Q_LOCAL), uu & 1, lim);
+        if (*abort) break;
+        const bool withhold = p.inject == INJECT_SKIP_Q_ARRIVAL && k == 0 && c == 1 && uu == 0;
+        if (!withhold) ptx::mbar_arrive_cluster(q_full);
         ++uu;
       }
       // drain: the last unit's Q_FREE commit lands in this CTA before it exits
-      if (uu > 0) wait_bar(BAR(B_Q_FREE), (uu & 1) ^ 1, abort, p.status, peer_abort);
+      if (uu > 0) wait_bar(BAR(B_Q_FREE), (uu & 1) ^ 1, abort, p.status, peer_abort, lim);
     }
+  } else if (warp == LOAD_WARP) {
+    // ------------------------------------------------------------------ FP8 producer (both CTAs)
+    if (lane == 0) producer_role<MODE>(p, k, base, abort, peer_abort, c);
   } else if (warp == QK_WARP) {
     // ------------------------------------------------------------------ Q.K^T issuer (CTA 0)
     // The whole warp runs the loop (descriptors stay warp-uniform); one elected lane issues.
@@ -1047,21 +1054,21 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) mla_decode_kernel(const __grid
       uint32_t g = 0, uq = 0;
       // descriptor bases; per K step only the start-address field (bits 0..13, bytes >> 4) moves
       const uint64_t dq0 = ptx::smem_desc(base + SQ, 16, 1024, ptx::SW_128B);
-      const uint64_t dk0 = ptx::smem_desc(base + SK0, 16, 1024, ptx::SW_128B);
+      const uint64_t dk0 = ptx::smem_desc(base + SK, 16, 1024, ptx::SW_128B);
       while (qc.valid) {
-        const uint32_t kb = g & 1;
+        const uint32_t sb = g & 1;
         if (qc.first) {
           MLA_POLL_WARP(BAR(B_Q_FULL), uq & 1);
           ++uq;
         }
-        MLA_POLL_WARP(BAR(B_K_FULL + kb), (g >> 1) & 1);
-        MLA_POLL_WARP(BAR(B_S_FREE + kb), ((g >> 1) & 1) ^ 1);
+        MLA_POLL_WARP(BAR(B_K_FULL), g & 1);
+        MLA_POLL_WARP(BAR(B_S_FREE + sb), ((g >> 1) & 1) ^ 1);
         ptx::tc_fence_after();
         if (ptx::elect_one()) {
           MLA_TRACE_EV(g, 20);
-          const uint32_t dS = tbase + T_S + 32 * kb;
+          const uint32_t dS = tbase + T_S + 32 * sb;
           // 9 atom columns of 64 dims x 4 K steps of 16 dims
-          uint64_t ad = dq0, bd = dk0 + ((kb * SK_STRIDE) >> 4);
+          uint64_t ad = dq0, bd = dk0;
 #pragma unroll 1
           for (int a = 0; a < 9; ++a) {
 #pragma unroll
@@ -1070,7 +1077,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) mla_decode_kernel(const __grid
             ad += SQ_ATOM >> 4;
             bd += SK_ATOM >> 4;
           }
-          ptx::mma_commit_pair(BAR(B_S_FULL + kb), 0x3);
+          ptx::mma_commit_pair(BAR(B_S_FULL + sb), 0x3);
           MLA_TRACE_EV(g, 21);
           if (qc.j == qc.u.te - 1) ptx::mma_commit_pair(BAR(B_Q_FREE), 0x3);
         }
@@ -1123,27 +1130,31 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) mla_decode_kernel(const __grid
 role_done:
 #undef MLA_POLL_WARP
 #undef MLA_WAIT_WARP
-  // every pair MMA issued by CTA 0 has finished before TMEM is released
+  // Every pair MMA issued by CTA 0 has finished before TMEM is released.  The commit arrives once
+  // all of the issuer's earlier MMAs are done; the MMAs themselves wait on nothing, so on a normal
+  // or an aborted call this wait ends well inside its bound (it only bounds the spin).
   if (c == 0 && (warp == QK_WARP || warp == PV_WARP) && lane == 0) {
     ptx::mma_commit_pair(BAR(B_DRAIN), 0x1);
-    const uint64_t t0 = ptx::globaltimer();
-    while (!ptx::mbar_try_wait(BAR(B_DRAIN), 0) && ptx::globaltimer() - t0 < WAIT_LIMIT_NS) {}
+    drain_bar(BAR(B_DRAIN), 0, lim);
   }
   ptx::tc_fence_before();
   __syncthreads();
   MLA_TRACE_CTA(2);
   // Exit handshake.  Every cross-CTA arrival and pair-MMA commit has been waited for above, so no
   // remote access can reach a CTA that has exited; the two CTAs still tell each other that they are
-  // done (one remote arrive each) before the pair's TMEM is released.  The wait polls: a thread
-  // suspended in try_wait (or in a cluster barrier) measured ~7 us to resume after the peer's
-  // remote arrival on B200, even with both CTAs arriving together.
+  // done (one remote arrive each) before the pair's TMEM is released.  The arrive releases at
+  // cluster scope, after the CTA barrier above, so every remote arrival this CTA's threads made
+  // earlier (also on an aborted call, where nothing on the peer waited for them) reaches the peer
+  // before the peer can exit.  The wait polls: a thread suspended in try_wait (or in a cluster
+  // barrier) measured ~7 us to resume after the peer's remote arrival on B200, even with both
+  // CTAs arriving together.
   if (threadIdx.x == 0) {
-    ptx::mbar_arrive_remote_relaxed(ptx::mapa(BAR(B_EXIT), peer));
+    ptx::mbar_arrive_remote(ptx::mapa(BAR(B_EXIT), peer));
 #ifdef MLA_TRACE
     if (p.trace) p.trace[2 * TRACE_TILES * TRACE_EVENTS + 4 * blockIdx.x + 1] = ptx::globaltimer();
 #endif
     const uint64_t t0 = ptx::globaltimer();
-    while (!ptx::mbar_test_wait(BAR(B_EXIT), 0) && ptx::globaltimer() - t0 < WAIT_LIMIT_NS) __nanosleep(32);
+    while (!ptx::mbar_test_wait(BAR(B_EXIT), 0) && ptx::globaltimer() - t0 < lim) __nanosleep(32);
   }
   __syncthreads();
 #undef BAR
@@ -1300,14 +1311,15 @@ mla_combine_kernel(const __grid_constant__ DecodeParams p) {
 }
 
 // =============================================================================================
-// gather + dequant kernel (steps A and C alone): one CTA of 256 threads per (request, 64-key tile,
-// key half c).  Runs the decode's converter (load_tile + store_tile) and copies its K-half buffer
-// back out.
+// gather + dequant kernel (steps A and C alone): one CTA of 384 threads per (request, 64-key tile,
+// key half c).  Runs the decode's producer (issue_half_tile: page runs -> one ring stage) and its
+// converter (load_ahead for block scales, convert_k), then copies the K-half buffer back out.
 // =============================================================================================
 constexpr int DQ_THREADS = CONV_THREADS;
 constexpr uint32_t DQ_SK = 0;
-constexpr uint32_t DQ_SV = SK_STRIDE;
-constexpr uint32_t DQ_SMEM_ALLOC = SK_STRIDE + SV_STRIDE + 1024;
+constexpr uint32_t DQ_RING = SK_BYTES;
+constexpr uint32_t DQ_BAR = DQ_RING + RING_STAGE;
+constexpr uint32_t DQ_SMEM_ALLOC = DQ_BAR + 64 + 1024;
 
 template <bool BS>
 __global__ void __launch_bounds__(DQ_THREADS)
@@ -1319,18 +1331,46 @@ mla_dequant_kernel(const __grid_constant__ DecodeParams p, const uint32_t* cache
   const int b = blockIdx.x / tiles_per_req;
   const int j = blockIdx.x % tiles_per_req;
   const int c = blockIdx.y;
+  if (b >= p.B) return;
   const int n = min(static_cast<int>(min(cache_lengths[b], 0x3FFFFFFFu)) + p.T, max_keys);
-  if (j * BN + HALF_BN * c >= n || b >= p.B) return;
-  RawTile R;
-  if (!load_tile<BS>(p, c, threadIdx.x, b, n, j, R)) raise_status(p.status, STATUS_BOUNDS);
-  store_tile<BS>(c, threadIdx.x, R, base + DQ_SK, base + DQ_SV);
+  const int tok0 = j * BN + HALF_BN * c;
+  if (tok0 >= n) return;
+  const int cnt = min(HALF_BN, n - tok0);
+  const uint32_t full = base + DQ_BAR, mask_addr = base + DQ_BAR + 8;
+  if (threadIdx.x == 0) {
+    ptx::mbar_init(full, 1);
+    ptx::fence_mbar_init();
+  }
   __syncthreads();
-  const int nv = min(HALF_BN, n - (j * BN + HALF_BN * c));
+  if (threadIdx.x == 0) issue_half_tile<!BS>(p, base + DQ_RING, full, mask_addr, b, tok0, cnt);
+  const int t = threadIdx.x, grp = t / CONV_GROUP, tau = t % CONV_GROUP;
+  const int r = conv_row(tau), cq = conv_cq(tau);
+  TileInfo ti;
+  ti.item = b * p.T * p.G;
+  ti.nvis = n;
+  ti.j = j;
+  ti.first = true;
+  ti.valid = true;
+  Ahead A;
+  if (!load_ahead<BS>(p, ti, c, grp, r, cq, false, A)) raise_status(p.status, STATUS_BOUNDS);
+  const uint64_t t0 = ptx::globaltimer();
+  bool landed;
+  while (!(landed = ptx::mbar_try_wait(full, 0)) && ptx::globaltimer() - t0 < p.wait_limit_ns) {}
+  if (!landed) raise_status(p.status, STATUS_TIMEOUT);
+  const bool own_ok = landed && ((ptx::ld_shared_u32(mask_addr) >> r) & 1u) != 0 && A.own_ok;
+  uint4 raw[3];
+#pragma unroll
+  for (int m = 0; m < 3; ++m) raw[m] = ptx::ld_shared_v4(base + DQ_RING + r * HEAD_DIM + 16 * (4 * (3 * grp + m) + cq));
+  const float s_own = BS ? 0.f : ptx::ld_shared_f32(base + DQ_RING + RING_ROWS + 4 * r);
+  uint32_t keep0[8], keep1[8];
+  int va0, va1;
+  convert_k<BS, false>(grp, r, cq, own_ok, raw, s_own, A.s_own, base + DQ_SK, c, keep0, keep1, va0, va1);
+  __syncthreads();
   for (int id = threadIdx.x; id < HALF_BN * 72; id += DQ_THREADS) {
     const int row = id / 72, cc = id - row * 72;        // 72 units of 8 bf16 per key
-    if (row >= nv) continue;
+    if (row >= cnt) continue;
     const uint4 v = ptx::ld_shared_v4(base + DQ_SK + (cc >> 3) * SK_ATOM + sw128_off(row, cc & 7));
-    uint16_t* dst = out_k + (static_cast<size_t>(b) * max_keys + j * BN + HALF_BN * c + row) * HEAD_DIM + cc * 8;
+    uint16_t* dst = out_k + (static_cast<size_t>(b) * max_keys + tok0 + row) * HEAD_DIM + cc * 8;
     *reinterpret_cast<uint4*>(dst) = v;
   }
 }

@@ -137,3 +137,28 @@ def test_product_path_fails_loudly_without_library(tmp_path):
             _lib.load(str(tmp_path / "missing.so"))
     finally:
         _lib._lib = saved
+
+
+def test_noalloc_rejects_more_items_than_its_fixed_scratch(lib):
+    """The no-allocation entry holds its plan in a fixed array sized for 65 536 (request, query token,
+    head group) items; one more is refused on the host with the reason, before any CUDA call."""
+    heads = 128
+    too_many = _shape(batch=65537, num_q_heads=heads, max_pages=8)
+
+    def noalloc(shape, T=1):
+        return lib.mla_decode_paged_fp8_noalloc(FAKE, FAKE, FAKE, FAKE, FAKE, None, T, 64, 0, 0.07,
+                                                ctypes.byref(shape), FAKE, None, None)
+    assert noalloc(too_many) == 2
+    msg = lib.mla_last_error_string().decode()
+    assert "65537" in msg and "65536" in msg
+    # the same count reached through query tokens and head groups: 32769 * 2 tokens * 1 group
+    assert noalloc(_shape(batch=32769, num_q_heads=heads, max_pages=8), T=2) == 2
+    assert "65538" in lib.mla_last_error_string().decode()
+
+
+def test_wait_limit_range(lib):
+    """The decode kernel's wait bound is settable within [1 ms, 60 s] (host check only)."""
+    assert lib.mla_set_wait_limit_ns(999_999) == 1
+    assert lib.mla_set_wait_limit_ns(60_000_000_001) == 1
+    assert lib.mla_set_wait_limit_ns(1_000_000) == 0
+    assert lib.mla_set_wait_limit_ns(2_000_000_000) == 0

@@ -121,9 +121,13 @@ def test_decode_config_full_parity(cfg_i):
     check_against(out, lse, ref_out, ref_lse)
 
 
-@pytest.mark.parametrize("cfg_i,reqs,heads", [(2, [0, 77, 127], None), (4, [2], list(range(0, 128, 9)))])
+@pytest.mark.parametrize("cfg_i,reqs,heads", [
+    (2, [int(x) for x in np.linspace(0, 127, 16)], None),     # 16 spread requests, every head
+    (4, [0, 1, 2, 3], None),                                   # the whole long-context workload
+])
 def test_decode_full_size_sampled(cfg_i, reqs, heads):
-    """Full-size configs in the bench's launch configuration, sampled rows against the oracle."""
+    """Full-size configs in the bench's launch configuration against the oracle: config 4 whole
+    (4 requests x 128 heads, 131 073 keys each), config 2 on 16 of its 128 requests."""
     inp = W.make_inputs(W.CONFIGS[cfg_i], device="cuda")
     out, lse = run(inp)
     ref_out, ref_lse = oracle_decode(inp, requests=reqs, heads=heads)
