@@ -21,16 +21,20 @@
 //
 // The FP8 pages reach shared memory through a two-stage ring ("KVLoad2CvtProducer", which stages
 // FP8 tiles in shared memory for converter warps behind a producer): per tile, CTA c's producer
-// bulk-copies its own 32 keys' rows (one contiguous 18 KB run per page) and their per-token
-// scales into a stage, with a full / empty mbarrier pair per stage.
+// bulk-copies its own 32 keys' rows (one contiguous 18 KB run per page) and the per-token scales of
+// all 64 keys into a stage, with a full / empty mbarrier pair per stage.
+//
+// Buffering: K halves are double buffered (K of tile g+1 is converted while Q.K^T(g) runs), the V
+// operand and P are single buffered (V(g) and P(g) are written once P.V(g-1) has finished, while
+// the tensor pipe runs Q.K^T(g+1)).
 //
 // Warp roles per CTA (640 threads):
-//   warps 0-11  converter, three groups of four warps (one warp of each group per scheduler).  Group
-//               q dequantises atom columns 3q..3q+2 (192 dims) of the CTA's own 32 keys from the
-//               ring into the K half buffer (single buffered: written once Q.K^T of the previous
-//               tile has finished), then its share of the V operand (double buffered) once P.V two
-//               tiles back has finished.  The other CTA's keys' D_c bytes are loaded from global
-//               memory (they are in L2: the other CTA's producer brought them) one tile ahead.
+//   warps 0-11  converter, three groups of four warps (one warp of each group per scheduler).  In
+//               step g group q dequantises atom columns 3q..3q+2 (192 dims) of the CTA's own 32
+//               keys of tile g from the ring into K half buffer g % 2 (free once Q.K^T(g-2) has
+//               finished), then writes its share of tile g-1's V operand (once P.V(g-2) has
+//               finished).  The other CTA's keys' D_c bytes are loaded from global memory (they are
+//               in L2: the other CTA's producer brought them) a step ahead.
 //   warps 12-15 softmax: online softmax of the CTA's 64 heads (two lanes per head row), P -> SMEM,
 //               lazy O rescale, epilogue
 //   warp 16     Q.K^T issuer (CTA 0 of the pair; one elected lane issues) and TMEM owner (pair
@@ -66,33 +70,35 @@ static_assert(SM_WARP0 % 4 == 0, "softmax warps must start a warpgroup (TMEM lan
 //      SWIZZLE_128B, one "atom column" = 64 bf16 dims x rows at 128 B, 8-row groups 1024 B apart
 constexpr uint32_t SQ = 0;                       // Q: 9 atom columns x (64 rows x 128 B)
 constexpr uint32_t SQ_ATOM = 8192;
-constexpr uint32_t SK = 9 * SQ_ATOM;             // K half (one buffer): 9 atom columns x (32 rows x 128 B)
+constexpr uint32_t SK0 = 9 * SQ_ATOM;            // K half (2 buffers): 9 atom columns x (32 rows x 128 B)
 constexpr uint32_t SK_ATOM = 4096;
-constexpr uint32_t SK_BYTES = 9 * SK_ATOM;
-constexpr uint32_t SV0 = SK + SK_BYTES;          // V operand (2 buffers): 4 atom columns x (64 rows x 128 B)
+constexpr uint32_t SK_STRIDE = 9 * SK_ATOM;
+constexpr uint32_t SV = SK0 + 2 * SK_STRIDE;     // V operand (1 buffer): 4 atom columns x (64 rows x 128 B)
 constexpr uint32_t SV_ATOM = 8192;
-constexpr uint32_t SV_STRIDE = 4 * SV_ATOM;
-constexpr uint32_t SP0 = SV0 + 2 * SV_STRIDE;    // P (2 buffers): 64 rows x 128 B
-constexpr uint32_t SP_STRIDE = 8192;
-constexpr uint32_t SRING = SP0 + 2 * SP_STRIDE;  // FP8 ring (2 stages): 32 rows x 576 B, then 32 fp32 scales
+constexpr uint32_t SV_BYTES = 4 * SV_ATOM;
+constexpr uint32_t SP = SV + SV_BYTES;           // P (1 buffer): 64 rows x 128 B; epilogue staging
+constexpr uint32_t SP_BYTES = 8192;
+constexpr uint32_t SRING = SP + SP_BYTES;        // FP8 ring (2 stages): 32 rows x 576 B, 32 own + 32 other scales
 constexpr uint32_t RING_ROWS = HALF_BN * HEAD_DIM;
-constexpr uint32_t RING_STAGE = RING_ROWS + HALF_BN * 4;
+constexpr uint32_t RING_OSC = RING_ROWS + HALF_BN * 4;   // the other CTA's keys' scales
+constexpr uint32_t RING_STAGE = RING_OSC + HALF_BN * 4;
 constexpr uint32_t SRED = SRING + 2 * RING_STAGE;   // row-max exchange [2][128] f32, row-sum exchange [128] f32
 constexpr uint32_t SBAR = SRED + 1536;
-constexpr uint32_t SMEM_USED = SBAR + 256;
+constexpr uint32_t SMEM_USED = SBAR + 512;
 constexpr uint32_t SMEM_ALLOC = SMEM_USED + 1024;   // slack for aligning the base
 static_assert(SMEM_ALLOC <= 232448, "shared memory map exceeds 227 KB");
 static_assert(RING_STAGE % 16 == 0 && SRING % 16 == 0, "bulk copies need 16-byte aligned stages");
-// Scale-folding mode only: the per-token scales of the last four tiles ([4][64] f32), handed from
+// Scale-folding mode only: the per-token scales of the last eight tiles ([8][64] f32), handed from
 // the converter to the softmax warps.  It sits after SMEM_USED, inside the alignment slack, with
 // the allocation at the 227 KB limit; the kernel checks that the base needed at most
 // SMEM_FOLD_MAX_PAD bytes of alignment (it needs none when the runtime places dynamic shared
 // memory on a 1 KB boundary) and reports STATUS_LAYOUT otherwise.
 constexpr uint32_t SSC = SMEM_USED;
 constexpr uint32_t SSC_STRIDE = 64 * 4;
+constexpr uint32_t SSC_SLOTS = 8;
 constexpr uint32_t SMEM_ALLOC_FOLD = 232448;
-constexpr uint32_t SMEM_FOLD_MAX_PAD = SMEM_ALLOC_FOLD - SSC - 4 * SSC_STRIDE;
-static_assert(SMEM_ALLOC_FOLD >= SSC + 4 * SSC_STRIDE, "fold scale array does not fit");
+constexpr uint32_t SMEM_FOLD_MAX_PAD = SMEM_ALLOC_FOLD - SSC - SSC_SLOTS * SSC_STRIDE;
+static_assert(SMEM_ALLOC_FOLD >= SSC + SSC_SLOTS * SSC_STRIDE, "fold scale array does not fit");
 
 // How the per-token scale enters the computation.
 enum ScaleMode : int {
@@ -102,34 +108,38 @@ enum ScaleMode : int {
 };
 
 enum Bar : uint32_t {
-  B_K_FULL = 0,       // CTA 0: 24 warp arrivals (12 converter warps of each CTA): K half converted
-  B_V_FULL = 1,       // [2] CTA 0: 24 warp arrivals: V operand converted
-  B_PV_DONE = 3,      // [2] both CTAs: pair commit after P.V of a tile (its V and P buffers are free)
-  B_S_FULL = 5,       // [2] both CTAs: pair commit after Q.K^T of a tile (S ready, K buffer free)
-  B_S_FREE = 7,       // [2] CTA 0: 8 warp arrivals (4 softmax warps of each CTA hold S in registers)
-  B_P_FULL = 9,       // [2] CTA 0: 8 warp arrivals
-  B_Q_FULL = 11,      // CTA 0: 2 arrivals (the Q loader of each CTA)
-  B_Q_FREE = 12,      // both CTAs: pair commit after the last Q.K^T of a unit
-  B_Q_LOCAL = 13,     // both CTAs: transaction barrier of this CTA's Q tile load
-  B_O_FREE = 14,      // CTA 0: 8 warp arrivals after each CTA's epilogue
-  B_DRAIN = 15,       // CTA 0: one commit from each issuer at exit
-  B_RED = 16,         // [2] softmax warps of this CTA: row-max exchange of a tile (4 warp arrivals)
-  B_REDL = 18,        // softmax warps of this CTA: row-sum exchange at a unit's end (4 warp arrivals)
-  B_EXIT = 19,        // both CTAs: the peer has finished (1 remote arrival)
-  B_SC_FULL = 20,     // [4] scale-folding mode: 12 converter-warp arrivals, a tile's scales are in SSC
-  B_RING_FULL = 24,   // [2] this CTA: the producer's expect_tx arrival + the stage's bulk-copy bytes
-  B_RING_EMPTY = 26,  // [2] this CTA: 12 converter-warp arrivals, the stage has been read
-  NUM_BARS = 28
+  B_K_FULL = 0,       // [2] CTA 0: 24 warp arrivals (12 converter warps of each CTA): K half converted
+  B_V_FULL = 2,       // [2] CTA 0: 24 warp arrivals: V operand converted (alternates by tile parity)
+  B_PV_DONE = 4,      // [2] both CTAs: pair commit after P.V of a tile (the V and P buffers are free)
+  B_S_FULL = 6,       // [2] both CTAs: pair commit after Q.K^T of a tile (S ready, its K buffer free)
+  B_S_FREE = 8,       // [2] CTA 0: 8 warp arrivals (4 softmax warps of each CTA hold S in registers)
+  B_P_FULL = 10,      // [2] CTA 0: 8 warp arrivals (alternates by tile parity)
+  B_Q_FULL = 12,      // CTA 0: 2 arrivals (the Q loader of each CTA)
+  B_Q_FREE = 13,      // both CTAs: pair commit after the last Q.K^T of a unit
+  B_Q_LOCAL = 14,     // both CTAs: transaction barrier of this CTA's Q tile load
+  B_O_FREE = 15,      // CTA 0: 8 warp arrivals after each CTA's epilogue
+  B_DRAIN = 16,       // CTA 0: one commit from each issuer at exit
+  B_RED = 17,         // [2] softmax warps of this CTA: row-max exchange of a tile (4 warp arrivals)
+  B_REDL = 19,        // softmax warps of this CTA: row-sum exchange at a unit's end (4 warp arrivals)
+  B_EXIT = 20,        // both CTAs: the peer has finished (1 remote arrival)
+  B_RING_FULL = 21,   // [2] this CTA: the producer's expect_tx arrival + the stage's bulk-copy bytes
+  B_RING_EMPTY = 23,  // [2] this CTA: 12 converter-warp arrivals, the stage has been read
+  B_SC_FULL = 25,     // [8] scale-folding mode: 12 converter-warp arrivals, a tile's scales are in SSC
+  NUM_BARS = 33
 };
-static_assert(8 * NUM_BARS <= 232, "barrier block overlaps the scalars after it");
-constexpr uint32_t S_MASK = SBAR + 232;      // [2] u32: rows of each ring stage that were copied
-constexpr uint32_t S_TMEM_BASE = SBAR + 240;
-constexpr uint32_t S_ABORT = SBAR + 244;
+static_assert(8 * NUM_BARS <= 480, "barrier block overlaps the scalars after it");
+constexpr uint32_t S_MASK = SBAR + 480;      // [2][2] u32: per ring stage, own rows copied, other scales copied
+constexpr uint32_t S_TMEM_BASE = SBAR + 496;
+constexpr uint32_t S_ABORT = SBAR + 500;
 
 // TMEM columns (pair layout)
 constexpr uint32_t T_O = 0;                      // P.V halves: cols 0..127 (dims 0..255), 128..255 (256..511)
 constexpr uint32_t T_S = 256;                    // + 32 * buffer
+constexpr uint32_t T_Q = 320;                    // Q dims 0..383 (atom columns 0..5), 2 bf16 per column,
+                                                 // head row r in lanes r and r + 64
+constexpr int Q_TMEM_ATOMS = 6;
 constexpr uint32_t TMEM_COLS = 512;
+static_assert(T_Q + 32 * Q_TMEM_ATOMS <= TMEM_COLS, "tensor memory map overflows");
 
 constexpr uint32_t IDESC_QK = ptx::idesc_bf16_f32(128, BN, false, false);
 constexpr uint32_t IDESC_PV = ptx::idesc_bf16_f32(128, 256, false, true);
@@ -147,7 +157,7 @@ constexpr int INJECT_SKIP_Q_ARRIVAL = 1;
 // Optional per-stage timestamps (build with -DMLA_TRACE): cluster 0 writes %clock64 values to
 // trace[(cta * TRACE_TILES + tile) * TRACE_EVENTS + event] for its first TRACE_TILES tiles.
 constexpr int TRACE_TILES = 64;
-constexpr int TRACE_EVENTS = 32;
+constexpr int TRACE_EVENTS = 64;   // 0..31 role stages, 32..43 K done per converter warp, 44..55 V done
 
 // Unsigned 32-bit division by a divisor fixed for the launch, as a multiply-high and two shifts
 // (Granlund and Montgomery, "Division by invariant integers using multiplication", 1994, Fig. 4.1):
@@ -488,50 +498,104 @@ __device__ __forceinline__ bool key_rows(const DecodeParams& p, int b, int tok, 
 }
 
 // ---------------------------------------------------------------------------------------------
-// Producer side of one ring stage: the page runs of the `n` keys starting at token tok0 of request
-// b (at most two runs: page sizes are multiples of 16 and a half tile is 32 keys), each one bulk
-// copy of its rows into stage rows [r0, r0 + len) and, with per-token scales (SC), one bulk copy of
-// their scales (rounded up to whole 16-byte units, which stays inside the page).  Writes the mask of
-// copied rows to `mask_addr`, then arrives on `full` with the byte count and issues the copies.
+// Producer side of one ring stage.  The keys of a half tile (n keys from token tok0 of request b)
+// lie in at most two page runs (page sizes are multiples of 16 and a half tile is 32 keys; the
+// second run starts on a page boundary).
 // ---------------------------------------------------------------------------------------------
-template <bool SC>
-__device__ __forceinline__ void issue_half_tile(const DecodeParams& p, uint32_t stage, uint32_t full,
-                                                uint32_t mask_addr, int b, int tok0, int n) {
-  bool bad = false;
-  uint32_t mask = 0, tx = 0;
-  // first run: from tok0 to the end of its page (or of the half tile)
-  const int len0 = min(n, p.P - static_cast<int>(p.divP.mod(static_cast<uint32_t>(tok0))));
-  uint32_t v0 = 0, s0 = 0, v1 = 0, s1 = 0;
-  const bool ok0 = n > 0 && key_rows(p, b, tok0, v0, s0, bad);
-  // second run: the rest, which starts on a page boundary and is at most 16 <= P keys long
-  const int len1 = n - max(len0, 0);
-  const bool ok1 = len1 > 0 && key_rows(p, b, tok0 + len0, v1, s1, bad);
-  if (ok0) {
-    mask |= (len0 >= 32 ? 0xFFFFFFFFu : ((1u << len0) - 1u));
-    tx += static_cast<uint32_t>(len0) * HEAD_DIM + (SC ? ((static_cast<uint32_t>(len0) + 3u) & ~3u) * 4u : 0u);
-  }
-  if (ok1) {
-    mask |= ((1u << len1) - 1u) << len0;
-    tx += static_cast<uint32_t>(len1) * HEAD_DIM + (SC ? ((static_cast<uint32_t>(len1) + 3u) & ~3u) * 4u : 0u);
-  }
-  if (bad) raise_status(p.status, STATUS_BOUNDS);
-  ptx::st_shared_u32(mask_addr, mask);
-  ptx::mbar_arrive_expect_tx(full, tx);
-  if (ok0) {
-    ptx::bulk_load(stage, p.blocks + static_cast<size_t>(v0) * HEAD_DIM, static_cast<uint32_t>(len0) * HEAD_DIM, full);
-    if (SC) ptx::bulk_load(stage + RING_ROWS, p.scales + s0, ((static_cast<uint32_t>(len0) + 3u) & ~3u) * 4u, full);
-  }
-  if (ok1) {
-    const uint32_t r1 = static_cast<uint32_t>(len0);
-    ptx::bulk_load(stage + r1 * HEAD_DIM, p.blocks + static_cast<size_t>(v1) * HEAD_DIM,
-                   static_cast<uint32_t>(len1) * HEAD_DIM, full);
-    if (SC) ptx::bulk_load(stage + RING_ROWS + 4u * r1, p.scales + s1, ((static_cast<uint32_t>(len1) + 3u) & ~3u) * 4u, full);
-  }
+struct Runs {
+  uint32_t v0, s0, v1, s1;     // value and scale rows of each run's first key
+  int len0, len1;
+  bool ok0, ok1;
+};
+
+__device__ __forceinline__ Runs half_runs(const DecodeParams& p, int b, int tok0, int n, bool& bad) {
+  Runs R;
+  R.v0 = R.s0 = R.v1 = R.s1 = 0;
+  R.len0 = min(n, p.P - static_cast<int>(p.divP.mod(static_cast<uint32_t>(max(tok0, 0)))));
+  R.ok0 = n > 0 && key_rows(p, b, tok0, R.v0, R.s0, bad);
+  R.len1 = n - max(R.len0, 0);
+  R.ok1 = R.len1 > 0 && key_rows(p, b, tok0 + R.len0, R.v1, R.s1, bad);
+  return R;
 }
 
-// Values a converter thread loads one tile ahead from global memory: the other CTA's key's D_c
-// chunks (V atom column = its group, and V atom column 3 for the extra group) with their scales,
-// and in the block-scale mode the scales of its own key's three K chunks.
+__device__ __forceinline__ uint32_t run_mask(const Runs& R) {
+  uint32_t m = 0;
+  if (R.ok0) m |= (R.len0 >= 32 ? 0xFFFFFFFFu : ((1u << R.len0) - 1u));
+  if (R.ok1) m |= ((1u << R.len1) - 1u) << R.len0;
+  return m;
+}
+
+// Scale bytes of a run, rounded up to whole 16-byte units (the rounding stays inside the page:
+// runs start at multiples of 16 slots and pages hold a multiple of 16).
+__device__ __forceinline__ uint32_t scale_bytes(int len) { return ((static_cast<uint32_t>(len) + 3u) & ~3u) * 4u; }
+
+// Fills one ring stage for tile j of request b (visible keys nvis): the CTA's own 32 keys' rows
+// (rows [0, 32) of the stage) and, with per-token scales (SC), their scales at RING_ROWS; with
+// OTHER also the other CTA's 32 keys' scales at RING_OSC.  Writes the masks of copied rows and
+// copied other-key scales to mask_addr and mask_addr + 4, then arrives on `full` with the byte
+// count and issues the bulk copies.
+template <bool SC, bool OTHER>
+__device__ __forceinline__ void issue_stage(const DecodeParams& p, uint32_t stage, uint32_t full, uint32_t mask_addr,
+                                            int b, int j, int nvis, int c) {
+  bool bad = false;
+  const int tok0 = j * BN + HALF_BN * c;
+  const Runs own = half_runs(p, b, tok0, max(0, min(HALF_BN, nvis - tok0)), bad);
+  Runs oth;
+  oth.ok0 = oth.ok1 = false;
+  oth.len0 = oth.len1 = 0;
+  oth.v0 = oth.s0 = oth.v1 = oth.s1 = 0;
+  const int tok1 = j * BN + HALF_BN * (1 - c);
+  if (OTHER) oth = half_runs(p, b, tok1, max(0, min(HALF_BN, nvis - tok1)), bad);
+  uint32_t tx = 0;
+  if (own.ok0) tx += static_cast<uint32_t>(own.len0) * HEAD_DIM + (SC ? scale_bytes(own.len0) : 0u);
+  if (own.ok1) tx += static_cast<uint32_t>(own.len1) * HEAD_DIM + (SC ? scale_bytes(own.len1) : 0u);
+  if (OTHER && oth.ok0) tx += scale_bytes(oth.len0);
+  if (OTHER && oth.ok1) tx += scale_bytes(oth.len1);
+  if (bad) raise_status(p.status, STATUS_BOUNDS);
+  ptx::st_shared_u32(mask_addr, run_mask(own));
+  ptx::st_shared_u32(mask_addr + 4, OTHER ? run_mask(oth) : 0u);
+  ptx::mbar_arrive_expect_tx(full, tx);
+  if (own.ok0) {
+    ptx::bulk_load(stage, p.blocks + static_cast<size_t>(own.v0) * HEAD_DIM, static_cast<uint32_t>(own.len0) * HEAD_DIM, full);
+    if (SC) ptx::bulk_load(stage + RING_ROWS, p.scales + own.s0, scale_bytes(own.len0), full);
+  }
+  if (own.ok1) {
+    const uint32_t r1 = static_cast<uint32_t>(own.len0);
+    ptx::bulk_load(stage + r1 * HEAD_DIM, p.blocks + static_cast<size_t>(own.v1) * HEAD_DIM,
+                   static_cast<uint32_t>(own.len1) * HEAD_DIM, full);
+    if (SC) ptx::bulk_load(stage + RING_ROWS + 4u * r1, p.scales + own.s1, scale_bytes(own.len1), full);
+  }
+  if (OTHER && oth.ok0) ptx::bulk_load(stage + RING_OSC, p.scales + oth.s0, scale_bytes(oth.len0), full);
+  if (OTHER && oth.ok1)
+    ptx::bulk_load(stage + RING_OSC + 4u * static_cast<uint32_t>(oth.len0), p.scales + oth.s1, scale_bytes(oth.len1), full);
+}
+
+// Page-table entries of a converter thread's other-CTA key of one tile, read a step before the
+// rows are formed from them (so that the dependent data loads do not wait on the table read).
+struct OthLut {
+  uint32_t blk, sblk, slot;
+  bool vis, in_table;
+};
+
+__device__ __forceinline__ OthLut oth_lut_issue(const DecodeParams& p, const TileInfo& ti, int c, int r) {
+  OthLut L;
+  const int tok = ti.j * BN + HALF_BN * (1 - c) + r;
+  const uint32_t page = p.divP.div(static_cast<uint32_t>(tok));
+  L.slot = static_cast<uint32_t>(tok) - page * static_cast<uint32_t>(p.P);
+  L.vis = tok < ti.nvis;
+  L.in_table = page < static_cast<uint32_t>(p.max_pages);
+  L.blk = L.sblk = 0;
+  if (L.vis && L.in_table) {
+    const size_t e = static_cast<size_t>(item_b(p, ti.item)) * p.max_pages + page;
+    L.blk = __ldg(p.lut + e);
+    L.sblk = p.slut ? __ldg(p.slut + e) : L.blk;
+  }
+  return L;
+}
+
+// Values a converter thread loads a step ahead from global memory: the other CTA's key's D_c
+// chunks (V atom column = its group, and V atom column 3 for the extra group) and, in the
+// block-scale mode, their scales and the scales of its own key's three K chunks.
 struct Ahead {
   uint4 oth[2];
   float s_oth[2];
@@ -539,37 +603,43 @@ struct Ahead {
   bool oth_ok, own_ok;
 };
 
+// Issues the other key's chunk loads from the table entries read by oth_lut_issue.  Returns false
+// on a bad page id (that key then reads as zero).
 template <bool BS>
-__device__ __forceinline__ bool load_ahead(const DecodeParams& p, const TileInfo& ti, int c, int grp, int r, int cq,
-                                           bool extra, Ahead& A) {
-  bool bad = false;
-  const int b = item_b(p, ti.item);
-  const int tok = ti.j * BN + HALF_BN * (1 - c) + r;
-  uint32_t vrow = 0, srow = 0;
-  A.oth_ok = tok < ti.nvis && key_rows(p, b, tok, vrow, srow, bad);
+__device__ __forceinline__ bool fetch_oth(const DecodeParams& p, const OthLut& L, int c, int grp, int cq, bool extra,
+                                          Ahead& A) {
+  const bool ids_ok = L.blk < static_cast<uint32_t>(p.NB) && L.sblk < static_cast<uint32_t>(p.NSB);
+  const bool bad = L.vis && (!L.in_table || !ids_ok);
+  A.oth_ok = L.vis && L.in_table && ids_ok;
   if (A.oth_ok) {
+    const uint32_t per_blk = static_cast<uint32_t>(p.KVD * p.NL * p.P);
+    const uint32_t lay = static_cast<uint32_t>(p.layer * p.P);
+    const uint32_t vrow = L.blk * per_blk + lay + L.slot;
     const uint8_t* row = p.blocks + static_cast<size_t>(vrow) * HEAD_DIM;
     const int q0 = 4 * v_atom(grp, c) + cq;
     A.oth[0] = ptx::ldg_stream_v4(row + 16 * q0);
-    if (BS) A.s_oth[0] = __ldg(p.scales + static_cast<size_t>(srow) * p.SG + p.divCPB.div(q0));
-    else A.s_oth[0] = __ldg(p.scales + srow);
-    if (extra) {
-      const int q1 = 4 * v_atom(3, c) + cq;
-      A.oth[1] = ptx::ldg_stream_v4(row + 16 * q1);
-      A.s_oth[1] = BS ? __ldg(p.scales + static_cast<size_t>(srow) * p.SG + p.divCPB.div(q1)) : A.s_oth[0];
+    const int q1 = 4 * v_atom(3, c) + cq;
+    if (extra) A.oth[1] = ptx::ldg_stream_v4(row + 16 * q1);
+    if (BS) {
+      const size_t srow = static_cast<size_t>(L.sblk * per_blk + lay + L.slot) * p.SG;
+      A.s_oth[0] = __ldg(p.scales + srow + p.divCPB.div(q0));
+      if (extra) A.s_oth[1] = __ldg(p.scales + srow + p.divCPB.div(q1));
     }
   }
-  if (BS) {
-    const int otok = ti.j * BN + HALF_BN * c + r;
-    uint32_t ov = 0, os = 0;
-    A.own_ok = otok < ti.nvis && key_rows(p, b, otok, ov, os, bad);
-    if (A.own_ok) {
+  return !bad;
+}
+
+// Block-scale mode: the scales of the thread's own key's three K chunks of one tile.
+__device__ __forceinline__ bool fetch_own_scales(const DecodeParams& p, const TileInfo& ti, int c, int grp, int r,
+                                                 int cq, Ahead& A) {
+  bool bad = false;
+  const int otok = ti.j * BN + HALF_BN * c + r;
+  uint32_t ov = 0, os = 0;
+  A.own_ok = otok < ti.nvis && key_rows(p, item_b(p, ti.item), otok, ov, os, bad);
+  if (A.own_ok) {
 #pragma unroll
-      for (int m = 0; m < 3; ++m)
-        A.s_own[m] = __ldg(p.scales + static_cast<size_t>(os) * p.SG + p.divCPB.div(4 * (3 * grp + m) + cq));
-    }
-  } else {
-    A.own_ok = true;
+    for (int m = 0; m < 3; ++m)
+      A.s_own[m] = __ldg(p.scales + static_cast<size_t>(os) * p.SG + p.divCPB.div(4 * (3 * grp + m) + cq));
   }
   return !bad;
 }
@@ -578,39 +648,39 @@ __device__ __forceinline__ bool load_ahead(const DecodeParams& p, const TileInfo
 // a ring stage (raw) and dequantised into the K half buffer at `sk`.
 template <bool BS, bool FOLD>
 __device__ __forceinline__ void convert_k(int grp, int r, int cq, bool ok, const uint4 (&raw)[3], float s_tok,
-                                          const float (&s_blk)[3], uint32_t sk, int c, uint32_t (&keep0)[8],
-                                          uint32_t (&keep1)[8], int& va0, int& va1) {
-  int nd = 0;
-  va0 = va1 = -1;
+                                          const float (&s_blk)[3], uint32_t sk) {
+#pragma unroll
+  for (int m = 0; m < 3; ++m) {
+    uint32_t w[8];
+    convert16<FOLD>(ok, raw[m], BS ? s_blk[m] : s_tok, w);
+    st_chunk(sk + (3 * grp + m) * SK_ATOM, r, cq, w);
+  }
+}
+
+// The own key's D_c chunks of a converted K half, copied into the V operand (rows 32c + r).
+__device__ __forceinline__ void copy_dc_chunks(int grp, int r, int cq, int c, uint32_t sk, uint32_t sv) {
 #pragma unroll
   for (int m = 0; m < 3; ++m) {
     const int a = 3 * grp + m;
-    uint32_t w[8];
-    convert16<FOLD>(ok, raw[m], BS ? s_blk[m] : s_tok, w);
-    st_chunk(sk + a * SK_ATOM, r, cq, w);
-    if (k_in_dc(a, c)) {
-      if (nd == 0) {
-#pragma unroll
-        for (int x = 0; x < 8; ++x) keep0[x] = w[x];
-        va0 = k_to_v(a, c);
-      } else {
-#pragma unroll
-        for (int x = 0; x < 8; ++x) keep1[x] = w[x];
-        va1 = k_to_v(a, c);
-      }
-      ++nd;
-    }
+    if (!k_in_dc(a, c)) continue;
+    const uint32_t src = sk + a * SK_ATOM, dst = sv + k_to_v(a, c) * SV_ATOM;
+    const uint4 x = ptx::ld_shared_v4(src + sw128_off(r, 2 * cq));
+    const uint4 y = ptx::ld_shared_v4(src + sw128_off(r, 2 * cq + 1));
+    const int vr = HALF_BN * c + r;
+    ptx::st_shared_v4(dst + sw128_off(vr, 2 * cq), x.x, x.y, x.z, x.w);
+    ptx::st_shared_v4(dst + sw128_off(vr, 2 * cq + 1), y.x, y.y, y.z, y.w);
   }
 }
 
 // =============================================================================================
 // converter role (warps 0-11); the same code in both CTAs of the pair (c = rank).
-// Per tile g: read the thread's three FP8 chunks and the own key's scale from ring stage g % 2 and
-// release the stage; once Q.K^T(g-1) has finished (the K half buffer is free) dequantise them into
-// it; once P.V(g-2) has finished (V buffer g % 2 is free) write the V operand: the kept own-key
-// D_c chunks and the other key's D_c chunks (loaded from global memory during tile g-1).  Then
-// load the other key's chunks of tile g+1.  Returns early (with the abort flag set by the failing
-// wait) when a wait gives up.
+// Step g: (K) read the thread's three FP8 chunks of tile g and the tile's scales from ring stage
+// g % 2 and release the stage; once Q.K^T(g-2) has finished (K half buffer g % 2 is free)
+// dequantise them into it.  (V) Dequantise the other key's D_c chunks of tile g-1 (loaded during
+// step g-1); once P.V(g-2) has finished (the V buffer is free) write tile g-1's V operand: those
+// chunks and the own key's D_c chunks copied from K half buffer (g-1) % 2.  Then read the other
+// key's chunks of tile g and the page-table entries of tile g+1.  Returns early (with the abort
+// flag set by the failing wait) when a wait gives up.
 // =============================================================================================
 template <int MODE>
 __device__ __forceinline__ void converter_role(const DecodeParams& p, int k, uint32_t base, int lane,
@@ -630,72 +700,91 @@ __device__ __forceinline__ void converter_role(const DecodeParams& p, int k, uin
   if (!__all_sync(0xffffffffu, poll_bar((b_), (parity), abort, p.status, peer_abort, lim))) return;
   const uint32_t k_full0 = ptx::mapa(BAR(B_K_FULL), 0), v_full0 = ptx::mapa(BAR(B_V_FULL), 0);
   TileStream ts(p, k);
-  TileInfo cur = ts.take(p);
-  if (!cur.valid) return;
-  TileInfo nxt = ts.take(p);
-  Ahead A;
-  if (!load_ahead<BS>(p, cur, C, grp, r, cq, extra, A)) raise_status(p.status, STATUS_BOUNDS);
+  TileInfo kt = ts.take(p);
+  if (!kt.valid) return;
+  TileInfo nt = ts.take(p);
+  OthLut L = oth_lut_issue(p, kt, C, r);
+  Ahead A;                       // the other key's chunks of the tile whose V operand is written next
+  A.oth_ok = false;
+  A.own_ok = true;
+  if (BS && !fetch_own_scales(p, kt, C, grp, r, cq, A)) raise_status(p.status, STATUS_BOUNDS);
+  float s_oth_v = 0.f;           // per-token scale of that key (from the ring)
   uint32_t g = 0;
   // Rolled loop (one copy of the step keeps the hot code small).
   while (true) {
-    const uint32_t st = g & 1;
-    MLA_WAIT_RET(BAR(B_RING_FULL + st), (g >> 1) & 1);
-    if (t == 0) MLA_TRACE_EV(g, 1);
-    const uint32_t stage = base + SRING + st * RING_STAGE;
-    const bool own_ok = ((ptx::ld_shared_u32(base + S_MASK + 4 * st) >> r) & 1u) != 0 && A.own_ok;
-    uint4 raw[3];
+    float s_oth_k = 0.f;
+    if (kt.valid) {
+      // ---------------------------------------------------------------- K half of tile g
+      const uint32_t st = g & 1;
+      if (t == 0) MLA_TRACE_EV(g, 1);
+      MLA_WAIT_RET(BAR(B_RING_FULL + st), (g >> 1) & 1);
+      if (t == 0) MLA_TRACE_EV(g, 3);
+      const uint32_t stage = base + SRING + st * RING_STAGE;
+      const bool own_ok = ((ptx::ld_shared_u32(base + S_MASK + 8 * st) >> r) & 1u) != 0 && A.own_ok;
+      uint4 raw[3];
 #pragma unroll
-    for (int m = 0; m < 3; ++m) raw[m] = ptx::ld_shared_v4(stage + r * HEAD_DIM + 16 * (4 * (3 * grp + m) + cq));
-    const float s_own = BS ? 0.f : ptx::ld_shared_f32(stage + RING_ROWS + 4 * r);
-    __syncwarp();
-    if (lane == 0) ptx::mbar_arrive(BAR(B_RING_EMPTY + st));    // the reads above are ordered before it
-    // K half buffer: free once Q.K^T of the previous tile has finished
-    if (g > 0) MLA_POLL_RET(BAR(B_S_FULL + ((g - 1) & 1)), ((g - 1) >> 1) & 1);
-    if (t == 0) MLA_TRACE_EV(g, 16);
-    if (FOLD) {
-      // the tile's 64 per-token scales for the softmax (0 for keys not read); the softmax of tile
-      // g - 4 has read this buffer (it finished before S_FREE(g - 3), which Q.K^T(g - 1) waited for)
-      if (grp == 0 && cq == 0) {
-        const uint32_t sa = base + SSC + (g & 3) * SSC_STRIDE + 4 * r;
-        ptx::st_shared_f32(sa + 4 * HALF_BN * C, own_ok ? s_own : 0.f);
-        ptx::st_shared_f32(sa + 4 * HALF_BN * (1 - C), A.oth_ok ? A.s_oth[0] : 0.f);
+      for (int m = 0; m < 3; ++m) raw[m] = ptx::ld_shared_v4(stage + r * HEAD_DIM + 16 * (4 * (3 * grp + m) + cq));
+      const float s_own = BS ? 0.f : ptx::ld_shared_f32(stage + RING_ROWS + 4 * r);
+      if (!BS) s_oth_k = ptx::ld_shared_f32(stage + RING_OSC + 4 * r);
+      if (FOLD) {
+        // the tile's 64 per-token scales for the softmax (0 for keys not read).  Slot g % 8 last
+        // held tile g - 8, which the softmax finished before S_FREE(g - 5), which Q.K^T(g - 3)
+        // waited for before the K-buffer wait of step g - 1 passed.
+        if (grp == 0 && cq == 0) {
+          const uint32_t om = ptx::ld_shared_u32(base + S_MASK + 8 * st + 4);
+          const uint32_t sa = base + SSC + (g % SSC_SLOTS) * SSC_STRIDE + 4 * r;
+          ptx::st_shared_f32(sa + 4 * HALF_BN * C, own_ok ? s_own : 0.f);
+          ptx::st_shared_f32(sa + 4 * HALF_BN * (1 - C), ((om >> r) & 1u) ? s_oth_k : 0.f);
+        }
+        __syncwarp();
+        if (lane == 0) ptx::mbar_arrive(BAR(B_SC_FULL + (g % SSC_SLOTS)));
       }
       __syncwarp();
-      if (lane == 0) ptx::mbar_arrive(BAR(B_SC_FULL + (g & 3)));
+      if (lane == 0) ptx::mbar_arrive(BAR(B_RING_EMPTY + st));    // the reads above are ordered before it
+      // K half buffer g % 2: free once Q.K^T(g - 2) has finished
+      MLA_POLL_RET(BAR(B_S_FULL + st), ((g >> 1) & 1) ^ 1);
+      if (t == 0) MLA_TRACE_EV(g, 16);
+      convert_k<BS, FOLD>(grp, r, cq, own_ok, raw, s_own, A.s_own, base + SK0 + st * SK_STRIDE);
+      ptx::fence_proxy_async_smem();
+      __syncwarp();
+      if (lane == 0) ptx::mbar_arrive_cluster(k_full0 + 8u * st);
+      if (t == 0) MLA_TRACE_EV(g, 5);
+      if (t == 352) MLA_TRACE_EV(g, 26);
+      if (lane == 0) MLA_TRACE_EV(g, 32 + (t >> 5));
     }
-    uint32_t keep0[8], keep1[8];
-    int va0, va1;
-    convert_k<BS, FOLD>(grp, r, cq, own_ok, raw, s_own, A.s_own, base + SK, C, keep0, keep1, va0, va1);
-    ptx::fence_proxy_async_smem();
-    __syncwarp();
-    if (lane == 0) ptx::mbar_arrive_cluster(k_full0);
-    if (t == 0) MLA_TRACE_EV(g, 5);
-    // V operand buffer g % 2: free once P.V(g - 2) has finished
-    MLA_WAIT_RET(BAR(B_PV_DONE + st), ((g >> 1) & 1) ^ 1);
-    if (t == 0) MLA_TRACE_EV(g, 6);
-    {
-      const uint32_t sv = base + SV0 + st * SV_STRIDE;
-      const int vrow_own = HALF_BN * C + r, vrow_oth = HALF_BN * (1 - C) + r;
-      if (va0 >= 0) st_chunk(sv + va0 * SV_ATOM, vrow_own, cq, keep0);
-      if (va1 >= 0) st_chunk(sv + va1 * SV_ATOM, vrow_own, cq, keep1);
-      uint32_t w[8];
-      convert16<FOLD>(A.oth_ok, A.oth[0], A.s_oth[0], w);
-      st_chunk(sv + grp * SV_ATOM, vrow_oth, cq, w);
-      if (extra) {
-        convert16<FOLD>(A.oth_ok, A.oth[1], A.s_oth[1], w);
-        st_chunk(sv + 3 * SV_ATOM, vrow_oth, cq, w);
-      }
+    if (g > 0) {
+      // ---------------------------------------------------------------- V operand of tile g - 1
+      const uint32_t vt = g - 1;
+      uint32_t w0[8], w1[8];
+      convert16<FOLD>(A.oth_ok, A.oth[0], BS ? A.s_oth[0] : s_oth_v, w0);
+      if (extra) convert16<FOLD>(A.oth_ok, A.oth[1], BS ? A.s_oth[1] : s_oth_v, w1);
+      // the V buffer is free once P.V(g - 2) has finished
+      if (t == 0) MLA_TRACE_EV(vt, 4);
+      MLA_WAIT_RET(BAR(B_PV_DONE + (g & 1)), ((g >> 1) & 1) ^ 1);
+      if (t == 0) MLA_TRACE_EV(vt, 6);
+      copy_dc_chunks(grp, r, cq, C, base + SK0 + (vt & 1) * SK_STRIDE, base + SV);
+      const int vrow_oth = HALF_BN * (1 - C) + r;
+      st_chunk(base + SV + grp * SV_ATOM, vrow_oth, cq, w0);
+      if (extra) st_chunk(base + SV + 3 * SV_ATOM, vrow_oth, cq, w1);
+      ptx::fence_proxy_async_smem();
+      __syncwarp();
+      if (lane == 0) ptx::mbar_arrive_cluster(v_full0 + 8u * (vt & 1));
+      if (t == 0) MLA_TRACE_EV(vt, 2);
+      if (t == 352) MLA_TRACE_EV(vt, 27);
+      if (lane == 0) MLA_TRACE_EV(vt, 44 + (t >> 5));
     }
-    ptx::fence_proxy_async_smem();
-    __syncwarp();
-    if (lane == 0) ptx::mbar_arrive_cluster(v_full0 + 8u * st);
-    if (t == 0) MLA_TRACE_EV(g, 2);
+    if (!kt.valid) break;
+    // ---------------------------------------------------------------- loads for the next step
+    s_oth_v = s_oth_k;
+    if (!fetch_oth<BS>(p, L, C, grp, cq, extra, A)) raise_status(p.status, STATUS_BOUNDS);
+    if (nt.valid) {
+      L = oth_lut_issue(p, nt, C, r);
+      if (BS && !fetch_own_scales(p, nt, C, grp, r, cq, A)) raise_status(p.status, STATUS_BOUNDS);
+    }
+    if (t == 0) MLA_TRACE_EV(g, 7);
+    kt = nt;
+    nt = ts.take(p);
     ++g;
-    if (!nxt.valid) break;
-    if (!load_ahead<BS>(p, nxt, C, grp, r, cq, extra, A)) raise_status(p.status, STATUS_BOUNDS);
-    if (t == 0) MLA_TRACE_EV(g - 1, 7);
-    cur = nxt;
-    nxt = ts.take(p);
   }
 #undef MLA_POLL_RET
 #undef MLA_WAIT_RET
@@ -720,11 +809,10 @@ __device__ __forceinline__ void producer_role(const DecodeParams& p, int k, uint
     if (!ti.valid) break;
     const uint32_t st = g & 1;
     if (!wait_bar(BAR(B_RING_EMPTY + st), ((g >> 1) & 1) ^ 1, abort, p.status, peer_abort, p.wait_limit_ns)) break;
-    if (g < 64 && k == 0) MLA_TRACE_EV(g, 24);
-    const int tok0 = ti.j * BN + HALF_BN * static_cast<int>(c);
-    const int n = max(0, min(HALF_BN, ti.nvis - tok0));
-    issue_half_tile<SC>(p, base + SRING + st * RING_STAGE, BAR(B_RING_FULL + st), base + S_MASK + 4 * st,
-                        item_b(p, ti.item), tok0, n);
+    MLA_TRACE_EV(g, 24);
+    issue_stage<SC, SC>(p, base + SRING + st * RING_STAGE, BAR(B_RING_FULL + st), base + S_MASK + 8 * st,
+                        item_b(p, ti.item), ti.j, ti.nvis, static_cast<int>(c));
+    MLA_TRACE_EV(g, 25);
     ++g;
   }
   for (uint32_t gd = (g >= 2 ? g - 2 : 0); gd < g; ++gd)
@@ -760,8 +848,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) mla_decode_kernel(const __grid
   MLA_TRACE_CTA(0);
 
   if (threadIdx.x == 0) {
-    ptx::mbar_init(BAR(B_K_FULL), 2 * CONV_WARPS);
     for (uint32_t i = 0; i < 2; ++i) {
+      ptx::mbar_init(BAR(B_K_FULL + i), 2 * CONV_WARPS);
       ptx::mbar_init(BAR(B_V_FULL + i), 2 * CONV_WARPS);
       ptx::mbar_init(BAR(B_PV_DONE + i), 1);
       ptx::mbar_init(BAR(B_S_FULL + i), 1);
@@ -778,7 +866,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) mla_decode_kernel(const __grid
     ptx::mbar_init(BAR(B_DRAIN), 2);
     ptx::mbar_init(BAR(B_REDL), 4);
     ptx::mbar_init(BAR(B_EXIT), 1);
-    for (uint32_t i = 0; i < 4; ++i) ptx::mbar_init(BAR(B_SC_FULL + i), CONV_WARPS);
+    for (uint32_t i = 0; i < SSC_SLOTS; ++i) ptx::mbar_init(BAR(B_SC_FULL + i), CONV_WARPS);
     *abort = 0u;
     ptx::fence_mbar_init();
   }
@@ -821,7 +909,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) mla_decode_kernel(const __grid
       for (int j = u.tb; j < u.te; ++j, ++g) {
         const uint32_t sb = g & 1;
         MLA_WAIT_WARP(BAR(B_S_FULL + sb), (g >> 1) & 1);
-        if (FOLD) MLA_WAIT_WARP(BAR(B_SC_FULL + (g & 3)), (g >> 2) & 1);
+        if (FOLD) MLA_WAIT_WARP(BAR(B_SC_FULL + (g % SSC_SLOTS)), (g / SSC_SLOTS) & 1);
         if (t == 0) MLA_TRACE_EV(g, 8);
         ptx::tc_fence_after();
         float x[32];
@@ -840,8 +928,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) mla_decode_kernel(const __grid
         const int nv = min(BN, u.nvis - j * BN) - HALF_BN * hh;   // valid keys in this lane's half
         float mt = -INFINITY;
         // scale-folding mode: the scales of this lane's 32 keys (written before K_FULL of this
-        // tile; buffer g & 3 is rewritten only after this warp has finished tile g)
-        const uint32_t sc_addr = base + SSC + (g & 3) * SSC_STRIDE + 4 * HALF_BN * hh;
+        // tile; slot g % 8 is rewritten only after this warp has finished tile g)
+        const uint32_t sc_addr = base + SSC + (g % SSC_SLOTS) * SSC_STRIDE + 4 * HALF_BN * hh;
         if (FOLD) {
 #pragma unroll
           for (int v = 0; v < 8; ++v) {
@@ -904,11 +992,11 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) mla_decode_kernel(const __grid
         }
         l += lsum;
         if (t == 0) MLA_TRACE_EV(g, 11);
-        // P buffer sb is free once P.V(g - 2) has finished
-        MLA_WAIT_WARP(BAR(B_PV_DONE + sb), ((g >> 1) & 1) ^ 1);
+        // the P buffer is free once P.V(g - 1) has finished (O may be rescaled from then on too)
+        if (g > 0) MLA_WAIT_WARP(BAR(B_PV_DONE + ((g - 1) & 1)), ((g - 1) >> 1) & 1);
         if (t == 0) MLA_TRACE_EV(g, 13);
         {
-          const uint32_t sp = base + SP0 + sb * SP_STRIDE;
+          const uint32_t sp = base + SP;
 #pragma unroll
           for (int v = 0; v < 4; ++v)
             ptx::st_shared_v4(sp + sw128_off(r, 4 * hh + v), pw[4 * v], pw[4 * v + 1], pw[4 * v + 2], pw[4 * v + 3]);
@@ -917,8 +1005,6 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) mla_decode_kernel(const __grid
         // reference max; rows that did not move use alpha = 1
         if (!rescale) alpha = 1.f;
         if (__any_sync(0xffffffffu, rescale)) {
-          const uint32_t gp = g - 1;
-          MLA_WAIT_WARP(BAR(B_PV_DONE + (gp & 1)), (gp >> 1) & 1);
           ptx::tc_fence_after();
 #pragma unroll 1
           for (int ch = 0; ch < 8; ++ch) {
@@ -952,11 +1038,13 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) mla_decode_kernel(const __grid
         const int head = u.g * MROWS + HPC * static_cast<int>(c) + r;
         const bool row_ok = head < p.H;
         const float lse_v = (m_ref + ptx::lg2_approx(l_row)) * 0.69314718055994530942f;
-        // O / l goes out through a per-warp 4 KB staging block in the (now idle) P buffers: each
-        // thread writes its row's 32 values of a chunk, then the warp stores whole 64- or 128-byte
-        // row segments (16-byte positions swizzled by row, so both passes are conflict-free).
-        const uint32_t stage = base + SP0 + static_cast<uint32_t>(quad) * 4096u;
+        // O / l goes out through a per-warp 2 KB staging block in the (now idle) P buffer: each
+        // thread writes 64 bytes of its row (32 bf16, or 16 fp32 per half of a chunk), then the warp
+        // stores whole 64-byte row segments; 16-byte chunk j of row x sits at x * 64 + 16 * (j ^
+        // ((x >> 1) & 3)), so both passes are conflict-free.
+        const uint32_t stage = base + SP + static_cast<uint32_t>(quad) * 2048u;
         const int row0 = HPC * static_cast<int>(c) + 32 * (quad & 1);   // CTA row of this warp's lane 0
+        const uint32_t my = stage + lane * 64;
 #pragma unroll 1
         for (int ch = 0; ch < 8; ++ch) {
           uint32_t rr[32];
@@ -964,14 +1052,13 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) mla_decode_kernel(const __grid
           ptx::tmem_wait_ld();
           const int dv = (ch < 4 ? 0 : 256) + 128 * hh + 32 * (ch & 3);
           if (u.slot < 0) {
-            // bf16: 32 rows x 64 B; 16-byte chunk j of row x at x * 64 + 16 * (j ^ ((x >> 1) & 3))
 #pragma unroll
             for (int v = 0; v < 4; ++v) {
               const uint32_t w0 = ptx::pack_bf16x2(__uint_as_float(rr[8 * v + 0]) * inv_l, __uint_as_float(rr[8 * v + 1]) * inv_l);
               const uint32_t w1 = ptx::pack_bf16x2(__uint_as_float(rr[8 * v + 2]) * inv_l, __uint_as_float(rr[8 * v + 3]) * inv_l);
               const uint32_t w2 = ptx::pack_bf16x2(__uint_as_float(rr[8 * v + 4]) * inv_l, __uint_as_float(rr[8 * v + 5]) * inv_l);
               const uint32_t w3 = ptx::pack_bf16x2(__uint_as_float(rr[8 * v + 6]) * inv_l, __uint_as_float(rr[8 * v + 7]) * inv_l);
-              ptx::st_shared_v4(stage + lane * 64 + 16 * (v ^ ((lane >> 1) & 3)), w0, w1, w2, w3);
+              ptx::st_shared_v4(my + 16 * (v ^ ((lane >> 1) & 3)), w0, w1, w2, w3);
             }
             __syncwarp();
 #pragma unroll
@@ -983,20 +1070,24 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) mla_decode_kernel(const __grid
                 *reinterpret_cast<uint4*>(p.out + ((static_cast<size_t>(u.b) * p.T + u.i) * p.H + hd) * V_DIM + dv + 8 * j) = w;
             }
           } else {
-            // fp32: 32 rows x 128 B; 16-byte chunk j of row x at x * 128 + 16 * (j ^ (x & 7))
 #pragma unroll
-            for (int v = 0; v < 8; ++v)
-              ptx::st_shared_v4(stage + lane * 128 + 16 * (v ^ (lane & 7)),
-                                __float_as_uint(__uint_as_float(rr[4 * v + 0]) * inv_l),
-                                __float_as_uint(__uint_as_float(rr[4 * v + 1]) * inv_l),
-                                __float_as_uint(__uint_as_float(rr[4 * v + 2]) * inv_l),
-                                __float_as_uint(__uint_as_float(rr[4 * v + 3]) * inv_l));
-            __syncwarp();
+            for (int hf = 0; hf < 2; ++hf) {
 #pragma unroll
-            for (int it = 0; it < 8; ++it) {
-              const int x = it * 4 + (lane >> 3), j = lane & 7;
-              const uint4 w = ptx::ld_shared_v4(stage + x * 128 + 16 * (j ^ (x & 7)));
-              *reinterpret_cast<uint4*>(p.part_o + (static_cast<size_t>(u.slot) * MROWS + row0 + x) * V_DIM + dv + 4 * j) = w;
+              for (int v = 0; v < 4; ++v)
+                ptx::st_shared_v4(my + 16 * (v ^ ((lane >> 1) & 3)),
+                                  __float_as_uint(__uint_as_float(rr[16 * hf + 4 * v + 0]) * inv_l),
+                                  __float_as_uint(__uint_as_float(rr[16 * hf + 4 * v + 1]) * inv_l),
+                                  __float_as_uint(__uint_as_float(rr[16 * hf + 4 * v + 2]) * inv_l),
+                                  __float_as_uint(__uint_as_float(rr[16 * hf + 4 * v + 3]) * inv_l));
+              __syncwarp();
+#pragma unroll
+              for (int it = 0; it < 4; ++it) {
+                const int x = it * 8 + (lane >> 2), j = lane & 3;
+                const uint4 w = ptx::ld_shared_v4(stage + x * 64 + 16 * (j ^ ((x >> 1) & 3)));
+                *reinterpret_cast<uint4*>(p.part_o + (static_cast<size_t>(u.slot) * MROWS + row0 + x) * V_DIM + dv +
+                                          16 * hf + 4 * j) = w;
+              }
+              __syncwarp();
             }
           }
           __syncwarp();
@@ -1054,26 +1145,47 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) mla_decode_kernel(const __grid
       uint32_t g = 0, uq = 0;
       // descriptor bases; per K step only the start-address field (bits 0..13, bytes >> 4) moves
       const uint64_t dq0 = ptx::smem_desc(base + SQ, 16, 1024, ptx::SW_128B);
-      const uint64_t dk0 = ptx::smem_desc(base + SK, 16, 1024, ptx::SW_128B);
+      const uint64_t dk0 = ptx::smem_desc(base + SK0, 16, 1024, ptx::SW_128B);
       while (qc.valid) {
         const uint32_t sb = g & 1;
         if (qc.first) {
+          // the unit's Q is in shared memory (both CTAs); its first 384 dims go to tensor memory
+          // once, so that the Q.K^T MMAs of the unit read that part of A from there.  The previous
+          // unit's MMAs have finished (the Q loader waited for Q_FREE before loading).
           MLA_POLL_WARP(BAR(B_Q_FULL), uq & 1);
           ++uq;
+          ptx::tc_fence_after();
+          if (ptx::elect_one()) {
+#pragma unroll 1
+            for (int a = 0; a < Q_TMEM_ATOMS; ++a)
+#pragma unroll
+              for (int j = 0; j < 8; ++j)
+                ptx::tmem_cp_pair_64x128_dup(tbase + T_Q + 32 * a + 4 * j,
+                                             ptx::smem_desc(base + SQ + a * SQ_ATOM + 16 * j, 16, 1024, ptx::SW_128B));
+          }
+          __syncwarp();
         }
-        MLA_POLL_WARP(BAR(B_K_FULL), g & 1);
+        MLA_POLL_WARP(BAR(B_K_FULL + sb), (g >> 1) & 1);
         MLA_POLL_WARP(BAR(B_S_FREE + sb), ((g >> 1) & 1) ^ 1);
         ptx::tc_fence_after();
         if (ptx::elect_one()) {
           MLA_TRACE_EV(g, 20);
           const uint32_t dS = tbase + T_S + 32 * sb;
-          // 9 atom columns of 64 dims x 4 K steps of 16 dims
-          uint64_t ad = dq0, bd = dk0;
+          // 9 atom columns of 64 dims x 4 K steps of 16 dims: A from tensor memory for atom
+          // columns 0..5 (8 columns per K step), from shared memory for 6..8
+          uint64_t bd = dk0 + ((sb * SK_STRIDE) >> 4);
 #pragma unroll 1
-          for (int a = 0; a < 9; ++a) {
+          for (int a = 0; a < Q_TMEM_ATOMS; ++a) {
 #pragma unroll
             for (int kk = 0; kk < 4; ++kk)
-              ptx::mma_pair_ss(dS, ad + kk * 2, bd + kk * 2, IDESC_QK, (a | kk) != 0 ? 1u : 0u);
+              ptx::mma_pair_ts(dS, tbase + T_Q + 32 * a + 8 * kk, bd + kk * 2, IDESC_QK, (a | kk) != 0 ? 1u : 0u);
+            bd += SK_ATOM >> 4;
+          }
+          uint64_t ad = dq0 + ((Q_TMEM_ATOMS * SQ_ATOM) >> 4);
+#pragma unroll 1
+          for (int a = Q_TMEM_ATOMS; a < 9; ++a) {
+#pragma unroll
+            for (int kk = 0; kk < 4; ++kk) ptx::mma_pair_ss(dS, ad + kk * 2, bd + kk * 2, IDESC_QK, 1u);
             ad += SQ_ATOM >> 4;
             bd += SK_ATOM >> 4;
           }
@@ -1093,8 +1205,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) mla_decode_kernel(const __grid
     if (c == 0) {
       TileCursor pc(p, k);
       uint32_t g = 0, up = 0;
-      const uint64_t dp0 = ptx::smem_desc(base + SP0, 16, 1024, ptx::SW_128B);
-      const uint64_t dv0 = ptx::smem_desc(base + SV0, SV_ATOM, 1024, ptx::SW_128B);
+      const uint64_t dp0 = ptx::smem_desc(base + SP, 16, 1024, ptx::SW_128B);
+      const uint64_t dv0 = ptx::smem_desc(base + SV, SV_ATOM, 1024, ptx::SW_128B);
       while (pc.valid) {
         const uint32_t hb = g & 1;
         const bool first = pc.first;
@@ -1111,8 +1223,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) mla_decode_kernel(const __grid
           for (int jv = 0; jv < 2; ++jv) {
 #pragma unroll
             for (int kk = 0; kk < 4; ++kk) {
-              const uint64_t ad = dp0 + ((hb * SP_STRIDE + kk * 32) >> 4);
-              const uint64_t bd = dv0 + ((hb * SV_STRIDE + 2 * jv * SV_ATOM + kk * 2048) >> 4);
+              const uint64_t ad = dp0 + ((kk * 32) >> 4);
+              const uint64_t bd = dv0 + ((2 * jv * SV_ATOM + kk * 2048) >> 4);
               ptx::mma_pair_ss(tbase + T_O + 128 * jv, ad, bd, IDESC_PV, (first && kk == 0) ? 0u : 1u);
             }
           }
@@ -1312,12 +1424,12 @@ mla_combine_kernel(const __grid_constant__ DecodeParams p) {
 
 // =============================================================================================
 // gather + dequant kernel (steps A and C alone): one CTA of 384 threads per (request, 64-key tile,
-// key half c).  Runs the decode's producer (issue_half_tile: page runs -> one ring stage) and its
-// converter (load_ahead for block scales, convert_k), then copies the K-half buffer back out.
+// key half c).  Runs the decode's producer (issue_stage: page runs -> one ring stage) and its
+// converter (fetch_own_scales for block scales, convert_k), then copies the K-half buffer out.
 // =============================================================================================
 constexpr int DQ_THREADS = CONV_THREADS;
 constexpr uint32_t DQ_SK = 0;
-constexpr uint32_t DQ_RING = SK_BYTES;
+constexpr uint32_t DQ_RING = SK_STRIDE;
 constexpr uint32_t DQ_BAR = DQ_RING + RING_STAGE;
 constexpr uint32_t DQ_SMEM_ALLOC = DQ_BAR + 64 + 1024;
 
@@ -1342,17 +1454,20 @@ mla_dequant_kernel(const __grid_constant__ DecodeParams p, const uint32_t* cache
     ptx::fence_mbar_init();
   }
   __syncthreads();
-  if (threadIdx.x == 0) issue_half_tile<!BS>(p, base + DQ_RING, full, mask_addr, b, tok0, cnt);
+  if (threadIdx.x == 0) issue_stage<!BS, false>(p, base + DQ_RING, full, mask_addr, b, j, n, c);
   const int t = threadIdx.x, grp = t / CONV_GROUP, tau = t % CONV_GROUP;
   const int r = conv_row(tau), cq = conv_cq(tau);
-  TileInfo ti;
-  ti.item = b * p.T * p.G;
-  ti.nvis = n;
-  ti.j = j;
-  ti.first = true;
-  ti.valid = true;
   Ahead A;
-  if (!load_ahead<BS>(p, ti, c, grp, r, cq, false, A)) raise_status(p.status, STATUS_BOUNDS);
+  A.own_ok = true;
+  if (BS) {
+    TileInfo ti;
+    ti.item = b * p.T * p.G;
+    ti.nvis = n;
+    ti.j = j;
+    ti.first = true;
+    ti.valid = true;
+    if (!fetch_own_scales(p, ti, c, grp, r, cq, A)) raise_status(p.status, STATUS_BOUNDS);
+  }
   const uint64_t t0 = ptx::globaltimer();
   bool landed;
   while (!(landed = ptx::mbar_try_wait(full, 0)) && ptx::globaltimer() - t0 < p.wait_limit_ns) {}
@@ -1362,9 +1477,7 @@ mla_dequant_kernel(const __grid_constant__ DecodeParams p, const uint32_t* cache
 #pragma unroll
   for (int m = 0; m < 3; ++m) raw[m] = ptx::ld_shared_v4(base + DQ_RING + r * HEAD_DIM + 16 * (4 * (3 * grp + m) + cq));
   const float s_own = BS ? 0.f : ptx::ld_shared_f32(base + DQ_RING + RING_ROWS + 4 * r);
-  uint32_t keep0[8], keep1[8];
-  int va0, va1;
-  convert_k<BS, false>(grp, r, cq, own_ok, raw, s_own, A.s_own, base + DQ_SK, c, keep0, keep1, va0, va1);
+  convert_k<BS, false>(grp, r, cq, own_ok, raw, s_own, A.s_own, base + DQ_SK);
   __syncthreads();
   for (int id = threadIdx.x; id < HALF_BN * 72; id += DQ_THREADS) {
     const int row = id / 72, cc = id - row * 72;        // 72 units of 8 bf16 per key

@@ -352,6 +352,27 @@ __device__ __forceinline__ void mma_pair_ss(uint32_t d_tmem, uint64_t a_desc, ui
       :: "r"(d_tmem), "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate) : "memory");
 }
 
+// The same with A read from tensor memory (a_tmem: lane 0, first column of the K slice).  In the pair
+// layout D lanes 0..63 take A from lanes 0..63 and D lanes 64..127 from lanes 64..127, so each A row
+// must be present in lane r and lane r + 64.
+__device__ __forceinline__ void mma_pair_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc, uint32_t idesc,
+                                            uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::2.kind::f16 [%0], [%1], %2, %3, p;\n\t}"
+      :: "r"(d_tmem), "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"(accumulate) : "memory");
+}
+
+// Pair-wide shared -> tensor memory copy of 64 rows x 16 bytes (one 16-byte column of a K-major
+// matrix described by s_desc) into 4 columns at t_addr, each row r written to lane r and to lane
+// r + 64 (warpx2::02_13: rows 0..31 to lane quadrants 0 and 2, rows 32..63 to quadrants 1 and 3).
+// Issued by one thread of CTA 0; both CTAs copy their own shared memory.  Later tcgen05.mma of the
+// same thread read the copied values (tcgen05.cp -> tcgen05.mma is ordered by the hardware).
+__device__ __forceinline__ void tmem_cp_pair_64x128_dup(uint32_t t_addr, uint64_t s_desc) {
+  asm volatile("tcgen05.cp.cta_group::2.64x128b.warpx2::02_13 [%0], %1;" :: "r"(t_addr), "l"(s_desc) : "memory");
+}
+
 // Arrive once on the barrier at `mbar`'s offset in every CTA of `cta_mask` when all pair MMAs
 // issued so far by this thread have completed.
 __device__ __forceinline__ void mma_commit_pair(uint32_t mbar, uint16_t cta_mask) {
