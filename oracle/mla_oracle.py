@@ -42,6 +42,10 @@ What it computes, step by step, in the order the pages lay out the data:
    attention over the unrounded products e4m3 * s_t; it differs from step 2's rounded keys by
    the fp32 and bf16 roundings of the dequant (reading R18).
 
+6. The FP8 P.V variant (per-token scales): scores and softmax as in steps 1-3, and the value
+   product taken with the exact e4m3 values and the scale folded into the weights, each weight
+   split into two e4m3 terms (attend_fp8_pv, reading R21).
+
 Everything after the e4m3 decode is float64 (the dequantised bf16 values are
 exact in float64).  Points the pages leave open and the reading taken here:
 cache_lengths count only tokens cached before this step (R1); query i sees
@@ -337,6 +341,89 @@ def decode_scale_folded(q, blocks, scales, cache_lengths, lookup_table, scales_l
         for i in range(T):
             vis = int(L[b]) + i + 1
             r = attend_scale_folded(q[b, i, hs], codes[:vis], sc[:vis, 0], softmax_scale)
+            out[b, i, hs] = r[0]
+            lse[b, i, hs] = r[1]
+    return out, lse
+
+
+# ----------------------------------------------------------------------------
+# FP8 P.V variant (per-token scales only)
+# ----------------------------------------------------------------------------
+E4M3_MAX = 448.0
+FP8_PV_HEADROOM = 1.75          # 448 / 2^8: the folded weight p * s * 2^sigma stays below 448 for p <= 2^8
+
+
+def fp8_pv_sigma(s_max):
+    """Power-of-two exponent of the folded weights: the largest integer sigma with
+    s_max * 2^sigma <= 1.75, so that p * s * 2^sigma <= 448 for every weight p <= 2^8."""
+    return int(np.floor(np.log2(FP8_PV_HEADROOM / float(s_max))))
+
+
+def e4m3_split2(w):
+    """Two-term e4m3 split of float32 values w (all >= 0): hi = e4m3_rn_sat(w), lo = e4m3_rn_sat(w - hi)
+    (the residual is exact in float32).  Returns (hi, lo) as float64 values."""
+    w = np.asarray(w, dtype=np.float32)
+    hi = e4m3_decode(e4m3_encode_rn_sat(w))
+    r = (w.astype(np.float64) - hi).astype(np.float32)       # exact: hi is w rounded to 4 significant bits
+    lo = e4m3_decode(e4m3_encode_rn_sat(r))
+    return hi, lo
+
+
+def attend_fp8_pv(q, codes, scale, softmax_scale):
+    """Attention whose P.V product is taken in e4m3 (the scope table's FP8-MMA variant, reading R21).
+
+    Scores and softmax are the decode's (keys dequantised by R3); the value rows are the exact e4m3
+    values C[t, :512] without their scale, and the scale moves into the weights:
+      x[t] = f32(softmax_scale) * q . K[t],   p[t] = exp(x[t] - max x),   l = sum_t p[t],
+      w[t] = f32(p[t] * s_t * 2^sigma)  with sigma = fp8_pv_sigma(max_t s_t),
+      (hi[t], lo[t]) = e4m3_split2(w[t]),
+      out[v] = 2^-sigma * sum_t (hi[t] + lo[t]) * C[t, v] / l,   lse = max x + ln l.
+    hi + lo is w to within 2^-8 of w (normal range), so out is attention over V[t] = s_t C[t]
+    (unrounded) up to that relative error of each weight.
+    """
+    q = np.asarray(q, dtype=np.float64)
+    s = np.asarray(scale, dtype=np.float32).astype(np.float64).reshape(-1)
+    K = dequant_rows(codes, s.astype(np.float32)[:, None])    # R3 dequant (bf16 values)
+    C = e4m3_decode(codes)
+    ss = float(np.float32(softmax_scale))
+    x = ss * (q @ K.T)
+    mx = x.max(axis=1, keepdims=True)
+    p = np.exp(x - mx)
+    l = p.sum(axis=1)
+    sigma = fp8_pv_sigma(s.max())
+    w = p * s[None, :] * 2.0 ** sigma
+    hi, lo = e4m3_split2(w)
+    out = ((hi + lo) @ C[:, :V_DIM]) * 2.0 ** (-sigma) / l[:, None]
+    lse = mx[:, 0] + np.log(l)
+    return out, lse
+
+
+def decode_fp8_pv(q, blocks, scales, cache_lengths, lookup_table, scales_lookup_table,
+                  max_prompt_length, layer_idx, softmax_scale, requests=None, heads=None):
+    """decode() with the FP8 P.V variant's arithmetic (one fp32 scale per token).
+
+    Same gather and visibility rules as decode(); rows not computed are NaN.
+    """
+    q = np.asarray(q)
+    if q.dtype == np.uint16:
+        q = bf16_bits_to_f64(q)
+    q = q.astype(np.float64)
+    B, T, H, D = q.shape
+    assert D == HEAD_DIM
+    if np.asarray(scales).shape[-1] != 1:
+        raise ValueError("the FP8 P.V variant takes one scale per token")
+    T = int(max_prompt_length)
+    L = np.asarray(cache_lengths).astype(np.int64) & 0xFFFFFFFF
+    n_all = num_keys(L, T)
+    out = np.full((B, T, H, V_DIM), np.nan)
+    lse = np.full((B, T, H), np.nan)
+    reqs = range(B) if requests is None else requests
+    hs = np.arange(H) if heads is None else np.asarray(heads)
+    for b in reqs:
+        codes, sc = gather_request(blocks, scales, lookup_table, scales_lookup_table, b, int(n_all[b]), layer_idx)
+        for i in range(T):
+            vis = int(L[b]) + i + 1
+            r = attend_fp8_pv(q[b, i, hs], codes[:vis], sc[:vis, 0], softmax_scale)
             out[b, i, hs] = r[0]
             lse[b, i, hs] = r[1]
     return out, lse
