@@ -44,6 +44,8 @@ def parse():
                     help="decode with g scales per token (head_dim_granularity), each over 576/g dims")
     ap.add_argument("--fold-scales", action="store_true",
                     help="time the scale-folding decode (per-token scale on score and weight columns)")
+    ap.add_argument("--e4m3-pv", action="store_true",
+                    help="time the decode whose value product runs on the e4m3 tensor-core path")
     ap.add_argument("--op", choices=["decode", "kv_store"], default="decode",
                     help="decode (the default contract line) or the KV-store step that fills the cache")
     ap.add_argument("--no-cpu-baseline", action="store_true")
@@ -163,7 +165,7 @@ def sum_over_ranks(dist, values, device):
     return [float(x) for x in t.tolist()]
 
 
-def cpu_oracle_baseline(inp, budget_s, rank_requests=None, fold=False):
+def cpu_oracle_baseline(inp, budget_s, rank_requests=None, fold=False, e4m3_pv=False):
     """The float64 oracle, as it stands, on whole requests of the same workload until ~budget_s."""
     import numpy as np
     from oracle import mla_oracle as O
@@ -178,7 +180,7 @@ def cpu_oracle_baseline(inp, budget_s, rank_requests=None, fold=False):
     order = rank_requests if rank_requests is not None else list(range(len(n)))
     done, nbytes = [], 0
     t0 = time.perf_counter()
-    fn = O.decode_scale_folded if fold else O.decode
+    fn = O.decode_scale_folded if fold else O.decode_fp8_pv if e4m3_pv else O.decode
     for b in order:
         fn(a["q"], a["blocks"], a["scales"], a["cache_lengths"], a["lookup_table"],
            a["scales_lookup_table"], a["max_prompt_length"], a["layer_idx"], a["softmax_scale"], requests=[b])
@@ -360,9 +362,12 @@ def main():
         from dataclasses import replace
         cfg = replace(cfg, name=f"{cfg.name}_g{args.scale_blocks}", scale_blocks=args.scale_blocks)
     fold = bool(args.fold_scales)
-    if fold:
+    pv = bool(args.e4m3_pv)
+    if fold and pv:
+        raise SystemExit("--fold-scales and --e4m3-pv select different kernels: pass at most one")
+    if fold or pv:
         from dataclasses import replace
-        cfg = replace(cfg, name=f"{cfg.name}_scale_folded")
+        cfg = replace(cfg, name=f"{cfg.name}_{'scale_folded' if fold else 'e4m3_pv'}")
     seed = rank_seed(cfg.seed, rank)
     inp = W.make_inputs(cfg, device="cuda", seed=seed)
     kv_bytes = inp.kv_scale_bytes()
@@ -377,7 +382,7 @@ def main():
     stream = torch.cuda.current_stream()
 
     def step():
-        M.decode_inputs(inp, out=out, lse=lse, stream=stream, fold_scales=fold)
+        M.decode_inputs(inp, out=out, lse=lse, stream=stream, fold_scales=fold, e4m3_pv=pv)
 
     for _ in range(max(3, args.warmup)):
         flush.zero_()
@@ -443,7 +448,7 @@ def main():
             if dslut is not None:
                 dslut.copy_(hslut, non_blocking=True)
             M.decode(dq, inp.blocks, inp.scales, dl, dlut, dslut, T, inp.max_cache_length, inp.layer_idx,
-                     inp.softmax_scale, out=out, lse=lse, stream=stream, fold_scales=fold)
+                     inp.softmax_scale, out=out, lse=lse, stream=stream, fold_scales=fold, e4m3_pv=pv)
             hout.copy_(out, non_blocking=True)
             hlse.copy_(lse, non_blocking=True)
 
@@ -474,12 +479,13 @@ def main():
     tflops_k = flops / (kern_ms * 1e-3) / 1e12
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        cpu = cpu_oracle_baseline(inp, args.cpu_seconds, fold=fold)
+        cpu = cpu_oracle_baseline(inp, args.cpu_seconds, fold=fold, e4m3_pv=pv)
     if rank == 0:
         line = {
             "metric": METRIC, "value": gbs, "unit": "GB/s", "n_gpus": world, "steps": K, "warmup": args.warmup,
             "ms_per_step": step_ms, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
-            "dtype": "e4m3 KV, bf16 MMA, fp32 accumulate", "data": "synthetic",
+            "dtype": ("e4m3 KV, bf16 Q.K^T MMA, e4m3 P.V MMA (two terms per weight), fp32 accumulate" if pv
+                      else "e4m3 KV, bf16 MMA, fp32 accumulate"), "data": "synthetic",
             "decode_tokens_per_s": B * T * world / (step_ms * 1e-3),
             "hbm_frac": gbs / world / peaks["hbm_gbs"],
             "config": {"workload": cfg.name, "config_index": args.config, "batch": B, "q_len": T,

@@ -141,6 +141,37 @@ mla_status_t mla_decode_paged_fp8_scale_folded(
     const mla_paged_shape_t* shape, void* out, float* lse, cudaStream_t stream);
 
 /*
+ * mla_decode_paged_fp8_e4m3_pv -- the decode with the value product taken on the e4m3 tensor-core
+ * path (kind::f8f6f4).  The pages' kernels compute the softmax-weighted sum of the value rows in
+ * bf16 after dequantising them; here the value rows stay e4m3 codes and the per-token scale moves
+ * into the weights, which are then represented by two e4m3 terms each.
+ *
+ * Scores, softmax and lse are those of mla_decode_paged_fp8 (keys dequantised to bf16 the same
+ * way).  With p_t = exp(x[t] - m) and sigma = floor(log2(112 / max_t s_t)):
+ *     w_t = p_t * s_t * 2^sigma,  hi_t = e4m3_rn_sat(w_t),  lo_t = e4m3_rn_sat(w_t - hi_t),
+ *     out[b,i,h,:] = 2^-sigma * sum_t (hi_t + lo_t) e4m3(code_t)[0:512] / sum_t p_t.
+ * hi_t + lo_t equals w_t to within 2^-8 of w_t in the normal e4m3 range (2^-10 absolute below it),
+ * so out is attention over the unrounded values s_t * e4m3(code_t) up to that error per weight.
+ * The largest weight lies in (56, 112], so the weights use the top of the e4m3 range.  The kernel
+ * takes m and sigma per split of the keys (a running maximum of the scores that may trail the true
+ * one by up to 2 in log2 units, so p_t <= 4 and w_t <= 448, and a running minimum of sigma over
+ * the scales seen so far); its weights are therefore those of the formula times a factor >= 1, and
+ * its result differs from a whole-row evaluation by roundings inside the same bound, not bit for
+ * bit.  On the moderate-batch workload (32 requests, 1k-4k keys) it is closer to attention over the
+ * unrounded values s_t * e4m3(code_t) than mla_decode_paged_fp8, whose bf16 values carry a 2^-9
+ * relative rounding each.
+ *
+ * Arguments, ownership, workspace and errors as for mla_decode_paged_fp8_scale_folded, with the
+ * same limits (head_dim_granularity 1, e4m3 NaN codes not propagated, the full 227 KB of shared
+ * memory with the same MLA_ERR_UNSUPPORTED report from mla_get_device_status).
+ */
+mla_status_t mla_decode_paged_fp8_e4m3_pv(
+    const void* q, const void* blocks, const float* scales,
+    const uint32_t* cache_lengths, const uint32_t* lookup_table, const uint32_t* scales_lookup_table,
+    uint32_t max_prompt_length, uint32_t max_cache_length, uint32_t layer_idx, float softmax_scale,
+    const mla_paged_shape_t* shape, void* out, float* lse, cudaStream_t stream);
+
+/*
  * mla_decode_paged_fp8_noalloc -- the same decode, for callers that cannot allocate device memory
  * (for instance while a CUDA graph is being captured, under an allocator that owns the whole
  * device, or in a service that forbids allocation once it is running).  The reference pages have

@@ -350,12 +350,16 @@ def decode_scale_folded(q, blocks, scales, cache_lengths, lookup_table, scales_l
 # FP8 P.V variant (per-token scales only)
 # ----------------------------------------------------------------------------
 E4M3_MAX = 448.0
-FP8_PV_HEADROOM = 1.75          # 448 / 2^8: the folded weight p * s * 2^sigma stays below 448 for p <= 2^8
+FP8_PV_HEADROOM = 112.0
 
 
 def fp8_pv_sigma(s_max):
     """Power-of-two exponent of the folded weights: the largest integer sigma with
-    s_max * 2^sigma <= 1.75, so that p * s * 2^sigma <= 448 for every weight p <= 2^8."""
+    s_max * 2^sigma <= 112 = 448 / 4.  Every weight p * s * 2^sigma then stays at or below 448
+    for p <= 4, which leaves an implementation room for a running maximum that trails the true
+    one by up to 2 (log2 units); here p <= 1, so the largest weight lies in (56, 112] and the
+    weights fill the top of the e4m3 range (the normal range, 4 significant bits, reaches down to
+    2^-6, i.e. 2^-13 of the largest weight)."""
     return int(np.floor(np.log2(FP8_PV_HEADROOM / float(s_max))))
 
 

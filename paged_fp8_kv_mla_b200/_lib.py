@@ -24,7 +24,7 @@ EXPORTED = ["mla_decode_paged_fp8", "mla_gather_dequant_bf16", "mla_set_num_clus
             "mla_get_num_clusters", "mla_last_error_string", "mla_get_device_status",
             "mla_release_workspace", "mla_version", "mla_set_timing_events", "mla_decode_paged_fp8_noalloc",
             "mla_kv_store_fp8", "mla_decode_paged_fp8_scale_folded", "mla_merge_lse_parts_bf16",
-            "mla_set_wait_limit_ns", "mla_debug_withhold_arrival_once"]
+            "mla_set_wait_limit_ns", "mla_debug_withhold_arrival_once", "mla_decode_paged_fp8_e4m3_pv"]
 
 
 class MlaError(RuntimeError):
@@ -58,6 +58,8 @@ def load(path: str = LIB_PATH) -> ctypes.CDLL:
     lib.mla_merge_lse_parts_bf16.restype = ctypes.c_int
     lib.mla_decode_paged_fp8_scale_folded.argtypes = lib.mla_decode_paged_fp8.argtypes
     lib.mla_decode_paged_fp8_scale_folded.restype = ctypes.c_int
+    lib.mla_decode_paged_fp8_e4m3_pv.argtypes = lib.mla_decode_paged_fp8.argtypes
+    lib.mla_decode_paged_fp8_e4m3_pv.restype = ctypes.c_int
     lib.mla_decode_paged_fp8_noalloc.argtypes = [vp, vp, vp, vp, vp, vp, u32, u32, u32, f32,
                                                  ctypes.POINTER(PagedShape), vp, vp, vp]
     lib.mla_decode_paged_fp8_noalloc.restype = ctypes.c_int
@@ -175,14 +177,17 @@ def _check_decode(q, blocks, scales, cache_lengths, lookup_table, scales_lookup_
 
 def decode(q, blocks, scales, cache_lengths, lookup_table, scales_lookup_table, max_prompt_length: int,
            max_cache_length: int, layer_idx: int, softmax_scale: float, out=None, lse=None, stream=None,
-           want_lse: bool = True, fold_scales: bool = False):
+           want_lse: bool = True, fold_scales: bool = False, e4m3_pv: bool = False):
     """mla_decode_paged_fp8 on torch tensors (all on the current CUDA device).
 
     q bf16 [B, T, H, 576]; blocks uint8 [NB, kv_dim, L, P, 1, 576]; scales fp32 [NSB, kv_dim, L, P, 1, g];
     cache_lengths / lookup_table / scales_lookup_table int32 tensors holding uint32 values.
-    fold_scales=True calls mla_decode_paged_fp8_scale_folded instead (g = 1 only).
+    fold_scales=True calls mla_decode_paged_fp8_scale_folded instead, e4m3_pv=True
+    mla_decode_paged_fp8_e4m3_pv (g = 1 only, at most one of the two).
     Returns (out bf16 [B, T, H, 512], lse fp32 [B, T, H] or None).
     """
+    if fold_scales and e4m3_pv:
+        raise ValueError("fold_scales and e4m3_pv select different kernels: pass at most one")
     _check_decode(q, blocks, scales, cache_lengths, lookup_table, scales_lookup_table, out, lse)
     lib = load()
     B, T, H, D = q.shape
@@ -191,7 +196,8 @@ def decode(q, blocks, scales, cache_lengths, lookup_table, scales_lookup_table, 
     if lse is None and want_lse:
         lse = torch.empty((B, T, H), dtype=torch.float32, device=q.device)
     shp = paged_shape(B, H, blocks, scales, lookup_table)
-    fn = lib.mla_decode_paged_fp8_scale_folded if fold_scales else lib.mla_decode_paged_fp8
+    fn = (lib.mla_decode_paged_fp8_scale_folded if fold_scales else
+          lib.mla_decode_paged_fp8_e4m3_pv if e4m3_pv else lib.mla_decode_paged_fp8)
     st = fn(_ptr(q), _ptr(blocks), _ptr(scales), _ptr(cache_lengths), _ptr(lookup_table), _ptr(scales_lookup_table),
             int(max_prompt_length), int(max_cache_length), int(layer_idx), float(softmax_scale), ctypes.byref(shp),
             _ptr(out), _ptr(lse), _stream(stream))

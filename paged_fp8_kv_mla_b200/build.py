@@ -23,8 +23,8 @@ def _deps():
     return sorted(os.path.join(d, f) for f in os.listdir(d) if f.endswith((".cu", ".cuh"))) + \
         [os.path.join(ROOT, "include", "mla_paged_fp8.h")]
 LIB = os.path.join(PKG, "libmla_paged_fp8.so")
-# Diagnostic variant with the decode kernel's per-stage %clock64 stamps compiled in (read by
-# paged_fp8_kv_mla_b200.trace); never the library the product path loads.
+# Diagnostic variant with the decode kernel's per-stage timer stamps compiled in (written to a
+# device buffer the caller registers); never the library the product path loads.
 TRACE_LIB = os.path.join(PKG, "libmla_paged_fp8_trace.so")
 
 

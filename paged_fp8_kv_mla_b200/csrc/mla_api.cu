@@ -105,6 +105,8 @@ mla_status_t device_setup(int dev, int* nc_out) {
                                   cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(mla::SMEM_ALLOC)));
     MLA_CUDA(cudaFuncSetAttribute(mla::mla_decode_kernel<mla::SCALE_FOLD>,
                                   cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(mla::SMEM_ALLOC_FOLD)));
+    MLA_CUDA(cudaFuncSetAttribute(mla::mla_decode_kernel<mla::SCALE_FP8PV>,
+                                  cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(mla::SMEM_ALLOC_FOLD)));
     MLA_CUDA(cudaFuncSetAttribute(mla::mla_dequant_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                   static_cast<int>(mla::DQ_SMEM_ALLOC)));
     MLA_CUDA(cudaFuncSetAttribute(mla::mla_dequant_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
@@ -123,13 +125,15 @@ mla_status_t device_setup(int dev, int* nc_out) {
     attr[0].val.clusterDim.z = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
-    int n = 0, n_bs = 0, n_fold = 0;
+    int n = 0, n_bs = 0, n_fold = 0, n_f8 = 0;
     MLA_CUDA(cudaOccupancyMaxActiveClusters(&n, mla::mla_decode_kernel<mla::SCALE_TOKEN>, &cfg));
     MLA_CUDA(cudaOccupancyMaxActiveClusters(&n_bs, mla::mla_decode_kernel<mla::SCALE_BLOCK>, &cfg));
     cfg.dynamicSmemBytes = mla::SMEM_ALLOC_FOLD;
     MLA_CUDA(cudaOccupancyMaxActiveClusters(&n_fold, mla::mla_decode_kernel<mla::SCALE_FOLD>, &cfg));
+    MLA_CUDA(cudaOccupancyMaxActiveClusters(&n_f8, mla::mla_decode_kernel<mla::SCALE_FP8PV>, &cfg));
     n = n < n_bs ? n : n_bs;
     n = n < n_fold ? n : n_fold;
+    n = n < n_f8 ? n : n_f8;
     if (n <= 0) return fail(MLA_ERR_UNSUPPORTED, "no 2-CTA cluster of the decode kernel fits on this device");
     g_default_nc[dev] = n;
   }
@@ -270,7 +274,7 @@ void set_wait_params(mla::DecodeParams* p) {
 // predecessor's results with griddepcontrol.wait.  With timing events set, the events bracket the
 // decode launch (the event between plan and decode then serialises the two).
 mla_status_t launch_path(const mla::DecodeParams& p, int NC, const uint32_t* cache_lengths, uint32_t max_cache_length,
-                         cudaStream_t stream, bool timing, bool fold = false) {
+                         cudaStream_t stream, bool timing, int mode = mla::SCALE_TOKEN) {
   mla::mla_plan_kernel<<<1, mla::PLAN_THREADS, 0, stream>>>(
       cache_lengths, p.B, p.T, p.G, max_cache_length, NC, const_cast<int32_t*>(p.item_start),
       const_cast<int32_t*>(p.item_nvis), const_cast<int32_t*>(p.cluster_first), const_cast<int32_t*>(p.hdr), p.status);
@@ -279,7 +283,8 @@ mla_status_t launch_path(const mla::DecodeParams& p, int NC, const uint32_t* cac
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(2 * NC);
   cfg.blockDim = dim3(mla::NUM_THREADS);
-  cfg.dynamicSmemBytes = fold ? mla::SMEM_ALLOC_FOLD : mla::SMEM_ALLOC;
+  const bool scales_in_smem = mode == mla::SCALE_FOLD || mode == mla::SCALE_FP8PV;
+  cfg.dynamicSmemBytes = scales_in_smem ? mla::SMEM_ALLOC_FOLD : mla::SMEM_ALLOC;
   cfg.stream = stream;
   cudaLaunchAttribute attr[2];
   attr[0].id = cudaLaunchAttributeClusterDimension;
@@ -291,8 +296,10 @@ mla_status_t launch_path(const mla::DecodeParams& p, int NC, const uint32_t* cac
   cfg.attrs = attr;
   cfg.numAttrs = 2;
   if (timing) MLA_CUDA(cudaEventRecord(g_ev_before, stream));
-  if (fold) {
+  if (mode == mla::SCALE_FOLD) {
     MLA_CUDA(cudaLaunchKernelEx(&cfg, mla::mla_decode_kernel<mla::SCALE_FOLD>, p));
+  } else if (mode == mla::SCALE_FP8PV) {
+    MLA_CUDA(cudaLaunchKernelEx(&cfg, mla::mla_decode_kernel<mla::SCALE_FP8PV>, p));
   } else if (p.SG > 1) {
     MLA_CUDA(cudaLaunchKernelEx(&cfg, mla::mla_decode_kernel<mla::SCALE_BLOCK>, p));
   } else {
@@ -404,19 +411,23 @@ int32_t mla_get_num_clusters(void) {
 }  // extern "C"
 
 namespace {
-// Body of mla_decode_paged_fp8 and mla_decode_paged_fp8_scale_folded (workspace from the pool).
+// Body of mla_decode_paged_fp8, mla_decode_paged_fp8_scale_folded and mla_decode_paged_fp8_e4m3_pv
+// (workspace from the pool).  mode: mla::SCALE_TOKEN (per-token or block scales by the shape),
+// mla::SCALE_FOLD or mla::SCALE_FP8PV.
 mla_status_t decode_alloc(const void* q, const void* blocks, const float* scales, const uint32_t* cache_lengths,
                           const uint32_t* lookup_table, const uint32_t* scales_lookup_table,
                           uint32_t max_prompt_length, uint32_t max_cache_length, uint32_t layer_idx,
                           float softmax_scale, const mla_paged_shape_t* shape, void* out, float* lse,
-                          cudaStream_t stream, bool fold) {
+                          cudaStream_t stream, int mode) {
   mla::DecodeParams p{};
   uint64_t rows = 0;
   mla_status_t st = check_cache(blocks, scales, cache_lengths, lookup_table, max_prompt_length, max_cache_length,
                                 layer_idx, shape, &p, &rows);
   if (st != MLA_OK) return st;
-  if (fold && p.SG != 1)
+  if (mode == mla::SCALE_FOLD && p.SG != 1)
     return fail(MLA_ERR_UNSUPPORTED, "the scale-folding decode takes one scale per token (head_dim_granularity 1)");
+  if (mode == mla::SCALE_FP8PV && p.SG != 1)
+    return fail(MLA_ERR_UNSUPPORTED, "the e4m3 P.V decode takes one scale per token (head_dim_granularity 1)");
   if (!q || !out) return fail(MLA_ERR_INVALID_ARG, "q and out must be non-NULL");
   if (!aligned16(q) || !aligned16(out)) return fail(MLA_ERR_INVALID_ARG, "q and out must be 16-byte aligned");
   if (!(softmax_scale == softmax_scale)) return fail(MLA_ERR_INVALID_ARG, "softmax_scale is NaN");
@@ -458,7 +469,7 @@ mla_status_t decode_alloc(const void* q, const void* blocks, const float* scales
   p.trace = g_trace;
 #endif
 
-  return launch_path(p, NC, cache_lengths, max_cache_length, stream, g_ev_before && g_ev_after, fold);
+  return launch_path(p, NC, cache_lengths, max_cache_length, stream, g_ev_before && g_ev_after, mode);
 }
 }  // namespace
 
@@ -470,7 +481,7 @@ mla_status_t mla_decode_paged_fp8(const void* q, const void* blocks, const float
                                   uint32_t max_cache_length, uint32_t layer_idx, float softmax_scale,
                                   const mla_paged_shape_t* shape, void* out, float* lse, cudaStream_t stream) {
   return decode_alloc(q, blocks, scales, cache_lengths, lookup_table, scales_lookup_table, max_prompt_length,
-                      max_cache_length, layer_idx, softmax_scale, shape, out, lse, stream, false);
+                      max_cache_length, layer_idx, softmax_scale, shape, out, lse, stream, mla::SCALE_TOKEN);
 }
 
 mla_status_t mla_decode_paged_fp8_scale_folded(const void* q, const void* blocks, const float* scales,
@@ -480,7 +491,16 @@ mla_status_t mla_decode_paged_fp8_scale_folded(const void* q, const void* blocks
                                                const mla_paged_shape_t* shape, void* out, float* lse,
                                                cudaStream_t stream) {
   return decode_alloc(q, blocks, scales, cache_lengths, lookup_table, scales_lookup_table, max_prompt_length,
-                      max_cache_length, layer_idx, softmax_scale, shape, out, lse, stream, true);
+                      max_cache_length, layer_idx, softmax_scale, shape, out, lse, stream, mla::SCALE_FOLD);
+}
+
+mla_status_t mla_decode_paged_fp8_e4m3_pv(const void* q, const void* blocks, const float* scales,
+                                          const uint32_t* cache_lengths, const uint32_t* lookup_table,
+                                          const uint32_t* scales_lookup_table, uint32_t max_prompt_length,
+                                          uint32_t max_cache_length, uint32_t layer_idx, float softmax_scale,
+                                          const mla_paged_shape_t* shape, void* out, float* lse, cudaStream_t stream) {
+  return decode_alloc(q, blocks, scales, cache_lengths, lookup_table, scales_lookup_table, max_prompt_length,
+                      max_cache_length, layer_idx, softmax_scale, shape, out, lse, stream, mla::SCALE_FP8PV);
 }
 
 mla_status_t mla_gather_dequant_bf16(const void* blocks, const float* scales, const uint32_t* cache_lengths,
@@ -685,7 +705,8 @@ mla_status_t mla_get_device_status(cudaStream_t stream) {
   if (v & mla::STATUS_TIMEOUT) return fail(MLA_ERR_TIMEOUT, "a kernel wait timed out (status 0x%x)", v);
   if (v & mla::STATUS_BOUNDS) return fail(MLA_ERR_DEVICE_BOUNDS, "page id or cache length out of range (status 0x%x)", v);
   if (v & mla::STATUS_LAYOUT)
-    return fail(MLA_ERR_UNSUPPORTED, "dynamic shared memory base not aligned as the scale-folding decode needs (status 0x%x)", v);
+    return fail(MLA_ERR_UNSUPPORTED,
+                "dynamic shared memory base not aligned as the scale-folding and e4m3 P.V decodes need (status 0x%x)", v);
   return MLA_OK;
 }
 

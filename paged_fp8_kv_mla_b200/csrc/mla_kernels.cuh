@@ -96,15 +96,31 @@ static_assert(RING_STAGE % 16 == 0 && SRING % 16 == 0, "bulk copies need 16-byte
 constexpr uint32_t SSC = SMEM_USED;
 constexpr uint32_t SSC_STRIDE = 64 * 4;
 constexpr uint32_t SSC_SLOTS = 8;
+// FP8 P.V mode only: per scale slot, the largest scale of the tile seen by each of the four
+// converter warps that write SSC ([8][4] f32).
+constexpr uint32_t SSMAX = SSC + SSC_SLOTS * SSC_STRIDE;
 constexpr uint32_t SMEM_ALLOC_FOLD = 232448;
-constexpr uint32_t SMEM_FOLD_MAX_PAD = SMEM_ALLOC_FOLD - SSC - SSC_SLOTS * SSC_STRIDE;
-static_assert(SMEM_ALLOC_FOLD >= SSC + SSC_SLOTS * SSC_STRIDE, "fold scale array does not fit");
+constexpr uint32_t SMEM_FOLD_MAX_PAD = SMEM_ALLOC_FOLD - SSMAX - SSC_SLOTS * 16;
+static_assert(SMEM_ALLOC_FOLD >= SSMAX + SSC_SLOTS * 16, "fold scale array does not fit");
+// FP8 P.V mode: the V operand is raw e4m3, double buffered in the bf16 V buffer's place: buffer b
+// at SV + b * SV8_STRIDE holds 2 atom columns (128 dims each: D_c's two halves) of 64 key rows at
+// 128 B, SWIZZLE_128B, 8-row groups 1 KB apart.  P keeps its buffer: row r holds the hi codes of the
+// 64 keys in bytes 0..63 and the lo codes in bytes 64..127 (same 128-byte swizzle).
+constexpr uint32_t SV8_STRIDE = 16384;
+constexpr uint32_t SV8_ATOM = 8192;
+static_assert(2 * SV8_STRIDE <= SV_BYTES, "FP8 V buffers do not fit the V buffer");
+// e4m3 P.V mode: the largest folded scale s_max * 2^sigma is at most 448 / 4, and the softmax keeps
+// its reference maximum within 2 (log2 units) of the running maximum, so p <= 4 and every weight
+// p * s * 2^sigma <= 448.
+constexpr float FP8_PV_LAZY_LOG2 = 2.f;
 
 // How the per-token scale enters the computation.
 enum ScaleMode : int {
   SCALE_TOKEN = 0,   // K, V = bf16_rn(f32_rn(e4m3 * s_t)), one scale per token
   SCALE_BLOCK = 1,   // the same with g scales per token, each over 576 / g contiguous dims
-  SCALE_FOLD = 2     // K, V = exact e4m3 values; s_t scales score column t and weight column t
+  SCALE_FOLD = 2,    // K, V = exact e4m3 values; s_t scales score column t and weight column t
+  SCALE_FP8PV = 3    // K as SCALE_TOKEN; P.V in e4m3: V = raw e4m3 bytes, s_t (and 2^sigma) carried by
+                     // the weights, each weight split into two e4m3 terms
 };
 
 enum Bar : uint32_t {
@@ -143,6 +159,7 @@ static_assert(T_Q + 32 * Q_TMEM_ATOMS <= TMEM_COLS, "tensor memory map overflows
 
 constexpr uint32_t IDESC_QK = ptx::idesc_bf16_f32(128, BN, false, false);
 constexpr uint32_t IDESC_PV = ptx::idesc_bf16_f32(128, 256, false, true);
+constexpr uint32_t IDESC_PV8 = ptx::idesc_e4m3_f32(128, 256, false, true);
 
 constexpr unsigned STATUS_BOUNDS = 1u;
 constexpr unsigned STATUS_TIMEOUT = 2u;
@@ -389,11 +406,12 @@ __device__ __forceinline__ void st_chunk(uint32_t atom_base, int row, int cq, co
 // Converter thread layout.  Thread t (0..383) is in group q = t / 128; thread tau = t % 128 of a
 // group owns key row conv_row(tau) (0..31) and chunk position conv_cq(tau) (0..3) of each 64-dim
 // atom column the group handles.  The 8 threads of one 16-byte shared-memory phase cover the 4
-// chunk positions of two adjacent rows, so their stores land on 8 different 16-byte positions of
-// the 128-byte swizzle row (even rows on even positions, odd rows on odd ones), and their 16-byte
-// reads of the FP8 ring (576-byte rows: adjacent rows start 16 banks apart) hit 8 distinct bank
-// quads.
-__device__ __forceinline__ int conv_row(int tau) { return ((tau >> 3) << 1) | ((tau >> 2) & 1); }
+// chunk positions of rows r and r ^ 5 (r even), which differ in bits 0 and 2.  So their 32-byte
+// bf16 stores land on 8 different 16-byte positions of the 128-byte swizzle row (even rows on even
+// positions, odd rows on odd ones); their 16-byte e4m3 stores (4 adjacent positions per row) land
+// in opposite halves of the swizzle row; and their 16-byte reads of the FP8 ring (576-byte rows:
+// rows an odd number apart start 16 banks apart) hit 8 distinct bank quads.
+__device__ __forceinline__ int conv_row(int tau) { return ((tau >> 3) << 1) ^ (((tau >> 2) & 1) * 5); }
 __device__ __forceinline__ int conv_cq(int tau) { return tau & 3; }
 
 // V atom column va (0..3) of CTA c's V operand holds the 64 dims of absolute atom column
@@ -791,6 +809,149 @@ __device__ __forceinline__ void converter_role(const DecodeParams& p, int k, uin
 #undef BAR
 }
 
+// Largest power of two 2^sigma with s_max * 2^sigma <= 112 = 1.75 * 2^6 (s_max a positive normal
+// float), so that every folded weight p * s * 2^sigma with p <= 4 stays at or below 448:
+// sigma = 133 - e - (m > 1.75), e the biased exponent and m the significand of s_max.  Clamped to
+// [-120, 120].
+__device__ __forceinline__ int fp8_pv_sigma(float s_max) {
+  if (!(s_max > 0.f)) return 120;
+  const uint32_t b = __float_as_uint(s_max);
+  const int e = static_cast<int>((b >> 23) & 0xFFu);
+  const int sg = 133 - e - ((b & 0x7FFFFFu) > 0x600000u ? 1 : 0);
+  return max(-120, min(120, sg));
+}
+
+__device__ __forceinline__ float exp2i(int k) { return __int_as_float((k + 127) << 23); }   // 2^k, |k| <= 126
+__device__ __forceinline__ float exp2i_or_zero(int k) { return k < -126 ? 0.f : exp2i(k); }   // 2^k, k <= 126
+
+// Two-term e4m3 split of two weights w0, w1 >= 0: hi = e4m3_rn_sat(w), lo = e4m3_rn_sat(w - hi); the
+// residual is exact in f32 (hi is w rounded to 4 significant bits, or 0).  w0's codes in the low bytes.
+__device__ __forceinline__ void split2_e4m3(float w0, float w1, uint32_t& hi, uint32_t& lo) {
+  const uint16_t h = ptx::e4m3x2_rn_satfinite(w0, w1);
+  const uint32_t hf = ptx::e4m3x2_to_f16x2(h);
+  hi = h;
+  lo = ptx::e4m3x2_rn_satfinite(w0 - ptx::f16_lo_to_f32(hf), w1 - ptx::f16_hi_to_f32(hf));
+}
+
+// 16-byte unit (0..7) of a P row that holds a softmax thread's chunk j (0..3) of its key half hh:
+// bf16 P: the thread's 32 weights at units 4hh..4hh+3; e4m3 P: its 32 hi codes at units 2hh, 2hh+1
+// and its 32 lo codes at units 4+2hh, 5+2hh.
+template <bool F8>
+__device__ __forceinline__ int p_unit(int hh, int j) {
+  return F8 ? ((j >> 1) << 2) + 2 * hh + (j & 1) : 4 * hh + j;
+}
+
+// =============================================================================================
+// converter role, FP8 P.V mode (warps 0-11).  Step g: read tile g's FP8 chunks and scales from ring
+// stage g % 2, hand the tile's 64 per-token scales and its largest scale to the softmax, release
+// the stage; once Q.K^T(g-2) has finished dequantise the K half into buffer g % 2 (as the per-token
+// mode does); once P.V(g-2) has finished write tile g's V operand into FP8 buffer g % 2 as raw e4m3
+// bytes: the own key's D_c chunks (from the ring reads above) and the other key's D_c chunks
+// (loaded from global memory during step g-1).  Then load the other key's chunks of tile g+1.
+// =============================================================================================
+__device__ __forceinline__ void converter_role_fp8pv(const DecodeParams& p, int k, uint32_t base, int lane,
+                                                     volatile uint32_t* abort, uint32_t peer_abort, uint32_t c) {
+  const int C = static_cast<int>(c);
+  const int t = threadIdx.x;
+  const int grp = t / CONV_GROUP, tau = t % CONV_GROUP;
+  const int r = conv_row(tau), cq = conv_cq(tau);
+  const bool extra = grp == extra_group(C);
+  const uint64_t lim = p.wait_limit_ns;
+#define BAR(i) (base + SBAR + 8u * (i))
+#define MLA_WAIT_RET(b_, parity)                                                               \
+  if (!__all_sync(0xffffffffu, wait_bar((b_), (parity), abort, p.status, peer_abort, lim))) return;
+#define MLA_POLL_RET(b_, parity)                                                               \
+  if (!__all_sync(0xffffffffu, poll_bar((b_), (parity), abort, p.status, peer_abort, lim))) return;
+  const uint32_t k_full0 = ptx::mapa(BAR(B_K_FULL), 0), v_full0 = ptx::mapa(BAR(B_V_FULL), 0);
+  const uint4 zero4 = make_uint4(0u, 0u, 0u, 0u);
+  const float no_blk[3] = {0.f, 0.f, 0.f};
+  TileStream ts(p, k);
+  TileInfo kt = ts.take(p);
+  if (!kt.valid) return;
+  TileInfo nt = ts.take(p);
+  Ahead A;
+  A.oth_ok = false;
+  A.own_ok = true;
+  OthLut L = oth_lut_issue(p, kt, C, r);
+  if (!fetch_oth<false>(p, L, C, grp, cq, extra, A)) raise_status(p.status, STATUS_BOUNDS);
+  if (nt.valid) L = oth_lut_issue(p, nt, C, r);
+  uint32_t g = 0;
+  while (true) {
+    const uint32_t st = g & 1;
+    MLA_WAIT_RET(BAR(B_RING_FULL + st), (g >> 1) & 1);
+    const uint32_t stage = base + SRING + st * RING_STAGE;
+    const uint32_t mask = ptx::ld_shared_u32(base + S_MASK + 8 * st);
+    const uint32_t omask = ptx::ld_shared_u32(base + S_MASK + 8 * st + 4);
+    const bool own_ok = ((mask >> r) & 1u) != 0;
+    uint4 raw[3];
+#pragma unroll
+    for (int m = 0; m < 3; ++m) raw[m] = ptx::ld_shared_v4(stage + r * HEAD_DIM + 16 * (4 * (3 * grp + m) + cq));
+    const float s_own = ptx::ld_shared_f32(stage + RING_ROWS + 4 * r);
+    // the tile's 64 per-token scales and its largest scale for the softmax (slot g % 8; the softmax
+    // finished tile g - 8 before S_FREE(g - 5), which Q.K^T(g - 3) waited for before the K-buffer
+    // wait of step g - 1 passed)
+    if (grp == 0) {
+      float mx = 0.f;
+      if (cq == 0) {
+        const float so = own_ok ? s_own : 0.f;
+        const float sx = ((omask >> r) & 1u) ? ptx::ld_shared_f32(stage + RING_OSC + 4 * r) : 0.f;
+        const uint32_t sa = base + SSC + (g % SSC_SLOTS) * SSC_STRIDE + 4 * r;
+        ptx::st_shared_f32(sa + 4 * HALF_BN * C, so);
+        ptx::st_shared_f32(sa + 4 * HALF_BN * (1 - C), sx);
+        mx = fmaxf(so, sx);
+      }
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+      if (lane == 0) ptx::st_shared_f32(base + SSMAX + (g % SSC_SLOTS) * 16 + 4 * (t >> 5), mx);
+    }
+    __syncwarp();
+    if (lane == 0) {
+      ptx::mbar_arrive(BAR(B_SC_FULL + (g % SSC_SLOTS)));
+      ptx::mbar_arrive(BAR(B_RING_EMPTY + st));    // the reads above are ordered before it
+    }
+    // K half buffer g % 2: free once Q.K^T(g - 2) has finished
+    MLA_POLL_RET(BAR(B_S_FULL + st), ((g >> 1) & 1) ^ 1);
+    convert_k<false, false>(grp, r, cq, own_ok, raw, s_own, no_blk, base + SK0 + st * SK_STRIDE);
+    ptx::fence_proxy_async_smem();
+    __syncwarp();
+    if (lane == 0) ptx::mbar_arrive_cluster(k_full0 + 8u * st);
+    // FP8 V buffer g % 2: free once P.V(g - 2) has finished
+    MLA_WAIT_RET(BAR(B_PV_DONE + st), ((g >> 1) & 1) ^ 1);
+    {
+      const uint32_t sv8 = base + SV + st * SV8_STRIDE;
+#pragma unroll
+      for (int m = 0; m < 3; ++m) {
+        const int a = 3 * grp + m;
+        if (!k_in_dc(a, C)) continue;
+        const uint4 v = own_ok ? raw[m] : zero4;
+        const uint32_t dst = sv8 + (((a >> 1) == C) ? 0u : SV8_ATOM) + sw128_off(HALF_BN * C + r, (a & 1) * 4 + cq);
+        ptx::st_shared_v4(dst, v.x, v.y, v.z, v.w);
+      }
+      const int vrow = HALF_BN * (1 - C) + r;
+      {
+        const uint4 v = A.oth_ok ? A.oth[0] : zero4;
+        ptx::st_shared_v4(sv8 + (grp >> 1) * SV8_ATOM + sw128_off(vrow, (grp & 1) * 4 + cq), v.x, v.y, v.z, v.w);
+      }
+      if (extra) {
+        const uint4 v = A.oth_ok ? A.oth[1] : zero4;
+        ptx::st_shared_v4(sv8 + SV8_ATOM + sw128_off(vrow, 4 + cq), v.x, v.y, v.z, v.w);
+      }
+    }
+    ptx::fence_proxy_async_smem();
+    __syncwarp();
+    if (lane == 0) ptx::mbar_arrive_cluster(v_full0 + 8u * st);
+    ++g;
+    if (!nt.valid) break;
+    if (!fetch_oth<false>(p, L, C, grp, cq, extra, A)) raise_status(p.status, STATUS_BOUNDS);
+    kt = nt;
+    nt = ts.take(p);
+    if (nt.valid) L = oth_lut_issue(p, nt, C, r);
+  }
+#undef MLA_POLL_RET
+#undef MLA_WAIT_RET
+#undef BAR
+}
+
 // =============================================================================================
 // producer role (lane 0 of warp 19): walks the cluster's tiles and fills ring stage g % 2 with the
 // own keys' rows (and per-token scales) of tile g once the converters have released the stage.
@@ -823,15 +984,18 @@ __device__ __forceinline__ void producer_role(const DecodeParams& p, int k, uint
 // =============================================================================================
 // decode kernel
 // =============================================================================================
-// MODE: a ScaleMode (per-token scales, block scales, or per-token scales folded into S and P).
+// MODE: a ScaleMode (per-token scales, block scales, per-token scales folded into S and P, or the
+// e4m3 P.V product).
 template <int MODE>
 __global__ void __launch_bounds__(NUM_THREADS, 1) mla_decode_kernel(const __grid_constant__ DecodeParams p) {
   constexpr bool FOLD = MODE == SCALE_FOLD;
+  constexpr bool F8 = MODE == SCALE_FP8PV;
+  constexpr bool SCALES = FOLD || F8;   // the converter hands per-token scales to the softmax
   if (threadIdx.x == 0) MLA_MARK_MIN(1);
   ptx::griddep_launch_dependents();   // the combine kernel may start launching (it waits for this grid)
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  if (FOLD && static_cast<uint32_t>(smem - smem_raw) > SMEM_FOLD_MAX_PAD) {
+  if (SCALES && static_cast<uint32_t>(smem - smem_raw) > SMEM_FOLD_MAX_PAD) {
     // every CTA of the launch sees the same base, so all of them leave here together
     if (threadIdx.x == 0) raise_status(p.status, STATUS_LAYOUT);
     return;
@@ -890,7 +1054,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) mla_decode_kernel(const __grid
 
   if (warp < CONV_WARPS) {
     // ------------------------------------------------------------------ converter
-    converter_role<MODE>(p, k, base, lane, abort, peer_abort, c);
+    if (F8) converter_role_fp8pv(p, k, base, lane, abort, peer_abort, c);
+    else converter_role<MODE>(p, k, base, lane, abort, peer_abort, c);
   } else if (warp < SM_WARP0 + 4) {
     // ------------------------------------------------------------------ softmax / epilogue
     const int t = threadIdx.x - 32 * SM_WARP0;
@@ -906,10 +1071,11 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) mla_decode_kernel(const __grid
     uint32_t g = 0, uu = 0;
     while (wk.next(p, u)) {
       float m_ref = -INFINITY, l = 0.f;
+      int sig = 0;   // e4m3 P.V: the unit's weights carry 2^sig (lowered, never raised, as tiles come in)
       for (int j = u.tb; j < u.te; ++j, ++g) {
         const uint32_t sb = g & 1;
         MLA_WAIT_WARP(BAR(B_S_FULL + sb), (g >> 1) & 1);
-        if (FOLD) MLA_WAIT_WARP(BAR(B_SC_FULL + (g % SSC_SLOTS)), (g / SSC_SLOTS) & 1);
+        if (SCALES) MLA_WAIT_WARP(BAR(B_SC_FULL + (g % SSC_SLOTS)), (g / SSC_SLOTS) & 1);
         if (t == 0) MLA_TRACE_EV(g, 8);
         ptx::tc_fence_after();
         float x[32];
@@ -959,15 +1125,49 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) mla_decode_kernel(const __grid
         if (t == 0) MLA_TRACE_EV(g, 10);
         float alpha = 1.f;
         bool rescale = false;
-        if (mt > m_ref + 8.f) {           // lazy max: keep the reference unless it grows by > 2^8
+        // lazy max: keep the reference unless it grows by more than 8 (2 for e4m3 weights) in log2 units
+        if (mt > m_ref + (F8 ? FP8_PV_LAZY_LOG2 : 8.f)) {
           alpha = (m_ref == -INFINITY) ? 0.f : ptx::ex2_approx(m_ref - mt);
           l *= alpha;
           rescale = (j != u.tb);
           m_ref = mt;
         }
+        // e4m3 P.V: sigma of this tile's largest scale; a drop scales O by 2^(new - old) as well
+        float sfac = 1.f;
+        if (F8) {
+          const uint4 m4 = ptx::ld_shared_v4(base + SSMAX + (g % SSC_SLOTS) * 16);
+          const float smx = fmaxf(fmaxf(__uint_as_float(m4.x), __uint_as_float(m4.y)),
+                                  fmaxf(__uint_as_float(m4.z), __uint_as_float(m4.w)));
+          const int st = fp8_pv_sigma(smx);
+          if (j == u.tb) {
+            sig = st;
+          } else if (st < sig) {
+            sfac = exp2i_or_zero(st - sig);
+            sig = st;
+          }
+        }
         float lsum = 0.f;
         uint32_t pw[16];
-        if (FOLD) {
+        if (F8) {
+          // l sums the weights p; P carries w = p * s_t * 2^sig as two e4m3 terms (p <= 4 under the
+          // lazy max, s_t * 2^sig <= 112, so w <= 448)
+          const float sf = exp2i(sig);
+#pragma unroll
+          for (int v = 0; v < 8; ++v) {
+            const uint4 s4 = ptx::ld_shared_v4(sc_addr + 16 * v);
+            const float p0 = ptx::ex2_approx(x[4 * v] - m_ref);
+            const float p1 = ptx::ex2_approx(x[4 * v + 1] - m_ref);
+            const float p2 = ptx::ex2_approx(x[4 * v + 2] - m_ref);
+            const float p3 = ptx::ex2_approx(x[4 * v + 3] - m_ref);
+            lsum += p0 + p1;
+            lsum += p2 + p3;
+            uint32_t h01, l01, h23, l23;
+            split2_e4m3(p0 * (__uint_as_float(s4.x) * sf), p1 * (__uint_as_float(s4.y) * sf), h01, l01);
+            split2_e4m3(p2 * (__uint_as_float(s4.z) * sf), p3 * (__uint_as_float(s4.w) * sf), h23, l23);
+            pw[v] = h01 | (h23 << 16);
+            pw[8 + v] = l01 | (l23 << 16);
+          }
+        } else if (FOLD) {
           // l sums the weights; the P operand carries weight * s_t
 #pragma unroll
           for (int v = 0; v < 8; ++v) {
@@ -999,12 +1199,14 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) mla_decode_kernel(const __grid
           const uint32_t sp = base + SP;
 #pragma unroll
           for (int v = 0; v < 4; ++v)
-            ptx::st_shared_v4(sp + sw128_off(r, 4 * hh + v), pw[4 * v], pw[4 * v + 1], pw[4 * v + 2], pw[4 * v + 3]);
+            ptx::st_shared_v4(sp + sw128_off(r, p_unit<F8>(hh, v)), pw[4 * v], pw[4 * v + 1], pw[4 * v + 2],
+                              pw[4 * v + 3]);
         }
         // O rescale (warp-collective TMEM access): a warp rescales when any of its rows moved its
-        // reference max; rows that did not move use alpha = 1
+        // reference max (or sigma dropped); rows that did not move use alpha = 1
         if (!rescale) alpha = 1.f;
-        if (__any_sync(0xffffffffu, rescale)) {
+        alpha *= sfac;
+        if (__any_sync(0xffffffffu, rescale) || sfac != 1.f) {
           ptx::tc_fence_after();
 #pragma unroll 1
           for (int ch = 0; ch < 8; ++ch) {
@@ -1034,17 +1236,22 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) mla_decode_kernel(const __grid
         if (lane == 0) ptx::mbar_arrive(BAR(B_REDL));
         MLA_WAIT_WARP(BAR(B_REDL), uu & 1);
         const float l_row = l + red_l[t ^ 64];
-        const float inv_l = 1.f / l_row;
+        const float inv_l = F8 ? exp2i(-sig) / l_row : 1.f / l_row;
         const int head = u.g * MROWS + HPC * static_cast<int>(c) + r;
         const bool row_ok = head < p.H;
         const float lse_v = (m_ref + ptx::lg2_approx(l_row)) * 0.69314718055994530942f;
-        // O / l goes out through a per-warp 2 KB staging block in the (now idle) P buffer: each
-        // thread writes 64 bytes of its row (32 bf16, or 16 fp32 per half of a chunk), then the warp
-        // stores whole 64-byte row segments; 16-byte chunk j of row x sits at x * 64 + 16 * (j ^
-        // ((x >> 1) & 3)), so both passes are conflict-free.
-        const uint32_t stage = base + SP + static_cast<uint32_t>(quad) * 2048u;
-        const int row0 = HPC * static_cast<int>(c) + 32 * (quad & 1);   // CTA row of this warp's lane 0
-        const uint32_t my = stage + lane * 64;
+        // O / l goes out through the P buffer, idle once the unit's last P.V has finished: each
+        // thread stages 64 bytes of its row (32 bf16, or 16 fp32 per half of a chunk) in the four
+        // 16-byte units of its own P row that it writes as P, then the warp stores whole 64-byte row
+        // segments.  A warp touches only its own P units, so a warp still in its epilogue is not
+        // disturbed by one that has begun the next unit.  The read-back takes rows x and x ^ PX in
+        // one 8-thread phase (PX = 4 for bf16 P, 2 for e4m3 P): their units sit in opposite halves
+        // of the swizzle row, so both passes are conflict-free.
+        const uint32_t sp = base + SP;
+        const int prow0 = 32 * (quad & 1);                                // P row of this warp's lane 0
+        const int row0 = HPC * static_cast<int>(c) + prow0;               // CTA row of this warp's lane 0
+        constexpr int PXB = F8 ? 1 : 2;
+        const int rb_j = lane & 3;
 #pragma unroll 1
         for (int ch = 0; ch < 8; ++ch) {
           uint32_t rr[32];
@@ -1058,13 +1265,14 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) mla_decode_kernel(const __grid
               const uint32_t w1 = ptx::pack_bf16x2(__uint_as_float(rr[8 * v + 2]) * inv_l, __uint_as_float(rr[8 * v + 3]) * inv_l);
               const uint32_t w2 = ptx::pack_bf16x2(__uint_as_float(rr[8 * v + 4]) * inv_l, __uint_as_float(rr[8 * v + 5]) * inv_l);
               const uint32_t w3 = ptx::pack_bf16x2(__uint_as_float(rr[8 * v + 6]) * inv_l, __uint_as_float(rr[8 * v + 7]) * inv_l);
-              ptx::st_shared_v4(my + 16 * (v ^ ((lane >> 1) & 3)), w0, w1, w2, w3);
+              ptx::st_shared_v4(sp + sw128_off(prow0 + lane, p_unit<F8>(hh, v)), w0, w1, w2, w3);
             }
             __syncwarp();
 #pragma unroll
             for (int it = 0; it < 4; ++it) {
-              const int x = it * 8 + (lane >> 2), j = lane & 3;
-              const uint4 w = ptx::ld_shared_v4(stage + x * 64 + 16 * (j ^ ((x >> 1) & 3)));
+              const int n = 4 * it + (lane >> 3), j = rb_j;
+              const int x = ((n >> PXB) << (PXB + 1)) | (n & ((1 << PXB) - 1)) | (((lane >> 2) & 1) << PXB);
+              const uint4 w = ptx::ld_shared_v4(sp + sw128_off(prow0 + x, p_unit<F8>(hh, j)));
               const int hd = u.g * MROWS + row0 + x;
               if (hd < p.H)
                 *reinterpret_cast<uint4*>(p.out + ((static_cast<size_t>(u.b) * p.T + u.i) * p.H + hd) * V_DIM + dv + 8 * j) = w;
@@ -1074,7 +1282,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) mla_decode_kernel(const __grid
             for (int hf = 0; hf < 2; ++hf) {
 #pragma unroll
               for (int v = 0; v < 4; ++v)
-                ptx::st_shared_v4(my + 16 * (v ^ ((lane >> 1) & 3)),
+                ptx::st_shared_v4(sp + sw128_off(prow0 + lane, p_unit<F8>(hh, v)),
                                   __float_as_uint(__uint_as_float(rr[16 * hf + 4 * v + 0]) * inv_l),
                                   __float_as_uint(__uint_as_float(rr[16 * hf + 4 * v + 1]) * inv_l),
                                   __float_as_uint(__uint_as_float(rr[16 * hf + 4 * v + 2]) * inv_l),
@@ -1082,8 +1290,9 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) mla_decode_kernel(const __grid
               __syncwarp();
 #pragma unroll
               for (int it = 0; it < 4; ++it) {
-                const int x = it * 8 + (lane >> 2), j = lane & 3;
-                const uint4 w = ptx::ld_shared_v4(stage + x * 64 + 16 * (j ^ ((x >> 1) & 3)));
+                const int n = 4 * it + (lane >> 3), j = rb_j;
+                const int x = ((n >> PXB) << (PXB + 1)) | (n & ((1 << PXB) - 1)) | (((lane >> 2) & 1) << PXB);
+                const uint4 w = ptx::ld_shared_v4(sp + sw128_off(prow0 + x, p_unit<F8>(hh, j)));
                 *reinterpret_cast<uint4*>(p.part_o + (static_cast<size_t>(u.slot) * MROWS + row0 + x) * V_DIM + dv +
                                           16 * hf + 4 * j) = w;
               }
@@ -1206,7 +1415,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) mla_decode_kernel(const __grid
       TileCursor pc(p, k);
       uint32_t g = 0, up = 0;
       const uint64_t dp0 = ptx::smem_desc(base + SP, 16, 1024, ptx::SW_128B);
-      const uint64_t dv0 = ptx::smem_desc(base + SV, SV_ATOM, 1024, ptx::SW_128B);
+      const uint64_t dv0 = ptx::smem_desc(base + SV, F8 ? SV8_ATOM : SV_ATOM, 1024, ptx::SW_128B);
       while (pc.valid) {
         const uint32_t hb = g & 1;
         const bool first = pc.first;
@@ -1219,13 +1428,30 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) mla_decode_kernel(const __grid
         ptx::tc_fence_after();
         if (ptx::elect_one()) {
           MLA_TRACE_EV(g, 22);
+          if (F8) {
+            // e4m3: per 128-dim half jv, (hi, lo) x two 32-key K steps; A = P bytes 0..63 (hi) and
+            // 64..127 (lo) of each head row, B = V buffer g % 2 (one 128-dim atom column per CTA)
 #pragma unroll
-          for (int jv = 0; jv < 2; ++jv) {
+            for (int jv = 0; jv < 2; ++jv) {
 #pragma unroll
-            for (int kk = 0; kk < 4; ++kk) {
-              const uint64_t ad = dp0 + ((kk * 32) >> 4);
-              const uint64_t bd = dv0 + ((2 * jv * SV_ATOM + kk * 2048) >> 4);
-              ptx::mma_pair_ss(tbase + T_O + 128 * jv, ad, bd, IDESC_PV, (first && kk == 0) ? 0u : 1u);
+              for (int tm = 0; tm < 2; ++tm) {
+#pragma unroll
+                for (int kb = 0; kb < 2; ++kb) {
+                  const uint64_t ad = dp0 + ((64 * tm + 32 * kb) >> 4);
+                  const uint64_t bd = dv0 + ((hb * SV8_STRIDE + jv * SV8_ATOM + kb * 4096) >> 4);
+                  ptx::mma_pair_ss_f8(tbase + T_O + 128 * jv, ad, bd, IDESC_PV8, (first && (tm | kb) == 0) ? 0u : 1u);
+                }
+              }
+            }
+          } else {
+#pragma unroll
+            for (int jv = 0; jv < 2; ++jv) {
+#pragma unroll
+              for (int kk = 0; kk < 4; ++kk) {
+                const uint64_t ad = dp0 + ((kk * 32) >> 4);
+                const uint64_t bd = dv0 + ((2 * jv * SV_ATOM + kk * 2048) >> 4);
+                ptx::mma_pair_ss(tbase + T_O + 128 * jv, ad, bd, IDESC_PV, (first && kk == 0) ? 0u : 1u);
+              }
             }
           }
           ptx::mma_commit_pair(BAR(B_PV_DONE + hb), 0x3);

@@ -287,6 +287,14 @@ __device__ __forceinline__ float f16_hi_to_f32(uint32_t h2) {
   return f;
 }
 
+// Two f32 to two e4m3 codes, round to nearest even with saturation to +-448: `lo` goes to the low
+// byte.
+__device__ __forceinline__ uint16_t e4m3x2_rn_satfinite(float lo, float hi) {
+  uint16_t r;
+  asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;" : "=h"(r) : "f"(hi), "f"(lo));
+  return r;
+}
+
 // Round two f32 to bf16 (nearest even) and pack: `lo` goes to the low 16 bits.
 __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
   uint32_t r;
@@ -371,6 +379,16 @@ __device__ __forceinline__ void mma_pair_ts(uint32_t d_tmem, uint32_t a_tmem, ui
 // same thread read the copied values (tcgen05.cp -> tcgen05.mma is ordered by the hardware).
 __device__ __forceinline__ void tmem_cp_pair_64x128_dup(uint32_t t_addr, uint64_t s_desc) {
   asm volatile("tcgen05.cp.cta_group::2.64x128b.warpx2::02_13 [%0], %1;" :: "r"(t_addr), "l"(s_desc) : "memory");
+}
+
+// The same for 8-bit operands (kind::f8f6f4: A and B e4m3 here, K = 32 per instruction).
+__device__ __forceinline__ void mma_pair_ss_f8(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc, uint32_t idesc,
+                                               uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::2.kind::f8f6f4 [%0], %1, %2, %3, p;\n\t}"
+      :: "r"(d_tmem), "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate) : "memory");
 }
 
 // Arrive once on the barrier at `mbar`'s offset in every CTA of `cta_mask` when all pair MMAs
@@ -465,6 +483,17 @@ __host__ __device__ constexpr uint32_t idesc_bf16_f32(uint32_t M, uint32_t N, bo
   return (1u << 4)                       // D format: f32
        | (1u << 7)                       // A format: bf16
        | (1u << 10)                      // B format: bf16
+       | ((a_mn_major ? 1u : 0u) << 15)
+       | ((b_mn_major ? 1u : 0u) << 16)
+       | ((N >> 3) << 17)
+       | ((M >> 4) << 24);
+}
+
+// Instruction descriptor for kind::f8f6f4 with e4m3 A and B and fp32 D.
+__host__ __device__ constexpr uint32_t idesc_e4m3_f32(uint32_t M, uint32_t N, bool a_mn_major, bool b_mn_major) {
+  return (1u << 4)                       // D format: f32
+       | (0u << 7)                       // A format: e4m3
+       | (0u << 10)                      // B format: e4m3
        | ((a_mn_major ? 1u : 0u) << 15)
        | ((b_mn_major ? 1u : 0u) << 16)
        | ((N >> 3) << 17)

@@ -61,9 +61,10 @@ def test_split_error_bound_from_the_format():
 
 def test_sigma_is_the_largest_power_that_fits():
     rng = np.random.default_rng(7)
-    for s_max in np.concatenate([2.0 ** rng.uniform(-30, 10, 500), [1.75, 0.875, 1.0, 448.0]]):
+    for s_max in np.concatenate([2.0 ** rng.uniform(-30, 10, 500), [112.0, 56.0, 1.75, 0.875, 1.0, 448.0]]):
         sg = O.fp8_pv_sigma(s_max)
-        assert s_max * 2.0 ** sg <= 1.75 < s_max * 2.0 ** (sg + 1)
+        assert s_max * 2.0 ** sg <= 112.0 < s_max * 2.0 ** (sg + 1)
+        assert 4.0 * s_max * 2.0 ** sg <= O.E4M3_MAX
 
 
 def _row(n, rng, pow2_scales=False):
