@@ -152,6 +152,9 @@ mla_status_t mla_decode_paged_fp8_scale_folded(
  *     out[b,i,h,:] = 2^-sigma * sum_t (hi_t + lo_t) e4m3(code_t)[0:512] / sum_t p_t.
  * hi_t + lo_t equals w_t to within 2^-8 of w_t in the normal e4m3 range (2^-10 absolute below it),
  * so out is attention over the unrounded values s_t * e4m3(code_t) up to that error per weight.
+ * The kernel takes the residual in f16, lo_t = e4m3_rn_sat(f16_rn(w_t) - hi_t), which moves lo_t by
+ * one step at most where the f16 rounding of w_t (2^-12 of it) crosses one of lo_t's rounding
+ * boundaries; the bound above then grows by 2^-12 of w_t.
  * The largest weight lies in (56, 112], so the weights use the top of the e4m3 range.  The kernel
  * takes m and sigma per split of the keys (a running maximum of the scores that may trail the true
  * one by up to 2 in log2 units, so p_t <= 4 and w_t <= 448, and a running minimum of sigma over

@@ -824,13 +824,17 @@ __device__ __forceinline__ int fp8_pv_sigma(float s_max) {
 __device__ __forceinline__ float exp2i(int k) { return __int_as_float((k + 127) << 23); }   // 2^k, |k| <= 126
 __device__ __forceinline__ float exp2i_or_zero(int k) { return k < -126 ? 0.f : exp2i(k); }   // 2^k, k <= 126
 
-// Two-term e4m3 split of two weights w0, w1 >= 0: hi = e4m3_rn_sat(w), lo = e4m3_rn_sat(w - hi); the
-// residual is exact in f32 (hi is w rounded to 4 significant bits, or 0).  w0's codes in the low bytes.
+// Two-term e4m3 split of two weights w0, w1 >= 0: hi = e4m3_rn_sat(w) from the f32 weight; the
+// residual is taken in f16, lo = e4m3_rn_sat(f16_rn(w) - hi): hi is exact in f16 and the difference
+// of the two f16 values is exact (they are within a few percent of each other, or hi = 0), so lo
+// differs from e4m3_rn_sat(w - hi) only where the f16 rounding of w (2^-12 of w) moves the residual
+// across a rounding boundary of lo; hi + lo stays within 2^-8 + 2^-12 of w in the normal range.
+// Five instructions per pair (f32 residuals would take three more conversions).  w0's codes in the
+// low bytes.
 __device__ __forceinline__ void split2_e4m3(float w0, float w1, uint32_t& hi, uint32_t& lo) {
   const uint16_t h = ptx::e4m3x2_rn_satfinite(w0, w1);
-  const uint32_t hf = ptx::e4m3x2_to_f16x2(h);
   hi = h;
-  lo = ptx::e4m3x2_rn_satfinite(w0 - ptx::f16_lo_to_f32(hf), w1 - ptx::f16_hi_to_f32(hf));
+  lo = ptx::e4m3x2_rn_satfinite_f16x2(ptx::sub_f16x2(ptx::pack_f16x2(w0, w1), ptx::e4m3x2_to_f16x2(h)));
 }
 
 // 16-byte unit (0..7) of a P row that holds a softmax thread's chunk j (0..3) of its key half hh:
@@ -878,7 +882,9 @@ __device__ __forceinline__ void converter_role_fp8pv(const DecodeParams& p, int 
   uint32_t g = 0;
   while (true) {
     const uint32_t st = g & 1;
+    if (t == 0) MLA_TRACE_EV(g, 1);
     MLA_WAIT_RET(BAR(B_RING_FULL + st), (g >> 1) & 1);
+    if (t == 0) MLA_TRACE_EV(g, 3);
     const uint32_t stage = base + SRING + st * RING_STAGE;
     const uint32_t mask = ptx::ld_shared_u32(base + S_MASK + 8 * st);
     const uint32_t omask = ptx::ld_shared_u32(base + S_MASK + 8 * st + 4);
@@ -911,12 +917,18 @@ __device__ __forceinline__ void converter_role_fp8pv(const DecodeParams& p, int 
     }
     // K half buffer g % 2: free once Q.K^T(g - 2) has finished
     MLA_POLL_RET(BAR(B_S_FULL + st), ((g >> 1) & 1) ^ 1);
+    if (t == 0) MLA_TRACE_EV(g, 16);
     convert_k<false, false>(grp, r, cq, own_ok, raw, s_own, no_blk, base + SK0 + st * SK_STRIDE);
     ptx::fence_proxy_async_smem();
     __syncwarp();
     if (lane == 0) ptx::mbar_arrive_cluster(k_full0 + 8u * st);
+    if (t == 0) MLA_TRACE_EV(g, 5);
+    if (t == 352) MLA_TRACE_EV(g, 26);
+    if (lane == 0) MLA_TRACE_EV(g, 32 + (t >> 5));
     // FP8 V buffer g % 2: free once P.V(g - 2) has finished
+    if (t == 0) MLA_TRACE_EV(g, 4);
     MLA_WAIT_RET(BAR(B_PV_DONE + st), ((g >> 1) & 1) ^ 1);
+    if (t == 0) MLA_TRACE_EV(g, 6);
     {
       const uint32_t sv8 = base + SV + st * SV8_STRIDE;
 #pragma unroll
@@ -940,9 +952,13 @@ __device__ __forceinline__ void converter_role_fp8pv(const DecodeParams& p, int 
     ptx::fence_proxy_async_smem();
     __syncwarp();
     if (lane == 0) ptx::mbar_arrive_cluster(v_full0 + 8u * st);
-    ++g;
+    if (t == 0) MLA_TRACE_EV(g, 2);
+    if (t == 352) MLA_TRACE_EV(g, 27);
+    if (lane == 0) MLA_TRACE_EV(g, 44 + (t >> 5));
     if (!nt.valid) break;
     if (!fetch_oth<false>(p, L, C, grp, cq, extra, A)) raise_status(p.status, STATUS_BOUNDS);
+    if (t == 0) MLA_TRACE_EV(g, 7);
+    ++g;
     kt = nt;
     nt = ts.take(p);
     if (nt.valid) L = oth_lut_issue(p, nt, C, r);
@@ -1093,10 +1109,22 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) mla_decode_kernel(const __grid
         if (t == 0) MLA_TRACE_EV(g, 9);
         const int nv = min(BN, u.nvis - j * BN) - HALF_BN * hh;   // valid keys in this lane's half
         float mt = -INFINITY;
-        // scale-folding mode: the scales of this lane's 32 keys (written before K_FULL of this
-        // tile; slot g % 8 is rewritten only after this warp has finished tile g)
+        // scale-folding and e4m3 P.V modes: the scales of this lane's 32 keys (written before
+        // SC_FULL of this tile; slot g % 8 is rewritten only after this warp has finished tile g)
         const uint32_t sc_addr = base + SSC + (g % SSC_SLOTS) * SSC_STRIDE + 4 * HALF_BN * hh;
-        if (FOLD) {
+        // Scores in log2 units are x = S * c (c = scale_log2, times s_t in the scale-folding mode),
+        // keys past the request's end at -inf.  The e4m3 P.V mode, whose softmax carries the weight
+        // split, saves instructions on whole half-tiles with c > 0 (every tile but a request's
+        // last): it keeps x = S, takes the row max as max(S) * c (rounding is monotone) and forms
+        // each exponent as one fma(S, c, -m).  (In the other modes the same change costs register
+        // spills at this kernel's 96-register limit and measured slower.)
+        const float c = p.scale_log2;
+        const bool fast = F8 && nv >= HALF_BN && c > 0.f;   // warp-uniform
+        if (fast) {
+#pragma unroll
+          for (int q = 0; q < 32; ++q) mt = fmaxf(mt, x[q]);
+          mt *= c;
+        } else if (FOLD) {
 #pragma unroll
           for (int v = 0; v < 8; ++v) {
             const uint4 s4 = ptx::ld_shared_v4(sc_addr + 16 * v);
@@ -1105,14 +1133,14 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) mla_decode_kernel(const __grid
 #pragma unroll
             for (int e = 0; e < 4; ++e) {
               const int q = 4 * v + e;
-              x[q] = (q < nv) ? x[q] * (p.scale_log2 * sc[e]) : -INFINITY;
+              x[q] = (q < nv) ? x[q] * (c * sc[e]) : -INFINITY;
               mt = fmaxf(mt, x[q]);
             }
           }
         } else {
 #pragma unroll
           for (int q = 0; q < 32; ++q) {
-            x[q] = (q < nv) ? x[q] * p.scale_log2 : -INFINITY;
+            x[q] = (q < nv) ? x[q] * c : -INFINITY;
             mt = fmaxf(mt, x[q]);
           }
         }
@@ -1148,25 +1176,28 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) mla_decode_kernel(const __grid
         }
         float lsum = 0.f;
         uint32_t pw[16];
+        const float cmul = fast ? c : 1.f;
         if (F8) {
-          // l sums the weights p; P carries w = p * s_t * 2^sig as two e4m3 terms (p <= 4 under the
-          // lazy max, s_t * 2^sig <= 112, so w <= 448)
-          const float sf = exp2i(sig);
+          // P carries w = p * s_t * 2^sig as two e4m3 terms (p <= 4 under the lazy max, s_t * 2^sig
+          // <= 112, so w <= 448).  The exponent takes 2^sig in (p' = 2^(x - m + sig)); l sums p'
+          // and is scaled back by 2^-sig once per tile.
+          const float mo = m_ref - static_cast<float>(sig);
 #pragma unroll
           for (int v = 0; v < 8; ++v) {
             const uint4 s4 = ptx::ld_shared_v4(sc_addr + 16 * v);
-            const float p0 = ptx::ex2_approx(x[4 * v] - m_ref);
-            const float p1 = ptx::ex2_approx(x[4 * v + 1] - m_ref);
-            const float p2 = ptx::ex2_approx(x[4 * v + 2] - m_ref);
-            const float p3 = ptx::ex2_approx(x[4 * v + 3] - m_ref);
+            const float p0 = ptx::ex2_approx(fmaf(x[4 * v], cmul, -mo));
+            const float p1 = ptx::ex2_approx(fmaf(x[4 * v + 1], cmul, -mo));
+            const float p2 = ptx::ex2_approx(fmaf(x[4 * v + 2], cmul, -mo));
+            const float p3 = ptx::ex2_approx(fmaf(x[4 * v + 3], cmul, -mo));
             lsum += p0 + p1;
             lsum += p2 + p3;
             uint32_t h01, l01, h23, l23;
-            split2_e4m3(p0 * (__uint_as_float(s4.x) * sf), p1 * (__uint_as_float(s4.y) * sf), h01, l01);
-            split2_e4m3(p2 * (__uint_as_float(s4.z) * sf), p3 * (__uint_as_float(s4.w) * sf), h23, l23);
+            split2_e4m3(p0 * __uint_as_float(s4.x), p1 * __uint_as_float(s4.y), h01, l01);
+            split2_e4m3(p2 * __uint_as_float(s4.z), p3 * __uint_as_float(s4.w), h23, l23);
             pw[v] = h01 | (h23 << 16);
             pw[8 + v] = l01 | (l23 << 16);
           }
+          lsum *= exp2i(-sig);
         } else if (FOLD) {
           // l sums the weights; the P operand carries weight * s_t
 #pragma unroll

@@ -295,6 +295,28 @@ __device__ __forceinline__ uint16_t e4m3x2_rn_satfinite(float lo, float hi) {
   return r;
 }
 
+// Two f16 (packed, low half = first element) to two e4m3 codes, nearest even, saturating: the low
+// half's code goes to the low byte.
+__device__ __forceinline__ uint16_t e4m3x2_rn_satfinite_f16x2(uint32_t h2) {
+  uint16_t r;
+  asm("cvt.rn.satfinite.e4m3x2.f16x2 %0, %1;" : "=h"(r) : "r"(h2));
+  return r;
+}
+
+// Round two f32 to f16 (nearest even) and pack: `lo` goes to the low 16 bits.
+__device__ __forceinline__ uint32_t pack_f16x2(float lo, float hi) {
+  uint32_t r;
+  asm("cvt.rn.f16x2.f32 %0, %1, %2;" : "=r"(r) : "f"(hi), "f"(lo));
+  return r;
+}
+
+// Packed f16 difference a - b (nearest even), element by element.
+__device__ __forceinline__ uint32_t sub_f16x2(uint32_t a, uint32_t b) {
+  uint32_t r;
+  asm("sub.rn.f16x2 %0, %1, %2;" : "=r"(r) : "r"(a), "r"(b));
+  return r;
+}
+
 // Round two f32 to bf16 (nearest even) and pack: `lo` goes to the low 16 bits.
 __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
   uint32_t r;
