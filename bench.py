@@ -50,6 +50,8 @@ def parse():
                     help="decode (the default contract line) or the KV-store step that fills the cache")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--e2e-chunks", type=int, default=0,
+                    help="request groups of the host-buffer call in the e2e measurement (0 = automatic)")
     ap.add_argument("--cpu-seconds", type=float, default=12.0, help="budget of the oracle CPU baseline")
     return ap.parse_args()
 
@@ -435,22 +437,16 @@ def main():
         hslut = None if inp.scales_lookup_table is None else inp.scales_lookup_table.cpu().pin_memory()
         hout = torch.empty(out.shape, dtype=out.dtype, pin_memory=True)
         hlse = torch.empty(lse.shape, dtype=lse.dtype, pin_memory=True)
-        dq, dl, dlut = torch.empty_like(inp.q), torch.empty_like(inp.cache_lengths), torch.empty_like(inp.lookup_table)
-        dslut = None if hslut is None else torch.empty_like(inp.scales_lookup_table)
         h2d = hq.numel() * hq.element_size() + hl.numel() * 4 + hlut.numel() * 4 + (0 if hslut is None else hslut.numel() * 4)
         d2h = hout.numel() * 2 + hlse.numel() * 4
         Ke = min(K, 100)
+        variant = M.VARIANT_SCALE_FOLDED if fold else M.VARIANT_E4M3_PV if pv else M.VARIANT_DECODE
 
         def e2e_step():
-            dq.copy_(hq, non_blocking=True)
-            dl.copy_(hl, non_blocking=True)
-            dlut.copy_(hlut, non_blocking=True)
-            if dslut is not None:
-                dslut.copy_(hslut, non_blocking=True)
-            M.decode(dq, inp.blocks, inp.scales, dl, dlut, dslut, T, inp.max_cache_length, inp.layer_idx,
-                     inp.softmax_scale, out=out, lse=lse, stream=stream, fold_scales=fold, e4m3_pv=pv)
-            hout.copy_(out, non_blocking=True)
-            hlse.copy_(lse, non_blocking=True)
+            # one call of the host-buffer entry point: q, lengths and tables in from pinned host
+            # memory, out and lse back, the copies of one request group overlapping another's decode
+            M.decode_host(hq, inp.blocks, inp.scales, hl, hlut, hslut, T, inp.max_cache_length, inp.layer_idx,
+                          inp.softmax_scale, hout, hlse, variant=variant, num_chunks=args.e2e_chunks, stream=stream)
 
         for _ in range(3):
             e2e_step()
@@ -469,7 +465,9 @@ def main():
         if dist:
             e2e_ms = max_over_ranks(dist, [e2e_ms], "cuda")[0]
         e2e = {"value": kv_bytes_all / (e2e_ms * 1e-3) / 1e9, "unit": "GB/s", "h2d_bytes_per_step": h2d,
-               "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms}
+               "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms,
+               "api": "mla_decode_paged_fp8_host (pinned host q, lengths, tables in; out, lse back)",
+               "num_chunks": args.e2e_chunks if args.e2e_chunks > 0 else "auto"}
 
     if dist:
         step_ms, kern_ms = max_over_ranks(dist, [step_ms, kern_ms], "cuda")

@@ -174,6 +174,53 @@ mla_status_t mla_decode_paged_fp8_e4m3_pv(
     uint32_t max_prompt_length, uint32_t max_cache_length, uint32_t layer_idx, float softmax_scale,
     const mla_paged_shape_t* shape, void* out, float* lse, cudaStream_t stream);
 
+/* Which decode mla_decode_paged_fp8_host runs. */
+enum {
+  MLA_VARIANT_DECODE = 0,          /* mla_decode_paged_fp8 */
+  MLA_VARIANT_SCALE_FOLDED = 1,    /* mla_decode_paged_fp8_scale_folded */
+  MLA_VARIANT_E4M3_PV = 2          /* mla_decode_paged_fp8_e4m3_pv */
+};
+
+/*
+ * mla_decode_paged_fp8_host -- one decode step whose per-step inputs and outputs live in host
+ * memory: q, cache_lengths, lookup_table and scales_lookup_table are read from the host, out and
+ * lse are written to the host; the KV cache (blocks, scales) stays in device memory.  The pages'
+ * kernels take device tensors only; this entry point is the same decode with the host copies
+ * folded in.
+ *
+ * The batch is cut into num_chunks contiguous groups of requests (0 = automatic: 4 for batch >= 64,
+ * 2 for batch >= 16, else 1; at most 16).  Each group's inputs are copied to a device staging area
+ * on an internal stream, decoded on `stream` (by the variant's device entry point, on the group
+ * alone), and its out and lse copied back on a second internal stream, so the copies of one group
+ * overlap the decode of another.  Each group is its own decode call, so the split-KV partition,
+ * and with it the rounding of split rows, can differ from one call over the whole batch (within
+ * the decode's tolerance; with num_chunks = 1 the results are the device entry point's bit for
+ * bit).
+ *
+ * Arguments: as for mla_decode_paged_fp8, except that q_host [batch, max_prompt_length,
+ * num_q_heads, 576] bf16, cache_lengths_host [batch], lookup_table_host and scales_lookup_table_host
+ * [batch, max_pages] (the latter may be NULL) and out_host [..., 512] bf16, lse_host [batch,
+ * max_prompt_length, num_q_heads] fp32 (may be NULL) are host pointers, best page-locked
+ * (cudaHostAlloc / cudaHostRegister: pageable memory makes the copies synchronous), and
+ * variant is one of MLA_VARIANT_*.  The caller keeps ownership of every buffer.
+ *
+ * Asynchronous on `stream`: when the call returns, the copies and decodes are enqueued; out_host
+ * and lse_host are complete once `stream` has been synchronised (the call makes `stream` wait for
+ * its last copy), and the host inputs must stay unchanged until then.  Calls must be ordered on
+ * one stream per device (they share the staging area, the workspace and the internal streams).
+ * The staging area grows on demand (cudaMalloc, with a device synchronisation when it is
+ * replaced), so a call that grows it must not be inside stream capture.  Errors: the device entry
+ * points' (checked before anything is enqueued), MLA_ERR_INVALID_ARG for a NULL host pointer, an
+ * unknown variant or num_chunks outside [0, 16], MLA_ERR_WORKSPACE, MLA_ERR_CUDA.  If an error
+ * occurs after copies were enqueued, the call waits for them before returning.
+ */
+mla_status_t mla_decode_paged_fp8_host(
+    const void* q_host, const void* blocks, const float* scales,
+    const uint32_t* cache_lengths_host, const uint32_t* lookup_table_host, const uint32_t* scales_lookup_table_host,
+    uint32_t max_prompt_length, uint32_t max_cache_length, uint32_t layer_idx, float softmax_scale,
+    const mla_paged_shape_t* shape, void* out_host, float* lse_host, int32_t variant, int32_t num_chunks,
+    cudaStream_t stream);
+
 /*
  * mla_decode_paged_fp8_noalloc -- the same decode, for callers that cannot allocate device memory
  * (for instance while a CUDA graph is being captured, under an allocator that owns the whole

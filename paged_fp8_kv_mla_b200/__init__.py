@@ -8,4 +8,5 @@ parallelism (`context_parallel`).
 from ._lib import (  # noqa: F401
     MlaError, decode, decode_inputs, gather_dequant, kv_store, set_num_clusters, get_num_clusters, set_wait_limit_ns, withhold_arrival_once, device_status,
     release_workspace, version, set_timing_events, load, LIB_PATH, EXPORTED, merge_parts, decode_noalloc,
+    decode_host, VARIANT_DECODE, VARIANT_SCALE_FOLDED, VARIANT_E4M3_PV,
 )

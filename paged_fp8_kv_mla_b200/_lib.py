@@ -24,7 +24,10 @@ EXPORTED = ["mla_decode_paged_fp8", "mla_gather_dequant_bf16", "mla_set_num_clus
             "mla_get_num_clusters", "mla_last_error_string", "mla_get_device_status",
             "mla_release_workspace", "mla_version", "mla_set_timing_events", "mla_decode_paged_fp8_noalloc",
             "mla_kv_store_fp8", "mla_decode_paged_fp8_scale_folded", "mla_merge_lse_parts_bf16",
-            "mla_set_wait_limit_ns", "mla_debug_withhold_arrival_once", "mla_decode_paged_fp8_e4m3_pv"]
+            "mla_set_wait_limit_ns", "mla_debug_withhold_arrival_once", "mla_decode_paged_fp8_e4m3_pv",
+            "mla_decode_paged_fp8_host"]
+
+VARIANT_DECODE, VARIANT_SCALE_FOLDED, VARIANT_E4M3_PV = 0, 1, 2
 
 
 class MlaError(RuntimeError):
@@ -60,6 +63,9 @@ def load(path: str = LIB_PATH) -> ctypes.CDLL:
     lib.mla_decode_paged_fp8_scale_folded.restype = ctypes.c_int
     lib.mla_decode_paged_fp8_e4m3_pv.argtypes = lib.mla_decode_paged_fp8.argtypes
     lib.mla_decode_paged_fp8_e4m3_pv.restype = ctypes.c_int
+    lib.mla_decode_paged_fp8_host.argtypes = [vp, vp, vp, vp, vp, vp, u32, u32, u32, f32,
+                                              ctypes.POINTER(PagedShape), vp, vp, i32, i32, vp]
+    lib.mla_decode_paged_fp8_host.restype = ctypes.c_int
     lib.mla_decode_paged_fp8_noalloc.argtypes = [vp, vp, vp, vp, vp, vp, u32, u32, u32, f32,
                                                  ctypes.POINTER(PagedShape), vp, vp, vp]
     lib.mla_decode_paged_fp8_noalloc.restype = ctypes.c_int
@@ -201,6 +207,42 @@ def decode(q, blocks, scales, cache_lengths, lookup_table, scales_lookup_table, 
     st = fn(_ptr(q), _ptr(blocks), _ptr(scales), _ptr(cache_lengths), _ptr(lookup_table), _ptr(scales_lookup_table),
             int(max_prompt_length), int(max_cache_length), int(layer_idx), float(softmax_scale), ctypes.byref(shp),
             _ptr(out), _ptr(lse), _stream(stream))
+    _check(st)
+    return out, lse
+
+
+def decode_host(q, blocks, scales, cache_lengths, lookup_table, scales_lookup_table, max_prompt_length: int,
+                max_cache_length: int, layer_idx: int, softmax_scale: float, out, lse=None, variant: int = 0,
+                num_chunks: int = 0, stream=None):
+    """mla_decode_paged_fp8_host: q, cache_lengths, the page tables, out and lse are CPU tensors (best
+    pinned), blocks and scales CUDA tensors on the current device.  Asynchronous on `stream`: out and
+    lse are complete after that stream is synchronised.  variant: VARIANT_DECODE, VARIANT_SCALE_FOLDED
+    or VARIANT_E4M3_PV; num_chunks 0 = automatic."""
+    _expect("q", q, (torch.bfloat16,), ndim=4, last=576)
+    B, T, H, _ = q.shape
+    _expect("blocks", blocks, _CODES, ndim=6)
+    _expect("scales", scales, (torch.float32,), ndim=6)
+    _expect("cache_lengths", cache_lengths, _U32, ndim=1)
+    _expect("lookup_table", lookup_table, _U32, ndim=2)
+    _expect("scales_lookup_table", scales_lookup_table, _U32, ndim=2, optional=True)
+    _expect("out", out, (torch.bfloat16,), ndim=4, last=512)
+    _expect("lse", lse, (torch.float32,), ndim=3, optional=True)
+    if cache_lengths.shape[0] != B or lookup_table.shape[0] != B:
+        raise ValueError(f"cache_lengths and lookup_table must have {B} rows (one per request)")
+    if scales_lookup_table is not None and tuple(scales_lookup_table.shape) != tuple(lookup_table.shape):
+        raise ValueError("scales_lookup_table must have the shape of lookup_table")
+    if tuple(out.shape) != (B, T, H, 512) or (lse is not None and tuple(lse.shape) != (B, T, H)):
+        raise ValueError("out / lse shapes do not match q")
+    host = [t for t in (q, cache_lengths, lookup_table, scales_lookup_table, out, lse) if t is not None]
+    if any(t.device.type != "cpu" for t in host):
+        raise ValueError("q, cache_lengths, the page tables, out and lse must be CPU tensors")
+    _same_device(blocks, scales)
+    lib = load()
+    shp = paged_shape(B, H, blocks, scales, lookup_table)
+    st = lib.mla_decode_paged_fp8_host(_ptr(q), _ptr(blocks), _ptr(scales), _ptr(cache_lengths), _ptr(lookup_table),
+                                       _ptr(scales_lookup_table), int(max_prompt_length), int(max_cache_length),
+                                       int(layer_idx), float(softmax_scale), ctypes.byref(shp), _ptr(out), _ptr(lse),
+                                       int(variant), int(num_chunks), _stream(stream))
     _check(st)
     return out, lse
 

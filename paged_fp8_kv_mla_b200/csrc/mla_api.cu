@@ -503,6 +503,167 @@ mla_status_t mla_decode_paged_fp8_e4m3_pv(const void* q, const void* blocks, con
                       max_cache_length, layer_idx, softmax_scale, shape, out, lse, stream, mla::SCALE_FP8PV);
 }
 
+}  // extern "C"
+
+namespace {
+// ---------------------------------------------------------------- decode from host buffers
+// Per device: a staging area in device memory for the call's inputs and outputs, two streams for
+// the copies (host -> device, device -> host) and an event per chunk and direction.
+constexpr int kMaxHostChunks = 16;
+struct HostPipe {
+  void* staging = nullptr;
+  size_t bytes = 0;
+  cudaStream_t s_in = nullptr, s_out = nullptr;
+  cudaEvent_t ev_start = nullptr, ev_end = nullptr;
+  cudaEvent_t ev_in[kMaxHostChunks] = {}, ev_dec[kMaxHostChunks] = {};
+};
+std::mutex g_hp_mu;
+HostPipe g_hp[kMaxDevices];
+
+mla_status_t host_pipe(int dev, size_t bytes, HostPipe** out) {
+  HostPipe& h = g_hp[dev];
+  if (!h.s_in) {
+    MLA_CUDA(cudaStreamCreateWithFlags(&h.s_in, cudaStreamNonBlocking));
+    MLA_CUDA(cudaStreamCreateWithFlags(&h.s_out, cudaStreamNonBlocking));
+    MLA_CUDA(cudaEventCreateWithFlags(&h.ev_start, cudaEventDisableTiming));
+    MLA_CUDA(cudaEventCreateWithFlags(&h.ev_end, cudaEventDisableTiming));
+    for (int i = 0; i < kMaxHostChunks; ++i) {
+      MLA_CUDA(cudaEventCreateWithFlags(&h.ev_in[i], cudaEventDisableTiming));
+      MLA_CUDA(cudaEventCreateWithFlags(&h.ev_dec[i], cudaEventDisableTiming));
+    }
+  }
+  if (h.bytes < bytes) {
+    if (h.staging) {
+      MLA_CUDA(cudaDeviceSynchronize());
+      MLA_CUDA(cudaFree(h.staging));
+      h.staging = nullptr;
+      h.bytes = 0;
+    }
+    const size_t want = align_up(bytes + bytes / 8, 1 << 20);
+    cudaError_t e = cudaMalloc(&h.staging, want);
+    if (e != cudaSuccess) {
+      h.staging = nullptr;
+      return fail(MLA_ERR_WORKSPACE, "host-call staging cudaMalloc(%zu) failed: %s", want, cudaGetErrorString(e));
+    }
+    h.bytes = want;
+  }
+  *out = &h;
+  return MLA_OK;
+}
+
+// Copies of a host range to device (or back) as one cudaMemcpyAsync each.
+mla_status_t copy_async(void* dst, const void* src, size_t n, cudaMemcpyKind kind, cudaStream_t s) {
+  if (n) MLA_CUDA(cudaMemcpyAsync(dst, src, n, kind, s));
+  return MLA_OK;
+}
+}  // namespace
+
+extern "C" {
+
+mla_status_t mla_decode_paged_fp8_host(const void* q_host, const void* blocks, const float* scales,
+                                       const uint32_t* cache_lengths_host, const uint32_t* lookup_table_host,
+                                       const uint32_t* scales_lookup_table_host, uint32_t max_prompt_length,
+                                       uint32_t max_cache_length, uint32_t layer_idx, float softmax_scale,
+                                       const mla_paged_shape_t* shape, void* out_host, float* lse_host,
+                                       int32_t variant, int32_t num_chunks, cudaStream_t stream) {
+  if (!shape) return fail(MLA_ERR_INVALID_ARG, "shape is NULL");
+  if (!q_host || !cache_lengths_host || !lookup_table_host || !out_host)
+    return fail(MLA_ERR_INVALID_ARG, "q_host, cache_lengths_host, lookup_table_host and out_host must be non-NULL");
+  if (variant < MLA_VARIANT_DECODE || variant > MLA_VARIANT_E4M3_PV)
+    return fail(MLA_ERR_INVALID_ARG, "variant %d is not one of MLA_VARIANT_*", variant);
+  if (num_chunks < 0 || num_chunks > kMaxHostChunks)
+    return fail(MLA_ERR_INVALID_ARG, "num_chunks %d outside [0, %d]", num_chunks, kMaxHostChunks);
+  // the same checks as the device entry points, before anything is enqueued (stand-in device
+  // pointers for the staged tables: only their presence is checked here)
+  {
+    mla::DecodeParams p{};
+    uint64_t rows = 0;
+    const mla_status_t st = check_cache(blocks, scales, cache_lengths_host, lookup_table_host, max_prompt_length,
+                                        max_cache_length, layer_idx, shape, &p, &rows);
+    if (st != MLA_OK) return st;
+    if (variant != MLA_VARIANT_DECODE && p.SG != 1)
+      return fail(MLA_ERR_UNSUPPORTED, "the scale-folding and e4m3 P.V decodes take one scale per token");
+    if (!(softmax_scale == softmax_scale)) return fail(MLA_ERR_INVALID_ARG, "softmax_scale is NaN");
+  }
+  const int B = shape->batch;
+  if (B == 0) return MLA_OK;
+  const size_t T = max_prompt_length, H = static_cast<size_t>(shape->num_q_heads);
+  const size_t MP = static_cast<size_t>(shape->max_pages);
+  const size_t q_row = T * H * mla::HEAD_DIM * 2, o_row = T * H * mla::V_DIM * 2, l_row = T * H * 4;
+  const size_t t_row = MP * 4;
+  size_t o = 0;
+  const size_t off_q = o;    o = align_up(o + q_row * B, 256);
+  const size_t off_len = o;  o = align_up(o + 4 * static_cast<size_t>(B), 256);
+  const size_t off_lut = o;  o = align_up(o + t_row * B, 256);
+  const size_t off_slut = o; o = align_up(o + (scales_lookup_table_host ? t_row * B : 0), 256);
+  const size_t off_out = o;  o = align_up(o + o_row * B, 256);
+  const size_t off_lse = o;  o = align_up(o + l_row * B, 256);
+
+  int dev = 0;
+  MLA_CUDA(cudaGetDevice(&dev));
+  if (dev >= kMaxDevices) return fail(MLA_ERR_UNSUPPORTED, "device index too large");
+  std::lock_guard<std::mutex> lk(g_hp_mu);
+  HostPipe* h = nullptr;
+  mla_status_t st = host_pipe(dev, o, &h);
+  if (st != MLA_OK) return st;
+  char* d = static_cast<char*>(h->staging);
+  const int nch = num_chunks > 0 ? (num_chunks < B ? num_chunks : B) : (B >= 64 ? 4 : B >= 16 ? 2 : 1);
+  const int mode = variant == MLA_VARIANT_SCALE_FOLDED ? mla::SCALE_FOLD
+                 : variant == MLA_VARIANT_E4M3_PV ? mla::SCALE_FP8PV : mla::SCALE_TOKEN;
+
+  // Chunk i: host -> device copies on s_in, its decode on `stream`, device -> host copies on
+  // s_out; copies of one chunk overlap the decode of another.  The staging area is reused by the
+  // next call, whose first copy waits for everything this call enqueued on `stream` (ev_start).
+  MLA_CUDA(cudaEventRecord(h->ev_start, stream));
+  MLA_CUDA(cudaStreamWaitEvent(h->s_in, h->ev_start, 0));
+  MLA_CUDA(cudaStreamWaitEvent(h->s_out, h->ev_start, 0));
+  mla_paged_shape_t cs = *shape;
+  for (int i = 0; i < nch && st == MLA_OK; ++i) {
+    const size_t b0 = static_cast<size_t>(B) * i / nch, b1 = static_cast<size_t>(B) * (i + 1) / nch, nb = b1 - b0;
+    const char* hq = static_cast<const char*>(q_host);
+    if ((st = copy_async(d + off_q + q_row * b0, hq + q_row * b0, q_row * nb, cudaMemcpyHostToDevice, h->s_in)) ||
+        (st = copy_async(d + off_len + 4 * b0, cache_lengths_host + b0, 4 * nb, cudaMemcpyHostToDevice, h->s_in)) ||
+        (st = copy_async(d + off_lut + t_row * b0, lookup_table_host + MP * b0, t_row * nb, cudaMemcpyHostToDevice,
+                         h->s_in)))
+      break;
+    if (scales_lookup_table_host &&
+        (st = copy_async(d + off_slut + t_row * b0, scales_lookup_table_host + MP * b0, t_row * nb,
+                         cudaMemcpyHostToDevice, h->s_in)))
+      break;
+    if (cudaEventRecord(h->ev_in[i], h->s_in) != cudaSuccess || cudaStreamWaitEvent(stream, h->ev_in[i], 0) != cudaSuccess) {
+      st = fail(MLA_ERR_CUDA, "event record / wait failed");
+      break;
+    }
+    cs.batch = static_cast<int32_t>(nb);
+    st = decode_alloc(d + off_q + q_row * b0, blocks, scales, reinterpret_cast<const uint32_t*>(d + off_len) + b0,
+                      reinterpret_cast<const uint32_t*>(d + off_lut) + MP * b0,
+                      scales_lookup_table_host ? reinterpret_cast<const uint32_t*>(d + off_slut) + MP * b0 : nullptr,
+                      max_prompt_length, max_cache_length, layer_idx, softmax_scale, &cs, d + off_out + o_row * b0,
+                      lse_host ? reinterpret_cast<float*>(d + off_lse + l_row * b0) : nullptr, stream, mode);
+    if (st != MLA_OK) break;
+    if (cudaEventRecord(h->ev_dec[i], stream) != cudaSuccess || cudaStreamWaitEvent(h->s_out, h->ev_dec[i], 0) != cudaSuccess) {
+      st = fail(MLA_ERR_CUDA, "event record / wait failed");
+      break;
+    }
+    if ((st = copy_async(static_cast<char*>(out_host) + o_row * b0, d + off_out + o_row * b0, o_row * nb,
+                         cudaMemcpyDeviceToHost, h->s_out)))
+      break;
+    if (lse_host && (st = copy_async(reinterpret_cast<char*>(lse_host) + l_row * b0, d + off_lse + l_row * b0,
+                                     l_row * nb, cudaMemcpyDeviceToHost, h->s_out)))
+      break;
+  }
+  if (st != MLA_OK) {
+    // nothing enqueued by this call may still touch the caller's host buffers when it returns
+    cudaStreamSynchronize(h->s_in);
+    cudaStreamSynchronize(stream);
+    cudaStreamSynchronize(h->s_out);
+    return st;
+  }
+  MLA_CUDA(cudaEventRecord(h->ev_end, h->s_out));
+  MLA_CUDA(cudaStreamWaitEvent(stream, h->ev_end, 0));
+  return MLA_OK;
+}
+
 mla_status_t mla_gather_dequant_bf16(const void* blocks, const float* scales, const uint32_t* cache_lengths,
                                      const uint32_t* lookup_table, const uint32_t* scales_lookup_table,
                                      uint32_t max_prompt_length, uint32_t max_cache_length, uint32_t layer_idx,

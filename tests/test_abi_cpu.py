@@ -162,3 +162,29 @@ def test_wait_limit_range(lib):
     assert lib.mla_set_wait_limit_ns(60_000_000_001) == 1
     assert lib.mla_set_wait_limit_ns(1_000_000) == 0
     assert lib.mla_set_wait_limit_ns(2_000_000_000) == 0
+
+
+def test_host_buffer_entry_validation(lib):
+    """mla_decode_paged_fp8_host checks everything on the host before any CUDA call: NULL host
+    pointers, an unknown variant, a chunk count outside [0, 16], the shared shape checks, and the
+    one-scale-per-token rule of its two variants; batch = 0 is a no-op."""
+    def host(shape, variant=0, chunks=0, **kw):
+        a = dict(q=FAKE, blocks=FAKE, scales=FAKE, lens=FAKE, lut=FAKE, out=FAKE, T=1, maxc=64, layer=0)
+        a.update(kw)
+        return lib.mla_decode_paged_fp8_host(a["q"], a["blocks"], a["scales"], a["lens"], a["lut"], None, a["T"],
+                                             a["maxc"], a["layer"], 0.07,
+                                             ctypes.byref(shape) if shape is not None else None, a["out"], None,
+                                             variant, chunks, None)
+    assert host(None) == 1
+    assert host(_shape(), q=None) == 1
+    assert host(_shape(), out=None) == 1
+    assert host(_shape(), variant=3) == 1
+    assert host(_shape(), variant=-1) == 1
+    assert host(_shape(), chunks=17) == 1
+    assert host(_shape(), chunks=-1) == 1
+    assert host(_shape(), layer=1) == 1
+    assert host(_shape(head_dim=512)) == 2
+    assert host(_shape(head_dim_granularity=9), variant=2) == 2
+    assert "one scale per token" in lib.mla_last_error_string().decode()
+    assert host(_shape(batch=0)) == 0
+    assert host(_shape(batch=0), variant=2, chunks=16) == 0
