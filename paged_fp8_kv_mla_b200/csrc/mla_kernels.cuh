@@ -547,29 +547,44 @@ __device__ __forceinline__ uint32_t run_mask(const Runs& R) {
 // runs start at multiples of 16 slots and pages hold a multiple of 16).
 __device__ __forceinline__ uint32_t scale_bytes(int len) { return ((static_cast<uint32_t>(len) + 3u) & ~3u) * 4u; }
 
-// Fills one ring stage for tile j of request b (visible keys nvis): the CTA's own 32 keys' rows
-// (rows [0, 32) of the stage) and, with per-token scales (SC), their scales at RING_ROWS; with
-// OTHER also the other CTA's 32 keys' scales at RING_OSC.  Writes the masks of copied rows and
-// copied other-key scales to mask_addr and mask_addr + 4, then arrives on `full` with the byte
-// count and issues the bulk copies.
-template <bool SC, bool OTHER>
-__device__ __forceinline__ void issue_stage(const DecodeParams& p, uint32_t stage, uint32_t full, uint32_t mask_addr,
-                                            int b, int j, int nvis, int c) {
-  bool bad = false;
+// Page runs of one ring stage for tile j of request b (visible keys nvis): the CTA's own 32 keys
+// and, with OTHER, the other CTA's 32 keys (whose scales only are copied).  Reads the page table;
+// the producer plans a tile while the stage before it is still being read, so that the table's
+// latency does not delay the copies.
+struct StagePlan {
+  Runs own, oth;
+  bool bad;
+};
+
+template <bool OTHER>
+__device__ __forceinline__ StagePlan plan_stage(const DecodeParams& p, int b, int j, int nvis, int c) {
+  StagePlan sp;
+  sp.bad = false;
   const int tok0 = j * BN + HALF_BN * c;
-  const Runs own = half_runs(p, b, tok0, max(0, min(HALF_BN, nvis - tok0)), bad);
-  Runs oth;
-  oth.ok0 = oth.ok1 = false;
-  oth.len0 = oth.len1 = 0;
-  oth.v0 = oth.s0 = oth.v1 = oth.s1 = 0;
+  sp.own = half_runs(p, b, tok0, max(0, min(HALF_BN, nvis - tok0)), sp.bad);
+  sp.oth.ok0 = sp.oth.ok1 = false;
+  sp.oth.len0 = sp.oth.len1 = 0;
+  sp.oth.v0 = sp.oth.s0 = sp.oth.v1 = sp.oth.s1 = 0;
   const int tok1 = j * BN + HALF_BN * (1 - c);
-  if (OTHER) oth = half_runs(p, b, tok1, max(0, min(HALF_BN, nvis - tok1)), bad);
+  if (OTHER) sp.oth = half_runs(p, b, tok1, max(0, min(HALF_BN, nvis - tok1)), sp.bad);
+  return sp;
+}
+
+// Fills one ring stage from its plan: the own keys' rows (rows [0, 32) of the stage) and, with
+// per-token scales (SC), their scales at RING_ROWS; with OTHER also the other keys' scales at
+// RING_OSC.  Writes the masks of copied rows and copied other-key scales to mask_addr and
+// mask_addr + 4, then arrives on `full` with the byte count and issues the bulk copies.
+template <bool SC, bool OTHER>
+__device__ __forceinline__ void issue_planned(const DecodeParams& p, uint32_t stage, uint32_t full, uint32_t mask_addr,
+                                              const StagePlan& sp) {
+  const Runs& own = sp.own;
+  const Runs& oth = sp.oth;
   uint32_t tx = 0;
   if (own.ok0) tx += static_cast<uint32_t>(own.len0) * HEAD_DIM + (SC ? scale_bytes(own.len0) : 0u);
   if (own.ok1) tx += static_cast<uint32_t>(own.len1) * HEAD_DIM + (SC ? scale_bytes(own.len1) : 0u);
   if (OTHER && oth.ok0) tx += scale_bytes(oth.len0);
   if (OTHER && oth.ok1) tx += scale_bytes(oth.len1);
-  if (bad) raise_status(p.status, STATUS_BOUNDS);
+  if (sp.bad) raise_status(p.status, STATUS_BOUNDS);
   ptx::st_shared_u32(mask_addr, run_mask(own));
   ptx::st_shared_u32(mask_addr + 4, OTHER ? run_mask(oth) : 0u);
   ptx::mbar_arrive_expect_tx(full, tx);
@@ -586,6 +601,12 @@ __device__ __forceinline__ void issue_stage(const DecodeParams& p, uint32_t stag
   if (OTHER && oth.ok0) ptx::bulk_load(stage + RING_OSC, p.scales + oth.s0, scale_bytes(oth.len0), full);
   if (OTHER && oth.ok1)
     ptx::bulk_load(stage + RING_OSC + 4u * static_cast<uint32_t>(oth.len0), p.scales + oth.s1, scale_bytes(oth.len1), full);
+}
+
+template <bool SC, bool OTHER>
+__device__ __forceinline__ void issue_stage(const DecodeParams& p, uint32_t stage, uint32_t full, uint32_t mask_addr,
+                                            int b, int j, int nvis, int c) {
+  issue_planned<SC, OTHER>(p, stage, full, mask_addr, plan_stage<OTHER>(p, b, j, nvis, c));
 }
 
 // Page-table entries of a converter thread's other-CTA key of one tile, read a step before the
@@ -970,7 +991,8 @@ __device__ __forceinline__ void converter_role_fp8pv(const DecodeParams& p, int 
 
 // =============================================================================================
 // producer role (lane 0 of warp 19): walks the cluster's tiles and fills ring stage g % 2 with the
-// own keys' rows (and per-token scales) of tile g once the converters have released the stage.
+// own keys' rows (and per-token scales) of tile g once the converters have released the stage;
+// tile g + 1's page runs are read from the page table before that wait.
 // Before returning it waits (bounded, whatever the other roles did) for the copies of the last
 // two stages it armed, so that no bulk copy into this CTA's shared memory is in flight at exit.
 // =============================================================================================
@@ -981,16 +1003,19 @@ __device__ __forceinline__ void producer_role(const DecodeParams& p, int k, uint
 #define BAR(i) (base + SBAR + 8u * (i))
   TileStream ts(p, k);
   uint32_t g = 0;
-  while (true) {
-    const TileInfo ti = ts.take(p);
-    if (!ti.valid) break;
+  TileInfo ti = ts.take(p);
+  StagePlan sp;
+  if (ti.valid) sp = plan_stage<SC>(p, item_b(p, ti.item), ti.j, ti.nvis, static_cast<int>(c));
+  while (ti.valid) {
     const uint32_t st = g & 1;
     if (!wait_bar(BAR(B_RING_EMPTY + st), ((g >> 1) & 1) ^ 1, abort, p.status, peer_abort, p.wait_limit_ns)) break;
     MLA_TRACE_EV(g, 24);
-    issue_stage<SC, SC>(p, base + SRING + st * RING_STAGE, BAR(B_RING_FULL + st), base + S_MASK + 8 * st,
-                        item_b(p, ti.item), ti.j, ti.nvis, static_cast<int>(c));
+    issue_planned<SC, SC>(p, base + SRING + st * RING_STAGE, BAR(B_RING_FULL + st), base + S_MASK + 8 * st, sp);
     MLA_TRACE_EV(g, 25);
     ++g;
+    // the next tile's page runs (table reads) while stage g % 2 is being read
+    ti = ts.take(p);
+    if (ti.valid) sp = plan_stage<SC>(p, item_b(p, ti.item), ti.j, ti.nvis, static_cast<int>(c));
   }
   for (uint32_t gd = (g >= 2 ? g - 2 : 0); gd < g; ++gd)
     drain_bar(BAR(B_RING_FULL + (gd & 1)), (gd >> 1) & 1, p.wait_limit_ns);
