@@ -587,6 +587,12 @@ __device__ __forceinline__ void issue_planned(const DecodeParams& p, uint32_t st
   if (sp.bad) raise_status(p.status, STATUS_BOUNDS);
   ptx::st_shared_u32(mask_addr, run_mask(own));
   ptx::st_shared_u32(mask_addr + 4, OTHER ? run_mask(oth) : 0u);
+  // The stage was last read by the converters' ordinary shared loads, which the empty-barrier
+  // wait orders before this thread's later generic accesses but not before the bulk copies (async
+  // proxy) that overwrite it: the proxy fence closes that write-after-read.  Without it a copy
+  // issued right after the wait overwrote rows that a converter load had not yet read (seen as
+  // run-to-run differences once the page-table reads no longer stood between the two).
+  ptx::fence_proxy_async_smem();
   ptx::mbar_arrive_expect_tx(full, tx);
   if (own.ok0) {
     ptx::bulk_load(stage, p.blocks + static_cast<size_t>(own.v0) * HEAD_DIM, static_cast<uint32_t>(own.len0) * HEAD_DIM, full);
