@@ -135,13 +135,14 @@ enum Bar : uint32_t {
   B_Q_LOCAL = 14,     // both CTAs: transaction barrier of this CTA's Q tile load
   B_O_FREE = 15,      // CTA 0: 8 warp arrivals after each CTA's epilogue
   B_DRAIN = 16,       // CTA 0: one commit from each issuer at exit
-  B_RED = 17,         // [2] softmax warps of this CTA: row-max exchange of a tile (4 warp arrivals)
-  B_REDL = 19,        // softmax warps of this CTA: row-sum exchange at a unit's end (4 warp arrivals)
-  B_EXIT = 20,        // both CTAs: the peer has finished (1 remote arrival)
-  B_RING_FULL = 21,   // [2] this CTA: the producer's expect_tx arrival + the stage's bulk-copy bytes
-  B_RING_EMPTY = 23,  // [2] this CTA: 12 converter-warp arrivals, the stage has been read
-  B_SC_FULL = 25,     // [8] scale-folding mode: 12 converter-warp arrivals, a tile's scales are in SSC
-  NUM_BARS = 33
+  B_RED = 17,         // [2][2] softmax warps of this CTA, by tile parity and warp pair (warps q and q + 2
+                      // hold the two halves of the same head rows): row-max exchange (2 warp arrivals)
+  B_REDL = 21,        // [2] by warp pair: row-sum exchange at a unit's end (2 warp arrivals)
+  B_EXIT = 23,        // both CTAs: the peer has finished (1 remote arrival)
+  B_RING_FULL = 24,   // [2] this CTA: the producer's expect_tx arrival + the stage's bulk-copy bytes
+  B_RING_EMPTY = 26,  // [2] this CTA: 12 converter-warp arrivals, the stage has been read
+  B_SC_FULL = 28,     // [8] scale-folding mode: 12 converter-warp arrivals, a tile's scales are in SSC
+  NUM_BARS = 36
 };
 static_assert(8 * NUM_BARS <= 480, "barrier block overlaps the scalars after it");
 constexpr uint32_t S_MASK = SBAR + 480;      // [2][2] u32: per ring stage, own rows copied, other scales copied
@@ -1066,7 +1067,9 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) mla_decode_kernel(const __grid
       ptx::mbar_init(BAR(B_S_FULL + i), 1);
       ptx::mbar_init(BAR(B_S_FREE + i), 8);
       ptx::mbar_init(BAR(B_P_FULL + i), 8);
-      ptx::mbar_init(BAR(B_RED + i), 4);
+      ptx::mbar_init(BAR(B_RED + 2 * i), 2);
+      ptx::mbar_init(BAR(B_RED + 2 * i + 1), 2);
+      ptx::mbar_init(BAR(B_REDL + i), 2);
       ptx::mbar_init(BAR(B_RING_FULL + i), 1);
       ptx::mbar_init(BAR(B_RING_EMPTY + i), CONV_WARPS);
     }
@@ -1075,7 +1078,6 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) mla_decode_kernel(const __grid
     ptx::mbar_init(BAR(B_Q_LOCAL), 1);
     ptx::mbar_init(BAR(B_O_FREE), 8);
     ptx::mbar_init(BAR(B_DRAIN), 2);
-    ptx::mbar_init(BAR(B_REDL), 4);
     ptx::mbar_init(BAR(B_EXIT), 1);
     for (uint32_t i = 0; i < SSC_SLOTS; ++i) ptx::mbar_init(BAR(B_SC_FULL + i), CONV_WARPS);
     *abort = 0u;
@@ -1178,8 +1180,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) mla_decode_kernel(const __grid
         // the other half of this head row lives in lane t ^ 64 (another warp of this warpgroup)
         red_max[sb * 128 + t] = mt;
         __syncwarp();
-        if (lane == 0) ptx::mbar_arrive(BAR(B_RED + sb));
-        MLA_WAIT_WARP(BAR(B_RED + sb), (g >> 1) & 1);
+        if (lane == 0) ptx::mbar_arrive(BAR(B_RED + 2 * sb + (quad & 1)));
+        MLA_WAIT_WARP(BAR(B_RED + 2 * sb + (quad & 1)), (g >> 1) & 1);
         mt = fmaxf(mt, red_max[sb * 128 + (t ^ 64)]);
         if (t == 0) MLA_TRACE_EV(g, 10);
         float alpha = 1.f;
@@ -1295,8 +1297,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) mla_decode_kernel(const __grid
         ptx::tc_fence_after();
         red_l[t] = l;
         __syncwarp();
-        if (lane == 0) ptx::mbar_arrive(BAR(B_REDL));
-        MLA_WAIT_WARP(BAR(B_REDL), uu & 1);
+        if (lane == 0) ptx::mbar_arrive(BAR(B_REDL + (quad & 1)));
+        MLA_WAIT_WARP(BAR(B_REDL + (quad & 1)), uu & 1);
         const float l_row = l + red_l[t ^ 64];
         const float inv_l = F8 ? exp2i(-sig) / l_row : 1.f / l_row;
         const int head = u.g * MROWS + HPC * static_cast<int>(c) + r;
