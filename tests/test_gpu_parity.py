@@ -1,6 +1,6 @@
 """GPU parity: the CUDA path (through the C ABI) against the float64 oracle.
 
-Tolerances (stated by the task for this method): per element
+Tolerances of the method: per element
 |out - ref| <= 2e-2 * max|ref| + 1e-2, and |lse - ref| <= 1e-3.  The dequantised
 bf16 tiles must be bit-exact.  Page permutation and scale id space must not
 change the GPU result at all (the reduction order depends only on logical token
