@@ -107,6 +107,8 @@ mla_status_t device_setup(int dev, int* nc_out) {
                                   cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(mla::SMEM_ALLOC_FOLD)));
     MLA_CUDA(cudaFuncSetAttribute(mla::mla_decode_kernel<mla::SCALE_FP8PV>,
                                   cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(mla::SMEM_ALLOC_FOLD)));
+    MLA_CUDA(cudaFuncSetAttribute(mla::mla_decode_kernel<mla::SCALE_BLOCKR>,
+                                  cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(mla::SMEM_ALLOC_FOLD)));
     MLA_CUDA(cudaFuncSetAttribute(mla::mla_dequant_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                   static_cast<int>(mla::DQ_SMEM_ALLOC)));
     MLA_CUDA(cudaFuncSetAttribute(mla::mla_dequant_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
@@ -125,15 +127,17 @@ mla_status_t device_setup(int dev, int* nc_out) {
     attr[0].val.clusterDim.z = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
-    int n = 0, n_bs = 0, n_fold = 0, n_f8 = 0;
+    int n = 0, n_bs = 0, n_fold = 0, n_f8 = 0, n_bsr = 0;
     MLA_CUDA(cudaOccupancyMaxActiveClusters(&n, mla::mla_decode_kernel<mla::SCALE_TOKEN>, &cfg));
     MLA_CUDA(cudaOccupancyMaxActiveClusters(&n_bs, mla::mla_decode_kernel<mla::SCALE_BLOCK>, &cfg));
     cfg.dynamicSmemBytes = mla::SMEM_ALLOC_FOLD;
     MLA_CUDA(cudaOccupancyMaxActiveClusters(&n_fold, mla::mla_decode_kernel<mla::SCALE_FOLD>, &cfg));
     MLA_CUDA(cudaOccupancyMaxActiveClusters(&n_f8, mla::mla_decode_kernel<mla::SCALE_FP8PV>, &cfg));
+    MLA_CUDA(cudaOccupancyMaxActiveClusters(&n_bsr, mla::mla_decode_kernel<mla::SCALE_BLOCKR>, &cfg));
     n = n < n_bs ? n : n_bs;
     n = n < n_fold ? n : n_fold;
     n = n < n_f8 ? n : n_f8;
+    n = n < n_bsr ? n : n_bsr;
     if (n <= 0) return fail(MLA_ERR_UNSUPPORTED, "no 2-CTA cluster of the decode kernel fits on this device");
     g_default_nc[dev] = n;
   }
@@ -283,8 +287,11 @@ mla_status_t launch_path(const mla::DecodeParams& p, int NC, const uint32_t* cac
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(2 * NC);
   cfg.blockDim = dim3(mla::NUM_THREADS);
-  const bool scales_in_smem = mode == mla::SCALE_FOLD || mode == mla::SCALE_FP8PV;
-  cfg.dynamicSmemBytes = scales_in_smem ? mla::SMEM_ALLOC_FOLD : mla::SMEM_ALLOC;
+  // block scales with g <= 9 take the kernel mode whose producer brings the own keys' block scales
+  // into shared memory with the ring stage
+  const bool block_ring = mode == mla::SCALE_TOKEN && p.SG > 1 && p.SG <= mla::BSC_MAX_G;
+  const bool big_smem = mode == mla::SCALE_FOLD || mode == mla::SCALE_FP8PV || block_ring;
+  cfg.dynamicSmemBytes = big_smem ? mla::SMEM_ALLOC_FOLD : mla::SMEM_ALLOC;
   cfg.stream = stream;
   cudaLaunchAttribute attr[2];
   attr[0].id = cudaLaunchAttributeClusterDimension;
@@ -300,6 +307,8 @@ mla_status_t launch_path(const mla::DecodeParams& p, int NC, const uint32_t* cac
     MLA_CUDA(cudaLaunchKernelEx(&cfg, mla::mla_decode_kernel<mla::SCALE_FOLD>, p));
   } else if (mode == mla::SCALE_FP8PV) {
     MLA_CUDA(cudaLaunchKernelEx(&cfg, mla::mla_decode_kernel<mla::SCALE_FP8PV>, p));
+  } else if (block_ring) {
+    MLA_CUDA(cudaLaunchKernelEx(&cfg, mla::mla_decode_kernel<mla::SCALE_BLOCKR>, p));
   } else if (p.SG > 1) {
     MLA_CUDA(cudaLaunchKernelEx(&cfg, mla::mla_decode_kernel<mla::SCALE_BLOCK>, p));
   } else {

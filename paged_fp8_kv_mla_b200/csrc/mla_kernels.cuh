@@ -113,14 +113,22 @@ static_assert(2 * SV8_STRIDE <= SV_BYTES, "FP8 V buffers do not fit the V buffer
 // its reference maximum within 2 (log2 units) of the running maximum, so p <= 4 and every weight
 // p * s * 2^sigma <= 448.
 constexpr float FP8_PV_LAZY_LOG2 = 2.f;
+// Block-scale mode with g <= 9 only (SCALE_BLOCKR): per ring stage the g scales of each of the 32
+// own keys (32 x g fp32, row r at 4 g r), after SMEM_USED like the scale-folding arrays (which this
+// mode does not use), inside the larger allocation.
+constexpr uint32_t SBSC = SMEM_USED;
+constexpr int BSC_MAX_G = 9;
+constexpr uint32_t BSC_STRIDE = HALF_BN * BSC_MAX_G * 4;
+static_assert(SBSC + 2 * BSC_STRIDE + 1023 <= SMEM_ALLOC_FOLD, "block-scale stages do not fit");
 
 // How the per-token scale enters the computation.
 enum ScaleMode : int {
   SCALE_TOKEN = 0,   // K, V = bf16_rn(f32_rn(e4m3 * s_t)), one scale per token
   SCALE_BLOCK = 1,   // the same with g scales per token, each over 576 / g contiguous dims
   SCALE_FOLD = 2,    // K, V = exact e4m3 values; s_t scales score column t and weight column t
-  SCALE_FP8PV = 3    // K as SCALE_TOKEN; P.V in e4m3: V = raw e4m3 bytes, s_t (and 2^sigma) carried by
+  SCALE_FP8PV = 3,   // K as SCALE_TOKEN; P.V in e4m3: V = raw e4m3 bytes, s_t (and 2^sigma) carried by
                      // the weights, each weight split into two e4m3 terms
+  SCALE_BLOCKR = 4   // SCALE_BLOCK for g <= 9: the own keys' block scales come through the ring (SBSC)
 };
 
 enum Bar : uint32_t {
@@ -575,9 +583,13 @@ __device__ __forceinline__ StagePlan plan_stage(const DecodeParams& p, int b, in
 // per-token scales (SC), their scales at RING_ROWS; with OTHER also the other keys' scales at
 // RING_OSC.  Writes the masks of copied rows and copied other-key scales to mask_addr and
 // mask_addr + 4, then arrives on `full` with the byte count and issues the bulk copies.
-template <bool SC, bool OTHER>
+// BSC (block-scale mode, g <= 9): also the own keys' g block scales per key, row r at
+// bsc + 4 g r, one bulk copy per run rounded up to 16 bytes (the rounding stays inside the page:
+// runs start at multiples of 16 slots, and a run that ends at the page's end needs none, since a
+// page holds a multiple of 16 g scales).
+template <bool SC, bool OTHER, bool BSC = false>
 __device__ __forceinline__ void issue_planned(const DecodeParams& p, uint32_t stage, uint32_t full, uint32_t mask_addr,
-                                              const StagePlan& sp) {
+                                              const StagePlan& sp, uint32_t bsc = 0) {
   const Runs& own = sp.own;
   const Runs& oth = sp.oth;
   uint32_t tx = 0;
@@ -585,6 +597,9 @@ __device__ __forceinline__ void issue_planned(const DecodeParams& p, uint32_t st
   if (own.ok1) tx += static_cast<uint32_t>(own.len1) * HEAD_DIM + (SC ? scale_bytes(own.len1) : 0u);
   if (OTHER && oth.ok0) tx += scale_bytes(oth.len0);
   if (OTHER && oth.ok1) tx += scale_bytes(oth.len1);
+  const uint32_t sg4 = 4u * static_cast<uint32_t>(p.SG);
+  if (BSC && own.ok0) tx += (static_cast<uint32_t>(own.len0) * sg4 + 15u) & ~15u;
+  if (BSC && own.ok1) tx += (static_cast<uint32_t>(own.len1) * sg4 + 15u) & ~15u;
   if (sp.bad) raise_status(p.status, STATUS_BOUNDS);
   ptx::st_shared_u32(mask_addr, run_mask(own));
   ptx::st_shared_u32(mask_addr + 4, OTHER ? run_mask(oth) : 0u);
@@ -608,6 +623,11 @@ __device__ __forceinline__ void issue_planned(const DecodeParams& p, uint32_t st
   if (OTHER && oth.ok0) ptx::bulk_load(stage + RING_OSC, p.scales + oth.s0, scale_bytes(oth.len0), full);
   if (OTHER && oth.ok1)
     ptx::bulk_load(stage + RING_OSC + 4u * static_cast<uint32_t>(oth.len0), p.scales + oth.s1, scale_bytes(oth.len1), full);
+  if (BSC && own.ok0)
+    ptx::bulk_load(bsc, p.scales + static_cast<size_t>(own.s0) * p.SG, (static_cast<uint32_t>(own.len0) * sg4 + 15u) & ~15u, full);
+  if (BSC && own.ok1)
+    ptx::bulk_load(bsc + static_cast<uint32_t>(own.len0) * sg4, p.scales + static_cast<size_t>(own.s1) * p.SG,
+                   (static_cast<uint32_t>(own.len1) * sg4 + 15u) & ~15u, full);
 }
 
 template <bool SC, bool OTHER>
@@ -731,7 +751,8 @@ __device__ __forceinline__ void copy_dc_chunks(int grp, int r, int cq, int c, ui
 template <int MODE>
 __device__ __forceinline__ void converter_role(const DecodeParams& p, int k, uint32_t base, int lane,
                                                volatile uint32_t* abort, uint32_t peer_abort, uint32_t c) {
-  constexpr bool BS = MODE == SCALE_BLOCK;
+  constexpr bool BSR = MODE == SCALE_BLOCKR;         // own block scales from the ring's side area
+  constexpr bool BS = MODE == SCALE_BLOCK || BSR;
   constexpr bool FOLD = MODE == SCALE_FOLD;
   const int C = static_cast<int>(c);
   const int t = threadIdx.x;
@@ -753,7 +774,7 @@ __device__ __forceinline__ void converter_role(const DecodeParams& p, int k, uin
   Ahead A;                       // the other key's chunks of the tile whose V operand is written next
   A.oth_ok = false;
   A.own_ok = true;
-  if (BS && !fetch_own_scales(p, kt, C, grp, r, cq, A)) raise_status(p.status, STATUS_BOUNDS);
+  if (BS && !BSR && !fetch_own_scales(p, kt, C, grp, r, cq, A)) raise_status(p.status, STATUS_BOUNDS);
   float s_oth_v = 0.f;           // per-token scale of that key (from the ring)
   uint32_t g = 0;
   // Rolled loop (one copy of the step keeps the hot code small).
@@ -772,6 +793,12 @@ __device__ __forceinline__ void converter_role(const DecodeParams& p, int k, uin
       for (int m = 0; m < 3; ++m) raw[m] = ptx::ld_shared_v4(stage + r * HEAD_DIM + 16 * (4 * (3 * grp + m) + cq));
       const float s_own = BS ? 0.f : ptx::ld_shared_f32(stage + RING_ROWS + 4 * r);
       if (!BS) s_oth_k = ptx::ld_shared_f32(stage + RING_OSC + 4 * r);
+      if (BSR) {
+        // the block scales of the thread's three chunks of its own key, from the stage's side area
+        const uint32_t bsc = base + SBSC + st * BSC_STRIDE + 4u * static_cast<uint32_t>(r * p.SG);
+#pragma unroll
+        for (int m = 0; m < 3; ++m) A.s_own[m] = ptx::ld_shared_f32(bsc + 4u * p.divCPB.div(4 * (3 * grp + m) + cq));
+      }
       if (FOLD) {
         // the tile's 64 per-token scales for the softmax (0 for keys not read).  Slot g % 8 last
         // held tile g - 8, which the softmax finished before S_FREE(g - 5), which Q.K^T(g - 3)
@@ -825,7 +852,7 @@ __device__ __forceinline__ void converter_role(const DecodeParams& p, int k, uin
     if (!fetch_oth<BS>(p, L, C, grp, cq, extra, A)) raise_status(p.status, STATUS_BOUNDS);
     if (nt.valid) {
       L = oth_lut_issue(p, nt, C, r);
-      if (BS && !fetch_own_scales(p, nt, C, grp, r, cq, A)) raise_status(p.status, STATUS_BOUNDS);
+      if (BS && !BSR && !fetch_own_scales(p, nt, C, grp, r, cq, A)) raise_status(p.status, STATUS_BOUNDS);
     }
     if (t == 0) MLA_TRACE_EV(g, 7);
     kt = nt;
@@ -1006,7 +1033,7 @@ __device__ __forceinline__ void converter_role_fp8pv(const DecodeParams& p, int 
 template <int MODE>
 __device__ __forceinline__ void producer_role(const DecodeParams& p, int k, uint32_t base, volatile uint32_t* abort,
                                               uint32_t peer_abort, uint32_t c) {
-  constexpr bool SC = MODE != SCALE_BLOCK;
+  constexpr bool SC = MODE != SCALE_BLOCK && MODE != SCALE_BLOCKR;
 #define BAR(i) (base + SBAR + 8u * (i))
   TileStream ts(p, k);
   uint32_t g = 0;
@@ -1017,7 +1044,11 @@ __device__ __forceinline__ void producer_role(const DecodeParams& p, int k, uint
     const uint32_t st = g & 1;
     if (!wait_bar(BAR(B_RING_EMPTY + st), ((g >> 1) & 1) ^ 1, abort, p.status, peer_abort, p.wait_limit_ns)) break;
     MLA_TRACE_EV(g, 24);
-    issue_planned<SC, SC>(p, base + SRING + st * RING_STAGE, BAR(B_RING_FULL + st), base + S_MASK + 8 * st, sp);
+    if (MODE == SCALE_BLOCKR)
+      issue_planned<false, false, true>(p, base + SRING + st * RING_STAGE, BAR(B_RING_FULL + st), base + S_MASK + 8 * st,
+                                        sp, base + SBSC + st * BSC_STRIDE);
+    else
+      issue_planned<SC, SC>(p, base + SRING + st * RING_STAGE, BAR(B_RING_FULL + st), base + S_MASK + 8 * st, sp);
     MLA_TRACE_EV(g, 25);
     ++g;
     // the next tile's page runs (table reads) while stage g % 2 is being read

@@ -25,10 +25,11 @@ def _lib():
     yield
 
 
-@pytest.mark.parametrize("cfg_i,runs,kw", [(3, 150, {}), (1, 60, {}), (3, 100, dict(e4m3_pv=True)),
-                                           (1, 40, dict(fold_scales=True))])
-def test_repeated_calls_agree_bit_for_bit(cfg_i, runs, kw):
-    inp = W.make_inputs(W.CONFIGS[cfg_i], device="cuda")
+@pytest.mark.parametrize("cfg_i,runs,kw,g", [(3, 150, {}, 1), (1, 60, {}, 1), (3, 100, dict(e4m3_pv=True), 1),
+                                             (1, 40, dict(fold_scales=True), 1), (3, 60, {}, 9), (1, 30, {}, 36)])
+def test_repeated_calls_agree_bit_for_bit(cfg_i, runs, kw, g):
+    from dataclasses import replace
+    inp = W.make_inputs(replace(W.CONFIGS[cfg_i], scale_blocks=g), device="cuda")
     o0, l0 = M.decode_inputs(inp, **kw)
     o0, l0 = o0.clone(), l0.clone()
     bad = 0
