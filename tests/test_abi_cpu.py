@@ -188,3 +188,11 @@ def test_host_buffer_entry_validation(lib):
     assert "one scale per token" in lib.mla_last_error_string().decode()
     assert host(_shape(batch=0)) == 0
     assert host(_shape(batch=0), variant=2, chunks=16) == 0
+
+
+def test_binding_rejects_two_variants_at_once():
+    """fold_scales and e4m3_pv select different kernels; asking for both is an argument error that
+    the binding raises before touching any tensor."""
+    import paged_fp8_kv_mla_b200 as M
+    with pytest.raises(ValueError, match="at most one"):
+        M.decode(None, None, None, None, None, None, 1, 64, 0, 0.07, fold_scales=True, e4m3_pv=True)

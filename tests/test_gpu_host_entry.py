@@ -130,3 +130,11 @@ def test_device_tensors_are_rejected():
     with pytest.raises(ValueError):
         M.decode_host(inp.q, inp.blocks, inp.scales, inp.cache_lengths.cpu(), inp.lookup_table.cpu(), None,
                       inp.max_prompt_length, inp.max_cache_length, inp.layer_idx, inp.softmax_scale, out)
+
+
+def test_block_scales_through_the_host_entry():
+    from dataclasses import replace
+    inp = W.make_inputs(replace(W.CONFIGS[1], scale_blocks=9), device="cuda")
+    o1, l1 = run_host(inp, chunks=2)
+    o2, l2 = device_by_groups(inp, 2)
+    assert torch.equal(o1, o2) and torch.equal(l1, l2)

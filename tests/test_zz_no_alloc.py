@@ -97,3 +97,19 @@ def test_noalloc_captured_in_a_cuda_graph_replays_with_new_inputs():
         torch.cuda.synchronize()
         assert torch.equal(out, ref_out) and torch.equal(lse, ref_lse)
     del graph
+
+
+@pytest.mark.parametrize("g", [9, 36])
+def test_noalloc_block_scales_match_regular_entry(g):
+    """Block scales take two kernel modes (g <= 9 through the ring, larger g by per-thread loads);
+    the no-allocation entry must pick the same one and agree bit for bit."""
+    from dataclasses import replace
+    inp = W.make_inputs(replace(W.CONFIGS[1], scale_blocks=g), device="cuda")
+    out_ref, lse_ref = M.decode_inputs(inp)
+    out = torch.full_like(out_ref, float("nan"))
+    lse = torch.full_like(lse_ref, float("nan"))
+    _lib.decode_noalloc(inp.q, inp.blocks, inp.scales, inp.cache_lengths, inp.lookup_table, inp.scales_lookup_table,
+                        inp.max_prompt_length, inp.max_cache_length, inp.layer_idx, inp.softmax_scale, out, lse)
+    torch.cuda.synchronize()
+    assert M.device_status() == 0
+    assert torch.equal(out, out_ref) and torch.equal(lse, lse_ref)
